@@ -1,0 +1,202 @@
+"""Seeded synthetic inputs shaped like the long-context workloads of LoD attention.
+
+This module holds no LoD arithmetic: it only draws keys, values and queries.
+It is the one piece shared by the CUDA path's tests and benchmark and by the
+CPU oracle's tests, so both see identical numbers.
+
+Recipe (one independent PCG64 stream per (workload, batch entry, KV head)):
+  * centres mu_j: Gaussian vectors normalised to unit length;
+  * key at position t: mu_z + sigma * N(0, I), z uniform over the centres;
+  * optional outlier channels: a few seeded channels get +/- magnitude added;
+  * optional RoPE (rotate-half pairing (i, i + d/2), inverse frequency
+    theta^(-2i/d)) applied to each key at its position, after the outliers;
+  * values N(0, 1); queries N(0, 1) / 8;
+  * zero-variance variant: every 256-token chunk draws `clusters` (key, value)
+    pairs and each position of the chunk copies one of them, so every k-means
+    group holds identical keys and values.
+Keys, values and queries are drawn in float32 and then rounded to the cache
+dtype (bfloat16, round-to-nearest-even, via torch) where the workload says so.
+"""
+from __future__ import annotations
+
+import zlib
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    T: int
+    dtype: str                 # "f32" or "bf16": the KV-cache dtype
+    n_centers: int
+    sigma: float = 0.3
+    rope_theta: float = 0.0    # 0: no RoPE
+    n_outliers: int = 0
+    outlier_mag: float = 8.0
+    clusters: tuple = (4,)
+    iters: int = 8
+    top_groups: int = 8
+    top_pages: int = 2
+    window: int = 256
+    sinks: int = 1
+    seed: int = 0
+    zero_variance: bool = False
+    mode: str = "decode"       # decode | prefill | build
+    chunk: int = 256
+    page: int = 16
+    note: str = ""
+
+    @property
+    def g(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+# The five workloads of the method's measurement plan, named by what they are.
+WORKLOADS = {
+    "decode_tiny_f32": Workload(
+        "decode_tiny_f32", B=1, Hq=1, Hkv=1, d=64, T=4096, dtype="f32", n_centers=64,
+        window=256, sinks=1, note="tiny single-head decode, fp32"),
+    "decode_tiny_f32_zero_variance": Workload(
+        "decode_tiny_f32_zero_variance", B=1, Hq=1, Hkv=1, d=64, T=4096, dtype="f32",
+        n_centers=64, window=256, sinks=1, zero_variance=True,
+        note="tiny decode with zero-variance groups: LoD equals dense attention"),
+    "decode_gqa_32k_bf16": Workload(
+        "decode_gqa_32k_bf16", B=8, Hq=64, Hkv=8, d=128, T=32768, dtype="bf16",
+        n_centers=512, rope_theta=1e6, n_outliers=4, window=512, sinks=4,
+        note="GQA decode at 32K"),
+    "decode_gqa_128k_bf16": Workload(
+        "decode_gqa_128k_bf16", B=4, Hq=64, Hkv=8, d=128, T=131072, dtype="bf16",
+        n_centers=512, rope_theta=1e6, n_outliers=4, window=512, sinks=4,
+        note="GQA decode at 128K (decode headline)"),
+    "prefill_128k_bf16": Workload(
+        "prefill_128k_bf16", B=1, Hq=32, Hkv=8, d=128, T=131072, dtype="bf16",
+        n_centers=512, rope_theta=1e6, window=512, sinks=4, mode="prefill",
+        note="chunked causal prefill at 128K"),
+    "build_128k_bf16": Workload(
+        "build_128k_bf16", B=1, Hq=8, Hkv=8, d=128, T=131072, dtype="bf16",
+        n_centers=2048, rope_theta=1e6, clusters=(4, 8), window=512, sinks=4, mode="build",
+        note="index build at 128K, k=4 and k=8"),
+}
+
+
+def _unit_rng(w: Workload, b: int, kvh: int, stream: str) -> np.random.Generator:
+    tag = zlib.crc32(w.name.replace("_zero_variance", "").encode())
+    s2 = zlib.crc32(stream.encode())
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, tag, b, kvh, s2])))
+
+
+def _rope(x: np.ndarray, theta: float, pos0: int = 0) -> np.ndarray:
+    T, d = x.shape
+    h = d // 2
+    inv = theta ** (-2.0 * np.arange(h, dtype=np.float64) / d)
+    ang = (np.arange(pos0, pos0 + T, dtype=np.float64)[:, None] * inv[None, :])
+    c = np.cos(ang).astype(np.float32)
+    s = np.sin(ang).astype(np.float32)
+    x1, x2 = x[:, :h], x[:, h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)
+
+
+def _mixture_keys(w: Workload, rng: np.random.Generator, T: int) -> np.ndarray:
+    cen = rng.standard_normal((w.n_centers, w.d), dtype=np.float32)
+    cen /= np.linalg.norm(cen, axis=1, keepdims=True)
+    z = rng.integers(0, w.n_centers, size=T)
+    k = cen[z] + np.float32(w.sigma) * rng.standard_normal((T, w.d), dtype=np.float32)
+    return k
+
+
+def unit_kv(w: Workload, b: int, kvh: int, T: int | None = None):
+    """Keys and values of one (batch entry, KV head): float32 [T, d] arrays
+    holding cache-dtype values (already rounded to bf16 where needed)."""
+    T = w.T if T is None else T
+    rk = _unit_rng(w, b, kvh, "keys")
+    rv = _unit_rng(w, b, kvh, "values")
+    if w.zero_variance:
+        nch = (T + w.chunk - 1) // w.chunk
+        npair = w.clusters[0]
+        pk = _mixture_keys(w, rk, nch * npair).reshape(nch, npair, w.d)
+        pv = rv.standard_normal((nch, npair, w.d), dtype=np.float32)
+        pick = rk.integers(0, npair, size=(nch, w.chunk))
+        K = np.take_along_axis(pk, pick[:, :, None], axis=1).reshape(-1, w.d)[:T]
+        V = np.take_along_axis(pv, pick[:, :, None], axis=1).reshape(-1, w.d)[:T]
+        K = np.ascontiguousarray(K)
+        V = np.ascontiguousarray(V)
+    else:
+        K = _mixture_keys(w, rk, T)
+        if w.n_outliers:
+            ro = _unit_rng(w, b, kvh, "outliers")
+            ch = ro.choice(w.d, size=w.n_outliers, replace=False)
+            sg = ro.choice(np.array([-1.0, 1.0], dtype=np.float32), size=w.n_outliers)
+            K[:, ch] += np.float32(w.outlier_mag) * sg
+        if w.rope_theta:
+            K = _rope(K, w.rope_theta)
+        V = rv.standard_normal((T, w.d), dtype=np.float32)
+    return to_cache_values(w, K), to_cache_values(w, V)
+
+
+def unit_queries(w: Workload, b: int, kvh: int, n_pos: int = 1, stream: str = "queries"):
+    """Queries of the g query heads of one KV head: float32 [g, n_pos, d]
+    (cache-dtype values), N(0, 1) / 8."""
+    r = _unit_rng(w, b, kvh, stream)
+    q = r.standard_normal((w.g, n_pos, w.d), dtype=np.float32) / np.float32(8.0)
+    return to_cache_values(w, q)
+
+
+def to_cache_values(w: Workload, a: np.ndarray) -> np.ndarray:
+    if w.dtype == "f32":
+        return np.ascontiguousarray(a, dtype=np.float32)
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.to(torch.float32).numpy()
+
+
+def kv_cache(w: Workload, T: int | None = None, threads: int = 8):
+    """The whole KV cache as torch CPU tensors [B, Hkv, T, d] in the cache dtype."""
+    T = w.T if T is None else T
+    K = torch.empty((w.B, w.Hkv, T, w.d), dtype=w.torch_dtype)
+    V = torch.empty_like(K)
+
+    def fill(u):
+        b, h = divmod(u, w.Hkv)
+        k, v = unit_kv(w, b, h, T)
+        K[b, h] = torch.from_numpy(k).to(w.torch_dtype)
+        V[b, h] = torch.from_numpy(v).to(w.torch_dtype)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(fill, range(w.B * w.Hkv)))
+    return K, V
+
+
+def decode_queries(w: Workload, stream: str = "queries"):
+    """Decode queries as a torch CPU tensor [B, Hq, d] in the cache dtype."""
+    q = torch.empty((w.B, w.Hq, w.d), dtype=w.torch_dtype)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            q[b, h * w.g:(h + 1) * w.g] = torch.from_numpy(
+                unit_queries(w, b, h, 1, stream)[:, 0]).to(w.torch_dtype)
+    return q
+
+
+def prefill_queries(w: Workload, q_begin: int, Tq: int, stream: str = "queries"):
+    """Prefill queries [B, Hq, Tq, d] (torch CPU, cache dtype) for positions
+    [q_begin, q_begin + Tq).  Drawn per position block so any window of
+    positions is reproducible on its own."""
+    q = torch.empty((w.B, w.Hq, Tq, w.d), dtype=w.torch_dtype)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            q[b, h * w.g:(h + 1) * w.g] = torch.from_numpy(
+                unit_queries(w, b, h, q_begin + Tq, stream)[:, q_begin:]).to(w.torch_dtype)
+    return q
