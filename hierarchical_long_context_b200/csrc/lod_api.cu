@@ -1,0 +1,351 @@
+// lod_api.cu -- the extern "C" entry points declared in include/lod.h:
+// argument validation, index and workspace sizing, and kernel launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "lod_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int32_t fail(int32_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int32_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(LOD_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t elem_bytes(const lod_params* p) { return p->dtype == LOD_DTYPE_F32 ? 4 : 2; }
+int32_t page_slots(const lod_params* p) { return p->chunk / p->page + p->clusters; }
+int32_t g_of(const lod_params* p) { return p->Hq / p->Hkv; }
+int kg_of(const lod_params* p) { return p->top_groups <= 8 ? 8 : 16; }
+int nq_max(const lod_params* p) { return p->d == 64 ? 16 : 8; }
+
+int32_t validate(const lod_params* p) {
+  if (!p) return fail(LOD_EINVAL, "params is NULL");
+  if (p->reserved0 != 0 || p->reserved1 != 0) return fail(LOD_EINVAL, "reserved fields must be 0");
+  if (p->dtype != LOD_DTYPE_F32 && p->dtype != LOD_DTYPE_BF16)
+    return fail(LOD_EUNSUPPORTED, "dtype %d unsupported (0=f32, 1=bf16)", p->dtype);
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1) return fail(LOD_EINVAL, "B, Hq, Hkv must be >= 1");
+  if (p->Hq % p->Hkv) return fail(LOD_EINVAL, "Hq (%d) must be a multiple of Hkv (%d)", p->Hq, p->Hkv);
+  const int g = g_of(p);
+  if (g & (g - 1)) return fail(LOD_EUNSUPPORTED, "Hq/Hkv = %d must be a power of two", g);
+  if (p->d != 64 && p->d != 128) return fail(LOD_EUNSUPPORTED, "d = %d unsupported (64 or 128)", p->d);
+  if (g > nq_max(p))
+    return fail(LOD_EUNSUPPORTED, "Hq/Hkv = %d exceeds %d at d = %d", g, nq_max(p), p->d);
+  if (p->chunk != lod::kChunk) return fail(LOD_EUNSUPPORTED, "chunk must be %d", lod::kChunk);
+  if (p->page != lod::kPage) return fail(LOD_EUNSUPPORTED, "page must be %d", lod::kPage);
+  if (p->clusters < 1 || p->clusters > lod::kMaxClusters)
+    return fail(LOD_EUNSUPPORTED, "clusters must be in [1, %d]", lod::kMaxClusters);
+  if (p->kmeans_iters < 1 || p->kmeans_iters > 64)
+    return fail(LOD_EUNSUPPORTED, "kmeans_iters must be in [1, 64]");
+  if (p->top_groups < 1 || p->top_groups > lod::kMaxTopGroups)
+    return fail(LOD_EUNSUPPORTED, "top_groups must be in [1, %d]", lod::kMaxTopGroups);
+  if (p->top_pages < 1 || p->top_pages > lod::kMaxTopPages)
+    return fail(LOD_EUNSUPPORTED, "top_pages must be in [1, %d]", lod::kMaxTopPages);
+  if (p->window < p->chunk || p->window % p->chunk)
+    return fail(LOD_EINVAL, "window (%d) must be a positive multiple of chunk", p->window);
+  if (p->sinks < 0 || p->sinks >= p->chunk) return fail(LOD_EINVAL, "sinks must be in [0, chunk)");
+  if (p->Tmax < p->chunk || p->Tmax % p->chunk)
+    return fail(LOD_EINVAL, "Tmax must be a positive multiple of chunk");
+  if (p->Tmax / p->chunk * (int64_t)p->clusters > (int64_t)1 << 30)
+    return fail(LOD_EUNSUPPORTED, "Tmax too large");
+  return LOD_OK;
+}
+
+int32_t validate_kv(const lod_params* p, const void* K, const void* V, const int64_t* s) {
+  if (!K || !V || !s) return fail(LOD_EINVAL, "K, V and kv_strides must be non-NULL");
+  if (!aligned16(K) || !aligned16(V)) return fail(LOD_EINVAL, "K and V must be 16-byte aligned");
+  const int64_t e = elem_bytes(p);
+  for (int i = 0; i < 3; ++i)
+    if (s[i] < 0 || (s[i] * e) % 16) return fail(LOD_EINVAL, "kv stride %d must be a non-negative multiple of 16 bytes", i);
+  if (s[2] < p->d) return fail(LOD_EINVAL, "token stride smaller than d");
+  return LOD_OK;
+}
+
+int32_t validate_index(const lod_index* ix) {
+  if (!ix) return fail(LOD_EINVAL, "index is NULL");
+  const void* ptrs[9] = {ix->gK, ix->gV, ix->gCnt, ix->pK, ix->pV, ix->pCnt, ix->pBeg, ix->gPage, ix->perm};
+  for (int i = 0; i < 9; ++i) {
+    if (!ptrs[i]) return fail(LOD_EINVAL, "index field %d is NULL", i);
+    if (i == 0 || i == 1 || i == 3 || i == 4) {
+      if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index summary %d must be 16-byte aligned", i);
+    } else if (reinterpret_cast<uintptr_t>(ptrs[i]) & 3u && i != 6 && i != 7 && i != 8) {
+      return fail(LOD_EINVAL, "index field %d misaligned", i);
+    }
+  }
+  return LOD_OK;
+}
+
+struct AttendShape {
+  int NQ, NP, nsg, nsw;
+  int64_t units;
+};
+
+// Decode: one unit per (b, kvh); group splits cover the largest index.
+AttendShape decode_shape(const lod_params* p) {
+  AttendShape s;
+  s.NP = 1;
+  s.NQ = g_of(p);
+  s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
+  s.nsw = (int)cdiv(p->window, lod::kScanRows);
+  s.units = (int64_t)p->B * p->Hkv;
+  return s;
+}
+
+// Prefill: one launch per query chunk; NP positions per unit.
+AttendShape prefill_shape(const lod_params* p) {
+  AttendShape s;
+  s.NP = nq_max(p) / g_of(p);
+  s.NQ = s.NP * g_of(p);
+  s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
+  s.nsw = (int)cdiv(p->window, lod::kScanRows);
+  s.units = (int64_t)p->B * p->Hkv * cdiv(p->chunk, s.NP);
+  return s;
+}
+
+size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
+  const int KG = kg_of(p);
+  size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
+  size_t cand = (sizeof(float) + sizeof(int)) * (size_t)s.units * s.nsg * s.NQ * KG;
+  return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((cand + 255) & ~size_t(255));
+}
+
+void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, const void* K,
+                 const void* V, const int64_t* kv, const lod_index* ix, void* ws) {
+  memset(&a, 0, sizeof(a));
+  a.K = K;
+  a.V = V;
+  a.sb = kv[0];
+  a.sh = kv[1];
+  a.st = kv[2];
+  a.gK = ix->gK;
+  a.gV = ix->gV;
+  a.gCnt = ix->gCnt;
+  a.pK = ix->pK;
+  a.pV = ix->pV;
+  a.pCnt = ix->pCnt;
+  a.pBeg = ix->pBeg;
+  a.gPage = ix->gPage;
+  a.perm = ix->perm;
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.g = g_of(p);
+  a.Tmax = p->Tmax;
+  a.Cmax = p->Tmax / p->chunk;
+  a.k = p->clusters;
+  a.P = page_slots(p);
+  a.G = p->top_groups;
+  a.TP = p->top_pages;
+  a.window = p->window;
+  a.sinks = p->sinks;
+  a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+  a.NP = s.NP;
+  a.nsg = s.nsg;
+  a.nsw = s.nsw;
+  a.units = s.units;
+  char* w = static_cast<char*>(ws);
+  a.status = reinterpret_cast<uint32_t*>(w);
+  const int KG = kg_of(p);
+  size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
+  part = (part + 255) & ~size_t(255);
+  a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
+  a.cand_s = reinterpret_cast<float*>(w + lod::kWsHeader + part);
+  a.cand_i = reinterpret_cast<int*>(w + lod::kWsHeader + part +
+                                     sizeof(float) * (size_t)s.units * s.nsg * s.NQ * KG);
+}
+
+int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
+                 int64_t c1, const lod_index* ix, cudaStream_t stream) {
+  lod::BuildArgs a;
+  memset(&a, 0, sizeof(a));
+  a.K = K;
+  a.V = V;
+  a.sb = kv[0];
+  a.sh = kv[1];
+  a.st = kv[2];
+  a.Hkv = p->Hkv;
+  a.Cmax = p->Tmax / p->chunk;
+  a.k = p->clusters;
+  a.iters = p->kmeans_iters;
+  a.sinks = p->sinks;
+  a.P = page_slots(p);
+  a.chunk_begin = c0;
+  a.seed = p->seed;
+  a.gK = ix->gK;
+  a.gV = ix->gV;
+  a.gCnt = ix->gCnt;
+  a.pK = ix->pK;
+  a.pV = ix->pV;
+  a.pCnt = ix->pCnt;
+  a.pBeg = ix->pBeg;
+  a.gPage = ix->gPage;
+  a.perm = ix->perm;
+  cudaError_t e = lod::launch_build(a, p->dtype, p->d, c1 - c0, p->B, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "index build launch");
+  return LOD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t lod_version(void) { return 100; }
+
+const char* lod_last_error(void) { return g_err; }
+
+int32_t lod_index_sizes(const lod_params* p, size_t bytes[9]) {
+  int32_t rc = validate(p);
+  if (rc) return rc;
+  if (!bytes) return fail(LOD_EINVAL, "bytes is NULL");
+  const size_t units = (size_t)p->B * p->Hkv, Cmax = p->Tmax / p->chunk, k = p->clusters,
+               P = page_slots(p), d = p->d, e = elem_bytes(p);
+  bytes[0] = bytes[1] = units * Cmax * k * d * e;
+  bytes[2] = units * Cmax * k * sizeof(int32_t);
+  bytes[3] = bytes[4] = units * Cmax * P * d * e;
+  bytes[5] = units * Cmax * P * sizeof(int32_t);
+  bytes[6] = units * Cmax * P * sizeof(int16_t);
+  bytes[7] = units * Cmax * (k + 1) * sizeof(int16_t);
+  bytes[8] = units * Cmax * p->chunk * sizeof(int16_t);
+  g_err[0] = 0;
+  return LOD_OK;
+}
+
+int32_t lod_workspace_bytes(const lod_params* p, int32_t op, size_t* bytes) {
+  int32_t rc = validate(p);
+  if (rc) return rc;
+  if (!bytes) return fail(LOD_EINVAL, "bytes is NULL");
+  switch (op) {
+    case LOD_OP_BUILD: *bytes = lod::kWsHeader; break;
+    case LOD_OP_DECODE: *bytes = attend_ws_bytes(p, decode_shape(p)); break;
+    case LOD_OP_PREFILL: *bytes = attend_ws_bytes(p, prefill_shape(p)); break;
+    default: return fail(LOD_EINVAL, "unknown op %d", op);
+  }
+  g_err[0] = 0;
+  return LOD_OK;
+}
+
+int32_t lod_build_index(const lod_params* p, const void* K, const void* V, const int64_t kv_strides[3],
+                        int64_t chunk_begin, int64_t chunk_end, const lod_index* index, void* ws,
+                        size_t ws_bytes, lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (!rc) rc = validate_index(index);
+  if (rc) return rc;
+  if (chunk_begin < 0 || chunk_end <= chunk_begin || chunk_end * p->chunk > p->Tmax)
+    return fail(LOD_EINVAL, "chunk range [%lld, %lld) invalid for Tmax %lld", (long long)chunk_begin,
+                (long long)chunk_end, (long long)p->Tmax);
+  if (chunk_end - chunk_begin > 0x7fffffff) return fail(LOD_EINVAL, "chunk range too large");
+  if (!ws || !aligned16(ws) || ws_bytes < lod::kWsHeader)
+    return fail(LOD_EINVAL, "workspace too small or misaligned");
+  rc = do_build(p, K, V, kv_strides, chunk_begin, chunk_end, index, (cudaStream_t)stream);
+  if (!rc) g_err[0] = 0;
+  return rc;
+}
+
+int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void* V,
+                   const int64_t kv_strides[3], const int64_t* seq_lens, const lod_index* index,
+                   void* out, float* lse, int32_t* sel_groups, int32_t* sel_pages, void* ws,
+                   size_t ws_bytes, lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (!rc) rc = validate_index(index);
+  if (rc) return rc;
+  if (!q || !out || !seq_lens) return fail(LOD_EINVAL, "q, out and seq_lens must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
+  const AttendShape s = decode_shape(p);
+  if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
+    return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
+  lod::AttendArgs a;
+  fill_attend(a, p, s, K, V, kv_strides, index, ws);
+  a.q = q;
+  a.Tq = 1;
+  a.q_begin = 0;
+  a.seq_lens = seq_lens;
+  a.pos_lo = 0;
+  a.pos_hi = 1;
+  a.out = out;
+  a.lse = lse;
+  a.sel_groups = sel_groups;
+  a.sel_pages = sel_pages;
+  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  g_err[0] = 0;
+  return LOD_OK;
+}
+
+int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t Tq, const void* K,
+                    const void* V, const int64_t kv_strides[3], const lod_index* index, void* out,
+                    float* lse, int32_t* sel_groups, int32_t* sel_pages, void* ws, size_t ws_bytes,
+                    lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (!rc) rc = validate_index(index);
+  if (rc) return rc;
+  if (!q || !out) return fail(LOD_EINVAL, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
+  if (q_begin < 0 || q_begin % p->chunk || Tq < 1 || q_begin + Tq > p->Tmax)
+    return fail(LOD_EINVAL, "query range [%lld, %lld) invalid", (long long)q_begin, (long long)(q_begin + Tq));
+  const AttendShape s = prefill_shape(p);
+  if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
+    return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
+  cudaStream_t st = (cudaStream_t)stream;
+  // 1) index of every chunk completed inside the query range (a pure function of K/V)
+  const int64_t c0 = q_begin / p->chunk, c1 = (q_begin + Tq) / p->chunk;
+  if (c1 > c0) {
+    rc = do_build(p, K, V, kv_strides, c0, c1, index, st);
+    if (rc) return rc;
+  }
+  // 2) attention, one launch pair per query chunk
+  lod::AttendArgs a;
+  fill_attend(a, p, s, K, V, kv_strides, index, ws);
+  a.q = q;
+  a.Tq = Tq;
+  a.q_begin = q_begin;
+  a.seq_lens = nullptr;
+  a.out = out;
+  a.lse = lse;
+  a.sel_groups = sel_groups;
+  a.sel_pages = sel_pages;
+  const int64_t nw = p->window / p->chunk;
+  for (int64_t lo = 0; lo < Tq; lo += p->chunk) {
+    const int64_t hi = lo + p->chunk < Tq ? lo + p->chunk : Tq;
+    const int64_t bt = (q_begin + lo) / p->chunk;
+    const int64_t wb = bt - nw + 1 > 0 ? bt - nw + 1 : 0;
+    a.pos_lo = lo;
+    a.pos_hi = hi;
+    a.nsg = (int)cdiv(wb * p->clusters, lod::kScanRows);
+    a.units = (int64_t)p->B * p->Hkv * cdiv(hi - lo, s.NP);
+    // part/cand keep the worst-case layout of fill_attend; a chunk uses a prefix
+    cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, st);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  }
+  g_err[0] = 0;
+  return LOD_OK;
+}
+
+int32_t lod_get_status(void* ws, lod_stream_t stream, uint32_t* status) {
+  if (!ws || !status) return fail(LOD_EINVAL, "ws and status must be non-NULL");
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  *status = v;
+  g_err[0] = 0;
+  return v ? LOD_EDEVICE : LOD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+// lod_common.cuh -- shared device helpers of the LoD attention kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lod.h"
+
+namespace lod {
+
+constexpr int kChunk = 256;  // tokens per indexed chunk ("How It Works", paragraph 1)
+constexpr int kPage = 16;    // keys per page (same paragraph)
+constexpr int kMaxClusters = 16;
+constexpr int kMaxTopGroups = 16;
+constexpr int kMaxTopPages = 4;
+
+// Workspace header: the device status word and padding to 256 bytes.
+constexpr size_t kWsHeader = 256;
+
+// ---------------------------------------------------------------- element I/O
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  __device__ __forceinline__ static float to_f(float x) { return x; }
+  __device__ __forceinline__ static float from_f(float x) { return x; }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  __device__ __forceinline__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  __device__ __forceinline__ static __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Load N consecutive elements (N * sizeof(T) in {4, 8, 16} bytes, naturally
+// aligned) as floats, through the read-only path.
+template <typename T, int N>
+__device__ __forceinline__ void load_f(const T* __restrict__ p, float (&v)[N]) {
+  if constexpr (sizeof(T) == 4) {
+    if constexpr (N == 4) {
+      float4 a = __ldg(reinterpret_cast<const float4*>(p));
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if constexpr (N == 2) {
+      float2 a = __ldg(reinterpret_cast<const float2*>(p));
+      v[0] = a.x; v[1] = a.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) v[i] = __ldg(reinterpret_cast<const float*>(p) + i);
+    }
+  } else {
+    static_assert(N % 2 == 0, "bf16 loads come in pairs");
+    if constexpr (N == 8) {
+      uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+      uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    } else if constexpr (N == 4) {
+      uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
+      v[0] = __uint_as_float(a.x << 16);
+      v[1] = __uint_as_float(a.x & 0xffff0000u);
+      v[2] = __uint_as_float(a.y << 16);
+      v[3] = __uint_as_float(a.y & 0xffff0000u);
+    } else {
+      static_assert(N == 2, "unsupported bf16 vector width");
+      uint32_t a = __ldg(reinterpret_cast<const unsigned int*>(p));
+      v[0] = __uint_as_float(a << 16);
+      v[1] = __uint_as_float(a & 0xffff0000u);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- warp helpers
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Candidate order used by every top-k of the method: larger score first,
+// then lower id (the tie rule of the rankings).
+__device__ __forceinline__ bool cand_better(float s, int id, float s2, int id2) {
+  return s > s2 || (s == s2 && id < id2);
+}
+
+// Warp-wide argmax of (score, -id): every lane receives the winner.
+__device__ __forceinline__ void warp_best(float& s, int& id) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    int i2 = __shfl_xor_sync(0xffffffffu, id, o);
+    if (cand_better(s2, i2, s, id)) {
+      s = s2;
+      id = i2;
+    }
+  }
+}
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+// SplitMix64 generator output for state x (Steele, Lea, Flood, OOPSLA 2014).
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+}  // namespace lod

@@ -1,0 +1,79 @@
+// lod_internal.cuh -- argument blocks and launchers shared by the library's
+// translation units (not part of the public ABI).
+#pragma once
+
+#include "lod_common.cuh"
+
+namespace lod {
+
+struct BuildArgs {
+  const void* K;
+  const void* V;
+  int64_t sb, sh, st;  // KV strides in elements (sequence, head, token)
+  int Hkv;
+  int64_t Cmax;        // index capacity in chunks
+  int k;               // clusters
+  int iters;           // Lloyd rounds
+  int sinks;
+  int P;               // page slots per chunk
+  int64_t chunk_begin;
+  uint64_t seed;
+  void* gK;
+  void* gV;
+  int32_t* gCnt;
+  void* pK;
+  void* pV;
+  int32_t* pCnt;
+  int16_t* pBeg;
+  int16_t* gPage;
+  int16_t* perm;
+};
+
+// Rows streamed by one scan CTA.
+constexpr int kScanRows = 128;
+
+// A batch of query rows handled by one scan/refine launch pair.
+//  decode:  unit = (b, kvh); the unit's NQ = g rows are its query heads, all
+//           at t = seq_lens[b] - 1.
+//  prefill: unit = (b, kvh, block of NP consecutive positions); row r of the
+//           unit is head (r % g) at position block*NP + r / g.
+struct AttendArgs {
+  const void* q;            // [B][Hq][Tq][d]
+  int64_t Tq;               // positions per sequence in q/out (1 for decode)
+  int64_t q_begin;          // position of q's first row (prefill)
+  const int64_t* seq_lens;  // decode: device [B]; prefill: null
+  int64_t pos_lo, pos_hi;   // prefill: q rows [pos_lo, pos_hi) handled by this launch
+  int NP;                   // positions per unit (1 for decode)
+  const void* K;
+  const void* V;
+  int64_t sb, sh, st;
+  const void* gK;
+  const void* gV;
+  const int32_t* gCnt;
+  const void* pK;
+  const void* pV;
+  const int32_t* pCnt;
+  const int16_t* pBeg;
+  const int16_t* gPage;
+  const int16_t* perm;
+  int B, Hq, Hkv, g;
+  int64_t Tmax, Cmax;
+  int k, P, G, TP, window, sinks;
+  float scale;
+  int nsg, nsw;             // group splits and window splits per unit
+  int64_t units;            // scan units in this launch
+  float* part;              // [units][nsg+nsw][NQ][d+2]  (m, l, acc[d])
+  float* cand_s;            // [units][nsg][NQ][G]
+  int* cand_i;              // [units][nsg][NQ][G]
+  void* out;                // [B][Hq][Tq][d]
+  float* lse;               // [B][Hq][Tq] or null
+  int32_t* sel_groups;      // [B][Hq][Tq][G] or null
+  int32_t* sel_pages;       // [B][Hq][Tq][G][TP] or null
+  uint32_t* status;
+};
+
+cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
+                         cudaStream_t stream);
+cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, cudaStream_t stream);
+
+}  // namespace lod

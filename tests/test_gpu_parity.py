@@ -1,0 +1,241 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Sizes are small enough for the oracle to finish in seconds yet span several
+scan splits, several chunks per group split, and ragged tails.  The rules
+(tolerances, tie handling, k-means margin rule) are in tests/lodtest.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hierarchical_long_context_b200 import api, synth
+from tests import lodtest as lt
+
+pytestmark = pytest.mark.gpu
+
+
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda")
+
+
+def _setup(w, k=None, T=None):
+    dev = _cuda()
+    T = T or w.T
+    Kc, Vc = synth.kv_cache(w, T)
+    p = lt.params_of(w, k, Tmax=((T + 255) // 256) * 256)
+    Kd = torch.zeros((w.B, w.Hkv, p.Tmax, w.d), dtype=w.torch_dtype, device=dev)
+    Vd = torch.zeros_like(Kd)
+    Kd[:, :, :T] = Kc.to(dev)
+    Vd[:, :, :T] = Vc.to(dev)
+    return p, Kc, Vc, Kd, Vd
+
+
+def _np(t):
+    return t.float().cpu().numpy()
+
+
+# ------------------------------------------------------------------ build
+
+@pytest.mark.parametrize("name, k, T", [
+    ("decode_tiny_f32", 4, 4096),
+    ("decode_tiny_f32_zero_variance", 4, 4096),
+    ("decode_tiny_f32_zero_variance", 8, 2048),   # more clusters than distinct keys: empty groups
+    ("decode_gqa_32k_bf16", 4, 4096),
+    ("build_128k_bf16", 8, 2048),
+])
+def test_build_matches_oracle(name, k, T):
+    w = synth.WORKLOADS[name]
+    w = w.with_(B=min(w.B, 2), Hkv=min(w.Hkv, 2), Hq=min(w.Hkv, 2) * w.g)
+    p, Kc, Vc, Kd, Vd = _setup(w, k, T)
+    ix = api.Index(p)
+    nch = T // 256
+    api.lod_build_index(p, Kd, Vd, 0, nch, ix)
+    torch.cuda.synchronize()
+    cfg = lt.oracle_cfg(w, k)
+    tot = dict(chunks=0, fragile=0, diverged=0, keys_checked=0)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            K, V = _np(Kc[b, h]), _np(Vc[b, h])
+            gu = lt.unit_from_gpu(ix, b, h, nch, p)
+            lt.check_index_consistency(gu, K, V, cfg, w.dtype == "bf16")
+            ou = oracle.build_sequence(cfg, b * w.Hkv + h, K, V, nch)
+            st = lt.compare_builds(gu, ou, cfg, w.dtype == "bf16")
+            for key in tot:
+                tot[key] += st[key]
+    print(name, k, tot)
+    assert tot["keys_checked"] > 0.9 * tot["chunks"] * 200
+    assert tot["diverged"] <= max(1, tot["chunks"] // 20)
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_rows(p, w, Kd, Vd, ix, seq_lens, draws):
+    dev = Kd.device
+    rows = []
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE)
+    for s in range(draws):
+        q = synth.decode_queries(w, stream="queries%d" % s).to(dev)
+        sl = torch.tensor(seq_lens, dtype=torch.int64, device=dev)
+        lse = torch.empty(w.B, w.Hq, dtype=torch.float32, device=dev)
+        sg = torch.empty(w.B, w.Hq, p.top_groups, dtype=torch.int32, device=dev)
+        sp = torch.empty(w.B, w.Hq, p.top_groups, p.top_pages, dtype=torch.int32, device=dev)
+        out = api.lod_decode(p, q, Kd, Vd, sl, ix, lse=lse, sel_groups=sg, sel_pages=sp, ws=ws)
+        torch.cuda.synchronize()
+        assert api.lod_get_status(ws) == 0
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                rows.append(((b, hq // w.g), _np(q[b, hq]), seq_lens[b] - 1, _np(out[b, hq]).astype(np.float64),
+                             float(lse[b, hq]), sg[b, hq].cpu().numpy(), sp[b, hq].cpu().numpy()))
+    return rows
+
+
+def _check_decode(w, p, Kc, Vc, ix, rows, cfg, use):
+    by_unit = {}
+    for r in rows:
+        by_unit.setdefault(r[0], []).append(r[1:])
+    stats = []
+    for (b, h), rr in by_unit.items():
+        K, V = _np(Kc[b, h]), _np(Vc[b, h])
+        nch = max(r[1] for r in rr) // 256 + 1
+        u = use(b, h, K, V, nch)
+        stats.append(lt.check_rows(cfg, w.dtype, K, V, u, rr))
+    return stats
+
+
+@pytest.mark.parametrize("name, T, seq_lens", [
+    ("decode_tiny_f32", 4096, [4096]),
+    ("decode_tiny_f32_zero_variance", 4096, [4096]),
+    ("decode_gqa_32k_bf16", 8192, [8192, 5000]),
+    ("decode_gqa_32k_bf16", 4096, [1, 700]),          # window covers everything: no index used
+])
+def test_decode_on_gpu_index_matches_oracle(name, T, seq_lens):
+    w = synth.WORKLOADS[name]
+    w = w.with_(B=len(seq_lens), Hkv=min(w.Hkv, 2), Hq=min(w.Hkv, 2) * w.g)
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    rows = _decode_rows(p, w, Kd, Vd, ix, seq_lens, draws=4 if w.Hq > 1 else 16)
+    cfg = lt.oracle_cfg(w)
+    st = _check_decode(w, p, Kc, Vc, ix, rows, cfg,
+                       lambda b, h, K, V, n: lt.unit_from_gpu(ix, b, h, T // 256, p))
+    print(name, st)
+
+
+def test_decode_on_oracle_index_matches_oracle():
+    """The attention kernels alone: the index is the oracle's, imported."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, Hkv=2, Hq=16)
+    T = 6144
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    cfg = lt.oracle_cfg(w)
+    ix = api.Index(p)
+    ous = {}
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            ous[(b, h)] = oracle.build_sequence(cfg, b * w.Hkv + h, _np(Kc[b, h]), _np(Vc[b, h]), T // 256)
+            lt.unit_to_gpu(ix, b, h, ous[(b, h)], p)
+    rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 300], draws=4)
+    st = _check_decode(w, p, Kc, Vc, ix, rows, cfg, lambda b, h, K, V, n: ous[(b, h)])
+    print(st)
+
+
+def test_zero_variance_decode_equals_dense():
+    """Level of Detail Attention, How It Works: zero-variance groups give full
+    attention -- checked on the GPU path directly against dense softmax."""
+    w = synth.WORKLOADS["decode_tiny_f32_zero_variance"]
+    p, Kc, Vc, Kd, Vd = _setup(w)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix)
+    cfg = lt.oracle_cfg(w)
+    K, V = _np(Kc[0, 0]), _np(Vc[0, 0])
+    for s in range(8):
+        q = synth.decode_queries(w, stream="dense%d" % s).cuda()
+        out = api.lod_decode(p, q, Kd, Vd, torch.tensor([w.T], device="cuda"), ix)
+        dout, _ = oracle.dense_row(cfg, _np(q[0, 0]), w.T - 1, K, V)
+        assert np.max(np.abs(_np(out[0, 0]) - dout)) < 1e-5
+
+
+# ------------------------------------------------------------------ prefill
+
+@pytest.mark.parametrize("name, T, split", [
+    ("prefill_128k_bf16", 2048 + 100, None),      # ragged tail, one call
+    ("prefill_128k_bf16", 2048 + 100, 1024),      # two calls: the second continues the first
+    ("decode_tiny_f32", 1536 + 37, None),
+])
+def test_prefill_matches_oracle(name, T, split):
+    w = synth.WORKLOADS[name]
+    w = w.with_(B=1, Hkv=min(w.Hkv, 2), Hq=min(w.Hkv, 2) * w.g, T=T)
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    dev = Kd.device
+    qc = synth.prefill_queries(w, 0, T)
+    q = qc.to(dev)
+    ix = api.Index(p)
+    lse = torch.empty(w.B, w.Hq, T, dtype=torch.float32, device=dev)
+    sg = torch.empty(w.B, w.Hq, T, p.top_groups, dtype=torch.int32, device=dev)
+    sp = torch.empty(w.B, w.Hq, T, p.top_groups, p.top_pages, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    ws = api.workspace(p, api._lib.LOD_OP_PREFILL)
+    cuts = [0, T] if split is None else [0, split, T]
+    for lo, hi in zip(cuts, cuts[1:]):
+        _prefill_piece(p, q, lo, hi, Kd, Vd, ix, out, lse, sg, sp, ws)
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws) == 0
+    cfg = lt.oracle_cfg(w)
+    rng = np.random.default_rng(3)
+    nch = T // 256
+    for h in range(w.Hkv):
+        K, V = _np(Kc[0, h]), _np(Vc[0, h])
+        u = lt.unit_from_gpu(ix, 0, h, nch, p)
+        lt.check_index_consistency(u, K, V, cfg, w.dtype == "bf16")
+        ts = sorted(set(rng.integers(0, T, 48).tolist()) | {0, 255, 256, 511, 512, T - 1})
+        rows = []
+        for hq in range(h * w.g, (h + 1) * w.g):
+            for t in ts:
+                rows.append((_np(q[0, hq, t]), t, _np(out[0, hq, t]).astype(np.float64),
+                             float(lse[0, hq, t]), sg[0, hq, t].cpu().numpy(), sp[0, hq, t].cpu().numpy()))
+        print(lt.check_rows(cfg, w.dtype, K, V, u, rows))
+
+
+def _prefill_piece(p, q, lo, hi, Kd, Vd, ix, out, lse, sg, sp, ws):
+    o = torch.empty_like(q[:, :, lo:hi].contiguous())
+    l_ = torch.empty(q.shape[0], q.shape[1], hi - lo, dtype=torch.float32, device=q.device)
+    g_ = torch.empty(q.shape[0], q.shape[1], hi - lo, p.top_groups, dtype=torch.int32, device=q.device)
+    p_ = torch.empty(q.shape[0], q.shape[1], hi - lo, p.top_groups, p.top_pages, dtype=torch.int32,
+                     device=q.device)
+    api.lod_prefill(p, q[:, :, lo:hi].contiguous(), lo, Kd, Vd, ix, out=o, lse=l_, sel_groups=g_,
+                    sel_pages=p_, ws=ws)
+    out[:, :, lo:hi] = o
+    lse[:, :, lo:hi] = l_
+    sg[:, :, lo:hi] = g_
+    sp[:, :, lo:hi] = p_
+
+
+# ------------------------------------------------------------------ faults
+
+def test_bad_index_values_are_skipped_and_reported():
+    """A corrupted index entry is bounds-checked by the kernel, skipped, and
+    reported through the status word; nothing out of range is dereferenced."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=1, Hkv=1, Hq=8)
+    T = 4096
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE)
+    q = synth.decode_queries(w).cuda()
+    sl = torch.tensor([T], device="cuda")
+    sg = torch.empty(1, 8, p.top_groups, dtype=torch.int32, device="cuda")
+    api.lod_decode(p, q, Kd, Vd, sl, ix, sel_groups=sg, ws=ws)
+    assert api.lod_get_status(ws) == 0
+    # corrupt every member offset of the chunks the first head opens
+    for gid in sg[0, 0].tolist():
+        c = gid // p.clusters
+        ix.perm[0, 0, c * 256:(c + 1) * 256] = 4000
+    api.lod_decode(p, q, Kd, Vd, sl, ix, ws=ws)
+    st = api.lod_get_status(ws)
+    assert st & api._lib.LOD_ST_BAD_MEMBER
+    assert api.lod_get_status(ws) == 0          # read clears it
+    # a sequence length beyond the cache
+    api.lod_decode(p, q, Kd, Vd, torch.tensor([T + 1], device="cuda"), ix, ws=ws)
+    assert api.lod_get_status(ws) & api._lib.LOD_ST_BAD_SEQLEN
