@@ -1,0 +1,409 @@
+"""Benchmark of the LoD attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: decode_gqa_128k_bf16 (batch 4, 64 query / 8 KV heads,
+head dim 128, context 131072, bf16; top-8 groups, top-2 pages, window 512,
+4 sinks).  One step = one lod_decode call for the whole batch (every query
+head of every sequence, one layer).  Inputs are seeded synthetic data resident
+in HBM; L2 is flushed (a 256 MiB write) between timed steps and each step is
+timed alone with CUDA events on the launching stream.  Rank 0 prints one JSON
+line.  Under torchrun every rank runs its own replica (the path shards by
+sequence with no exchange), and the line reports the aggregate over ranks with
+the max-over-ranks time.
+
+The line also carries the chunked prefill (prefill_128k_bf16) and index build
+(build_128k_bf16, k=4) numbers measured in the same run, the roofline of the
+decode call, the oracle's CPU throughput on a bounded sample, the end-to-end
+rate through the public API with host buffers, and the SM clocks sampled
+during the timed region.
+
+--impl reference times the CPU oracle instead (rank 0 only), on bounded
+samples of the same workload, with the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = "/tmp/lod_clocks_%d_%d.csv" % (os.getpid(), gpu_index)
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1].split()[0]), float(parts[2].split()[0]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        sm = sorted(r[0] for r in rows)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def l2_flusher(dev):
+    buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    return lambda: buf.zero_()
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    """Per-step device time (ms) with an L2 flush between steps, events on `stream`."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- workloads
+
+def params_for(w, k=None):
+    from hierarchical_long_context_b200 import api
+    return api.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, Tmax=((w.T + 255) // 256) * 256,
+                      dtype=w.torch_dtype, clusters=k or w.clusters[0], kmeans_iters=w.iters,
+                      top_groups=w.top_groups, top_pages=w.top_pages, window=w.window, sinks=w.sinks,
+                      seed=w.seed)
+
+
+def run_decode(w, args, dev, stream, world, rank, peaks):
+    from hierarchical_long_context_b200 import api, metrics
+    p = params_for(w)
+    K, V = synth_kv(w)
+    Kd, Vd = K.to(dev), V.to(dev)
+    ix = api.Index(p, dev)
+    api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix, stream=stream)
+    q = synth_q(w).to(dev)
+    sl = torch.full((w.B,), w.T, dtype=torch.int64, device=dev)
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE, dev)
+    out = torch.empty_like(q)
+    sg = torch.empty(w.B, w.Hq, p.top_groups, dtype=torch.int32, device=dev)
+    spg = torch.empty(w.B, w.Hq, p.top_groups, p.top_pages, dtype=torch.int32, device=dev)
+    api.lod_decode(p, q, Kd, Vd, sl, ix, out=out, sel_groups=sg, sel_pages=spg, ws=ws, stream=stream)
+    torch.cuda.synchronize()
+    touched = metrics.decode_touched_bytes(p, ix, sl, sg, spg)
+    flush = l2_flusher(dev)
+    step = lambda: api.lod_decode(p, q, Kd, Vd, sl, ix, out=out, ws=ws, stream=stream)
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device() if world == 1 else int(os.environ.get("LOCAL_RANK", 0))) as cs:
+        t0 = time.perf_counter()
+        ts = time_steps(step, args.steps, args.warmup, flush, stream)
+        wall = time.perf_counter() - t0
+    barrier(world)
+    status = api.lod_get_status(ws, stream)
+    ms = float(np.mean(ts))
+    ms_max = dist_max(ms, world)
+    # end to end through the public API: pinned host q (and this token's K/V row) in, out back
+    qh = q.cpu().pin_memory()
+    newkv = torch.empty(2, w.B, w.Hkv, w.d, dtype=w.torch_dtype).pin_memory()
+    newkv[0] = K[:, :, w.T - 1]
+    newkv[1] = V[:, :, w.T - 1]
+    outh = torch.empty_like(qh).pin_memory()
+    qd = torch.empty_like(q)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        Kd[:, :, w.T - 1].copy_(newkv[0], non_blocking=True)
+        Vd[:, :, w.T - 1].copy_(newkv[1], non_blocking=True)
+        api.lod_decode(p, qd, Kd, Vd, sl, ix, out=out, ws=ws, stream=stream)
+        outh.copy_(out, non_blocking=True)
+
+    e2e_steps = max(10, min(args.steps, 200))
+    te = time_steps(e2e_step, e2e_steps, 3, flush, stream)
+    e2e_ms = dist_max(float(np.mean(te)), world)
+    achieved = touched / (ms * 1e-3) / 1e9
+    res = dict(
+        metric="LoD decode queries/s (batch 4 x 64 heads at 128K context, one layer)",
+        value=world * w.B / (ms_max * 1e-3), unit="queries/s", ms_per_step=ms_max,
+        ms_p10=float(np.percentile(ts, 10)), ms_p90=float(np.percentile(ts, 90)),
+        head_rows_per_s=world * w.B * w.Hq / (ms_max * 1e-3), wall_s_timed=wall,
+        status_word=status,
+        roofline=dict(bound="hbm", kernel="lod_decode (scan + refine kernels)", achieved=achieved,
+                      peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved / peaks["hbm_gbs"],
+                      traffic=None, algorithmic_bytes_per_launch=touched,
+                      peak_source=peaks["source"], nominal_peak_gbs=8000.0),
+        e2e=dict(value=world * w.B / (e2e_ms * 1e-3), unit="queries/s",
+                 h2d_bytes_per_step=qh.numel() * qh.element_size() + newkv.numel() * newkv.element_size(),
+                 d2h_bytes_per_step=outh.numel() * outh.element_size(), ms_per_step=e2e_ms),
+        gpu_launches=2 * args.steps,
+        clocks=cs.summary(),
+        _touch=(K, V, ix),
+    )
+    return res
+
+
+_KV_CACHE = {}
+
+
+def synth_kv(w):
+    from hierarchical_long_context_b200 import synth
+    key = (w.name, w.T, w.B, w.Hkv, w.seed)
+    if key not in _KV_CACHE:
+        _KV_CACHE[key] = synth.kv_cache(w, threads=min(16, host_cores()))
+    return _KV_CACHE[key]
+
+
+def synth_q(w):
+    from hierarchical_long_context_b200 import synth
+    return synth.decode_queries(w)
+
+
+def run_prefill(w, dev, stream, steps, peaks):
+    from hierarchical_long_context_b200 import api, metrics, synth
+    p = params_for(w)
+    K, V = synth_kv(w)
+    Kd, Vd = K.to(dev), V.to(dev)
+    q = synth.prefill_queries(w, 0, w.T).to(dev)
+    out = torch.empty_like(q)
+    ix = api.Index(p, dev)
+    ws = api.workspace(p, api._lib.LOD_OP_PREFILL, dev)
+    flush = l2_flusher(dev)
+    ts = time_steps(lambda: api.lod_prefill(p, q, 0, Kd, Vd, ix, out=out, ws=ws, stream=stream),
+                    steps, 1, flush, stream)
+    ms = float(np.mean(ts))
+    fl = metrics.prefill_flops(p, 0, w.T)
+    tf = fl / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    return dict(workload=w.name, value=w.T * w.B / (ms * 1e-3), unit="tok/s", ms_per_step=ms,
+                roofline=dict(bound="tensor", achieved=tf, peak=peak, unit="TFLOP/s", frac=tf / peak,
+                              algorithmic_flops=fl, peak_source=peaks["source"] + " (sustained)"),
+                status_word=api.lod_get_status(ws, stream))
+
+
+def run_build(w, dev, stream, steps, peaks, k):
+    from hierarchical_long_context_b200 import api, metrics
+    p = params_for(w, k)
+    K, V = synth_kv(w)
+    Kd, Vd = K.to(dev), V.to(dev)
+    ix = api.Index(p, dev)
+    nch = w.T // 256
+    flush = l2_flusher(dev)
+    ts = time_steps(lambda: api.lod_build_index(p, Kd, Vd, 0, nch, ix, stream=stream), steps, 2, flush, stream)
+    ms = float(np.mean(ts))
+    by = metrics.build_bytes(p, nch)
+    gbs = by / (ms * 1e-3) / 1e9
+    fl = metrics.build_flops(p, nch)
+    return dict(workload="%s k=%d" % (w.name, k), value=gbs, unit="GB/s", ms_per_step=ms,
+                chunks_per_s=p.B * p.Hkv * nch / (ms * 1e-3),
+                roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                              frac=gbs / peaks["hbm_gbs"], algorithmic_bytes=by,
+                              fp32_tflops=fl / (ms * 1e-3) / 1e12))
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_decode_rate(w, budget_s=15.0):
+    """The oracle as it stands on this host: per-(b, kvh) index build (untimed,
+    it is the index-build step), then the decode rows of whole sequences, timed,
+    on a thread pool over all host cores.  Returns (queries/s, sample, cores)."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    cores = host_cores()
+    K, V = synth_kv(w)
+    q = synth_q(w)
+    cfg = oracle.Config(d=w.d, clusters=w.clusters[0], iters=w.iters, top_groups=w.top_groups,
+                        top_pages=w.top_pages, window=w.window, sinks=w.sinks,
+                        store_bf16=(w.dtype == "bf16"), seed=w.seed)
+    nch = w.T // 256
+    b = 0
+    with ThreadPoolExecutor(cores) as ex:
+        idx = list(ex.map(lambda h: oracle.build_sequence(cfg, b * w.Hkv + h, K[b, h].float().numpy(),
+                                                           V[b, h].float().numpy(), nch), range(w.Hkv)))
+    Kn = [K[b, h].float().numpy() for h in range(w.Hkv)]
+    Vn = [V[b, h].float().numpy() for h in range(w.Hkv)]
+    rows = [(hq, q[b, hq].float().numpy()) for hq in range(w.Hq)]
+
+    def one(r):
+        hq, qq = r
+        h = hq // w.g
+        oracle.attend_row(cfg, qq, w.T - 1, Kn[h], Vn[h], idx[h])
+
+    n = 0
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        while True:
+            list(ex.map(one, rows))
+            n += 1
+            if time.perf_counter() - t0 > budget_s or n >= 50:
+                break
+    dt = time.perf_counter() - t0
+    return n / dt, "%d decode steps of one sequence (all %d heads) at t=%d" % (n, w.Hq, w.T - 1), cores
+
+
+def run_reference(args, w):
+    rate, sample, cores = oracle_decode_rate(w, budget_s=max(5.0, min(60.0, 3.0 * args.steps)))
+    line = dict(impl="reference", metric="LoD decode queries/s (batch 4 x 64 heads at 128K context, one layer)",
+                value=rate, unit="queries/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64 (oracle)",
+                data="synthetic", config=dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                                              seq_len=w.T, l2="cpu"),
+                cpu_baseline=dict(value=rate, unit="queries/s", cores=cores, kind="oracle", sample=sample),
+                e2e=dict(value=rate, unit="queries/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode_gqa_128k_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the prefill/build/oracle legs")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from hierarchical_long_context_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+    if world > 1:
+        w = w.with_(seed=w.seed + rank)  # every rank its own replica of the batch
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    res = run_decode(w, args, dev, stream, world, rank, peaks)
+    res.pop("_touch")
+    extras = {}
+    if not args.no_extras:
+        wp = synth.WORKLOADS["prefill_128k_bf16"]
+        extras["prefill"] = run_prefill(wp, dev, stream, 2, peaks)
+        wb = synth.WORKLOADS["build_128k_bf16"]
+        extras["build"] = run_build(wb, dev, stream, 5, peaks, 4)
+        if rank == 0 and world == 1:
+            rate, sample, cores = oracle_decode_rate(w)
+            extras["cpu_baseline"] = dict(value=rate, unit="queries/s", cores=cores, kind="oracle", sample=sample)
+    barrier(world)
+    if rank == 0:
+        line = dict(metric=res["metric"], value=res["value"], unit=res["unit"], n_gpus=world,
+                    steps=args.steps, warmup=args.warmup, ms_per_step=res["ms_per_step"],
+                    higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+                    data="synthetic (seeded Gaussian-mixture keys + RoPE + outlier channels, N(0,1) values)",
+                    config=dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, seq_len=w.T,
+                                clusters=w.clusters[0], top_groups=w.top_groups, top_pages=w.top_pages,
+                                window=w.window, sinks=w.sinks, parallelism="replicas x%d" % world,
+                                l2="flushed (256 MiB write) between timed steps"),
+                    roofline=res["roofline"], cpu_baseline=extras.pop("cpu_baseline", None),
+                    e2e=res["e2e"], gpu_launches=res["gpu_launches"], clocks=res["clocks"],
+                    ms_p10=res["ms_p10"], ms_p90=res["ms_p90"], head_rows_per_s=res["head_rows_per_s"],
+                    status_word=res["status_word"], **extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
