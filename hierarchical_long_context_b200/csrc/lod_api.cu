@@ -30,7 +30,8 @@ int64_t elem_bytes(const lod_params* p) { return p->dtype == LOD_DTYPE_F32 ? 4 :
 int32_t page_slots(const lod_params* p) { return p->chunk / p->page + p->clusters; }
 int32_t g_of(const lod_params* p) { return p->Hq / p->Hkv; }
 int kg_of(const lod_params* p) { return p->top_groups <= 8 ? 8 : 16; }
-int nq_max(const lod_params* p) { return p->d == 64 ? 16 : 8; }
+// query rows per scan unit (registers: NQ x 8 fp32 accumulators per lane)
+int nq_max(const lod_params*) { return 8; }
 
 int32_t validate(const lod_params* p) {
   if (!p) return fail(LOD_EINVAL, "params is NULL");
@@ -42,8 +43,7 @@ int32_t validate(const lod_params* p) {
   const int g = g_of(p);
   if (g & (g - 1)) return fail(LOD_EUNSUPPORTED, "Hq/Hkv = %d must be a power of two", g);
   if (p->d != 64 && p->d != 128) return fail(LOD_EUNSUPPORTED, "d = %d unsupported (64 or 128)", p->d);
-  if (g > nq_max(p))
-    return fail(LOD_EUNSUPPORTED, "Hq/Hkv = %d exceeds %d at d = %d", g, nq_max(p), p->d);
+  if (g > nq_max(p)) return fail(LOD_EUNSUPPORTED, "Hq/Hkv = %d exceeds %d", g, nq_max(p));
   if (p->chunk != lod::kChunk) return fail(LOD_EUNSUPPORTED, "chunk must be %d", lod::kChunk);
   if (p->page != lod::kPage) return fail(LOD_EUNSUPPORTED, "page must be %d", lod::kPage);
   if (p->clusters < 1 || p->clusters > lod::kMaxClusters)
@@ -81,7 +81,11 @@ int32_t validate_index(const lod_index* ix) {
     if (!ptrs[i]) return fail(LOD_EINVAL, "index field %d is NULL", i);
     if (i == 0 || i == 1 || i == 3 || i == 4) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index summary %d must be 16-byte aligned", i);
-    } else if (reinterpret_cast<uintptr_t>(ptrs[i]) & 3u && i != 6 && i != 7 && i != 8) {
+    } else if (i == 8) {
+      if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index member list (perm) must be 16-byte aligned");
+    } else if ((i == 2 || i == 5) && (reinterpret_cast<uintptr_t>(ptrs[i]) & 3u)) {
+      return fail(LOD_EINVAL, "index field %d misaligned", i);
+    } else if (reinterpret_cast<uintptr_t>(ptrs[i]) & 1u) {
       return fail(LOD_EINVAL, "index field %d misaligned", i);
     }
   }
@@ -99,7 +103,7 @@ AttendShape decode_shape(const lod_params* p) {
   s.NP = 1;
   s.NQ = g_of(p);
   s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
-  s.nsw = (int)cdiv(p->window, lod::kScanRows);
+  s.nsw = (int)cdiv(p->window + p->sinks, lod::kScanRows);
   s.units = (int64_t)p->B * p->Hkv;
   return s;
 }
@@ -110,7 +114,7 @@ AttendShape prefill_shape(const lod_params* p) {
   s.NP = nq_max(p) / g_of(p);
   s.NQ = s.NP * g_of(p);
   s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
-  s.nsw = (int)cdiv(p->window, lod::kScanRows);
+  s.nsw = (int)cdiv(p->window + p->sinks, lod::kScanRows);
   s.units = (int64_t)p->B * p->Hkv * cdiv(p->chunk, s.NP);
   return s;
 }
@@ -118,7 +122,7 @@ AttendShape prefill_shape(const lod_params* p) {
 size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
   const int KG = kg_of(p);
   size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
-  size_t cand = (sizeof(float) + sizeof(int)) * (size_t)s.units * s.nsg * s.NQ * KG;
+  size_t cand = lod::cand_bytes() * (size_t)s.units * s.nsg * s.NQ * KG;
   return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((cand + 255) & ~size_t(255));
 }
 
@@ -162,9 +166,8 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
   part = (part + 255) & ~size_t(255);
   a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
-  a.cand_s = reinterpret_cast<float*>(w + lod::kWsHeader + part);
-  a.cand_i = reinterpret_cast<int*>(w + lod::kWsHeader + part +
-                                     sizeof(float) * (size_t)s.units * s.nsg * s.NQ * KG);
+  a.cand = w + lod::kWsHeader + part;
+  (void)KG;
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,

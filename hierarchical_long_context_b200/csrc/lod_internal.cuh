@@ -62,9 +62,8 @@ struct AttendArgs {
   float scale;
   int nsg, nsw;             // group splits and window splits per unit
   int64_t units;            // scan units in this launch
-  float* part;              // [units][nsg+nsw][NQ][d+2]  (m, l, acc[d])
-  float* cand_s;            // [units][nsg][NQ][G]
-  int* cand_i;              // [units][nsg][NQ][G]
+  float* part;              // [units][nsg+nsw][NQ][d+2]  (m, l, acc)
+  void* cand;               // [units][nsg][NQ][KG] candidate records (cand_bytes() each)
   void* out;                // [B][Hq][Tq][d]
   float* lse;               // [B][Hq][Tq] or null
   int32_t* sel_groups;      // [B][Hq][Tq][G] or null
@@ -75,5 +74,6 @@ struct AttendArgs {
 cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
                          cudaStream_t stream);
 cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, cudaStream_t stream);
+size_t cand_bytes();
 
 }  // namespace lod

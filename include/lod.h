@@ -61,6 +61,7 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
 #define LOD_ST_BAD_PAGE 0x2u     /* page range or page slot outside the chunk's slots */
 #define LOD_ST_BAD_MEMBER 0x4u   /* member offset outside the chunk */
 #define LOD_ST_BAD_COUNT 0x8u    /* group or page count outside [0, chunk] */
+#define LOD_ST_TIMEOUT 0x10u     /* an asynchronous copy did not complete within the kernel's wait limit */
 
 /*
  * Parameters.  Supported: dtype F32 or BF16 (cache, summaries, q and out all
@@ -68,8 +69,7 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
  * values); 1 <= clusters <= 16; 1 <= kmeans_iters <= 64; 1 <= top_groups
  * <= 16; 1 <= top_pages <= 4; window a positive multiple of chunk (the
  * page says 256-512); 0 <= sinks < chunk; Hq a multiple of Hkv with
- * Hq/Hkv a power of two, at most 8 at d = 128 and 16 at d = 64; Tmax a
- * positive multiple of chunk.
+ * Hq/Hkv a power of two no larger than 8; Tmax a positive multiple of chunk.
  * scale <= 0 selects 1/sqrt(d).
  */
 typedef struct lod_params {
@@ -105,7 +105,8 @@ typedef struct lod_params {
  *   gPage   [Cmax*(k+1)]  int16 pages of group j are slots [gPage[j], gPage[j+1])
  *   perm    [Cmax*chunk]  int16 chunk-local token offsets, group-major and
  *                         ascending within a group; -1 past the last member
- * Every array is laid out [B][Hkv][...] in that order.
+ * Every array is laid out [B][Hkv][...] in that order.  gK, gV, pK, pV and
+ * perm must be 16-byte aligned, gCnt and pCnt 4-byte aligned.
  */
 typedef struct lod_index {
   void* gK;

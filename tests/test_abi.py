@@ -59,7 +59,8 @@ def test_index_sizes_match_the_documented_layout():
     (dict(d=96), _lib.LOD_EUNSUPPORTED),
     (dict(Hq=12, Hkv=8), _lib.LOD_EINVAL),
     (dict(Hq=48, Hkv=8), _lib.LOD_EUNSUPPORTED),     # g = 6 is not a power of two
-    (dict(Hq=128, Hkv=8), _lib.LOD_EUNSUPPORTED),    # g = 16 at d = 128
+    (dict(Hq=128, Hkv=8), _lib.LOD_EUNSUPPORTED),    # g = 16
+    (dict(Hq=16, Hkv=1, d=64), _lib.LOD_EUNSUPPORTED),
     (dict(window=300), _lib.LOD_EINVAL),
     (dict(window=0), _lib.LOD_EINVAL),
     (dict(sinks=256), _lib.LOD_EINVAL),
