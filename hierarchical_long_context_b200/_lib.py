@@ -19,7 +19,8 @@ LOD_ST_BAD_SEQLEN, LOD_ST_BAD_PAGE, LOD_ST_BAD_MEMBER, LOD_ST_BAD_COUNT = 1, 2, 
 
 # Every symbol include/lod.h declares.
 EXPORTS = ("lod_version", "lod_last_error", "lod_index_sizes", "lod_workspace_bytes",
-           "lod_build_index", "lod_decode", "lod_prefill", "lod_get_status")
+           "lod_build_index", "lod_decode", "lod_prefill", "lod_get_status", "lod_decode_noalloc")
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class lod_params(ctypes.Structure):
@@ -79,6 +80,9 @@ def load():
     lib.lod_prefill.restype = ctypes.c_int32
     lib.lod_prefill.argtypes = [_P(lod_params), _vp, _i64, _i64, _vp, _vp, _P(_i64), _P(lod_index),
                                 _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.lod_decode_noalloc.restype = ctypes.c_int32
+    lib.lod_decode_noalloc.argtypes = [_P(lod_params), _vp, _vp, _vp, _P(_i64), _vp, _P(lod_index), _vp,
+                                       _vp, _vp, _vp, _vp, _vp]
     lib.lod_get_status.restype = ctypes.c_int32
     lib.lod_get_status.argtypes = [_vp, _vp, _P(ctypes.c_uint32)]
     _lib = lib

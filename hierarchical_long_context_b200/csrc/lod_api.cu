@@ -1,8 +1,10 @@
 // lod_api.cu -- the extern "C" entry points declared in include/lod.h:
 // argument validation, index and workspace sizing, and kernel launches.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "lod_internal.cuh"
 
@@ -352,3 +354,96 @@ int32_t lod_get_status(void* ws, lod_stream_t stream, uint32_t* status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// lod_decode_noalloc: lod_decode without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc at all: an inference engine whose
+// memory pool owns every device allocation, a runtime that must not allocate
+// while a CUDA graph or a latency-critical step is being recorded, or a
+// plugin host that gives its kernels only their input and output buffers.
+// For them this entry point keeps the decode scratch (split partial states,
+// candidate records and the status word) in a fixed array compiled into the
+// library.  The array is `static __device__`, so each GPU that loads this
+// library holds its kLodNoallocScratchBytes until the process exits.  Host
+// code cannot use the array's name as an address; the device address is
+// looked up once per device with cudaGetSymbolAddress, with that device
+// current, on the first call made on that device.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kLodNoallocScratchBytes = LOD_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kLodNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::atomic<int> g_noalloc_ready[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of this device's copy of the scratch array (set-up on first use).
+int32_t noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LOD_EUNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  if (!g_noalloc_ready[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ready[dev].load(std::memory_order_relaxed)) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+      g_noalloc_ptr[dev] = p;
+      g_noalloc_ready[dev].store(1, std::memory_order_release);
+    }
+  }
+  *out = g_noalloc_ptr[dev];
+  return LOD_OK;
+}
+
+}  // namespace
+
+extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const void* K, const void* V,
+                                      const int64_t kv_strides[3], const int64_t* seq_lens,
+                                      const lod_index* index, void* out, float* lse, int32_t* sel_groups,
+                                      int32_t* sel_pages, uint32_t* status, lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (!rc) rc = validate_index(index);
+  if (rc) return rc;
+  if (!q || !out || !seq_lens) return fail(LOD_EINVAL, "q, out and seq_lens must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
+  const AttendShape s = decode_shape(p);
+  const size_t need = attend_ws_bytes(p, s);
+  if (need > kLodNoallocScratchBytes)
+    return fail(LOD_EINVAL,
+                "decode scratch of %zu bytes exceeds the built-in %zu-byte array of lod_decode_noalloc "
+                "(fewer sequences, KV heads or a smaller Tmax fit; otherwise use lod_decode)",
+                need, kLodNoallocScratchBytes);
+  void* ws = nullptr;
+  rc = noalloc_scratch(&ws);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  // The partial states and candidates are fully rewritten by every call; only
+  // the status word must start from zero when no caller word is given.
+  if (!status) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc status word");
+  }
+  lod::AttendArgs a;
+  fill_attend(a, p, s, K, V, kv_strides, index, ws);
+  if (status) a.status = status;
+  a.q = q;
+  a.Tq = 1;
+  a.q_begin = 0;
+  a.seq_lens = seq_lens;
+  a.pos_lo = 0;
+  a.pos_hi = 1;
+  a.out = out;
+  a.lse = lse;
+  a.sel_groups = sel_groups;
+  a.sel_pages = sel_pages;
+  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, st);
+  if (e != cudaSuccess) return cuda_fail(e, "no-alloc decode launch");
+  g_err[0] = 0;
+  return LOD_OK;
+}

@@ -209,6 +209,45 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
                     int32_t* sel_pages, void* ws, size_t ws_bytes, lod_stream_t stream);
 
 /*
+ * Size of the scratch array built into the library for lod_decode_noalloc.
+ */
+#define LOD_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * lod_decode without a workspace argument, for callers that cannot allocate
+ * device memory themselves: a serving engine whose memory pool owns every
+ * allocation, a runtime that may not allocate while it records a CUDA graph
+ * or runs a latency-critical step, or a plugin host that hands its kernels
+ * only input and output buffers.  The method's pages have no counterpart of
+ * this entry point: it exists only for those callers.
+ *
+ * Computes exactly what lod_decode computes, with the same arguments and
+ * layouts, except:
+ *   - no ws / ws_bytes: the scratch lives in a fixed device array of
+ *     LOD_NOALLOC_SCRATCH_BYTES (8 MiB) compiled into the library.  Every GPU
+ *     that loads the library holds that array until the process exits.
+ *     Shapes whose scratch (lod_workspace_bytes(LOD_OP_DECODE)) exceeds it
+ *     are rejected with LOD_EINVAL and a message naming both sizes; nothing
+ *     is enqueued then.  (The 128K-context decode of 4 sequences x 8 KV heads
+ *     x 8 query heads per KV head needs about 3.3 MB.)
+ *   - status: nullable device pointer to a uint32_t that receives (bitwise
+ *     OR) this call's LOD_ST_* bits; the caller zeroes it.  When NULL the
+ *     bits are recorded in the built-in array and not reported.
+ * No device memory is allocated or freed by this call, by the library or by
+ * any library it calls.  The first call on each device looks up that
+ * device's address of the built-in array (cudaGetSymbolAddress, with that
+ * device current); make the first call on a device outside any stream
+ * capture.  All calls on one device share the one array and it keeps the
+ * last call's contents: calls whose executions can overlap on the GPU
+ * (different streams without ordering, or concurrent host threads) race on
+ * it and produce undefined results.  Order them on one stream.
+ */
+int32_t lod_decode_noalloc(const lod_params* p, const void* q, const void* K, const void* V,
+                           const int64_t kv_strides[3], const int64_t* seq_lens, const lod_index* index,
+                           void* out, float* lse, int32_t* sel_groups, int32_t* sel_pages,
+                           uint32_t* status, lod_stream_t stream);
+
+/*
  * Read and clear the device status word kept in `ws` (the only synchronising
  * call: it waits for `stream`).  *status (host) receives the LOD_ST_* bits
  * recorded since the last read; returns LOD_EDEVICE if any bit was set.
