@@ -1,10 +1,13 @@
 // lod_api.cu -- the extern "C" entry points declared in include/lod.h:
 // argument validation, index and workspace sizing, and kernel launches.
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+
+#include <cudaTypedefs.h>
 
 #include "lod_internal.cuh"
 
@@ -95,36 +98,101 @@ int32_t validate_index(const lod_index* ix) {
 }
 
 struct AttendShape {
-  int NQ, NP, nsg, nsw;
+  int NQ, NP, nsplit;
   int64_t units;
+  bool tc;  // tensor-core scan (bf16, d = 128)
 };
 
-// Decode: one unit per (b, kvh); group splits cover the largest index.
+// Splits per unit: enough scan CTAs to fill the GPU (`target` CTAs), never
+// fewer than one pipeline stage of rows per split.
+int split_count(int64_t units, int64_t rows, int64_t target, int64_t rows_per_stage) {
+  int64_t s = units >= target ? 1 : target / units;
+  const int64_t most = cdiv(rows, rows_per_stage);
+  if (s > most) s = most;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+// Longest row list of a unit: every group of the index and the window.
+int64_t max_rows(const lod_params* p) { return p->Tmax / p->chunk * p->clusters + p->window; }
+
+// The tensor-core scan runs for bf16 caches with d = 128 (one CTA per SM,
+// 128-row tiles, up to 16 query rows per unit); everything else takes the
+// CUDA-core scan (two CTAs per SM, 64-row stages, up to 8 query rows).
+bool use_tc(const lod_params* p) {
+  return p->dtype == LOD_DTYPE_BF16 && p->d == 128 &&
+         (int64_t)p->B * p->Hkv * (p->Tmax / p->chunk) * p->clusters < ((int64_t)1 << 31) &&
+         p->Tmax < ((int64_t)1 << 31);
+}
+constexpr int64_t kTcCtas = 148, kTcTile = 128, kCoreCtas = lod::kTargetCtas;
+
+int split_for(const lod_params* p, bool tc, int64_t units, int64_t rows) {
+  return tc ? split_count(units, rows, kTcCtas, kTcTile) : split_count(units, rows, kCoreCtas, lod::kScanSlab);
+}
+
+// Decode: one unit per (b, kvh).
 AttendShape decode_shape(const lod_params* p) {
   AttendShape s;
+  s.tc = use_tc(p);
   s.NP = 1;
   s.NQ = g_of(p);
-  s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
-  s.nsw = (int)cdiv(p->window + p->sinks, lod::kScanRows);
   s.units = (int64_t)p->B * p->Hkv;
+  s.nsplit = split_for(p, s.tc, s.units, max_rows(p));
   return s;
 }
 
 // Prefill: one launch per query chunk; NP positions per unit.
 AttendShape prefill_shape(const lod_params* p) {
   AttendShape s;
-  s.NP = nq_max(p) / g_of(p);
+  s.tc = use_tc(p);
+  s.NP = (s.tc ? 16 : nq_max(p)) / g_of(p);
   s.NQ = s.NP * g_of(p);
-  s.nsg = (int)cdiv(p->Tmax / p->chunk * p->clusters, lod::kScanRows);
-  s.nsw = (int)cdiv(p->window + p->sinks, lod::kScanRows);
   s.units = (int64_t)p->B * p->Hkv * cdiv(p->chunk, s.NP);
+  s.nsplit = split_for(p, s.tc, s.units, max_rows(p));
   return s;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int32_t encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                   const cuuint64_t* strides_bytes) {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(LOD_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint32_t box4[4] = {64, 128, 1, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+                        strides_bytes, box4, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LOD_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LOD_OK;
+}
+
+// Tensor maps of the group summaries and the KV cache for the tensor-core scan.
+int32_t make_tc_maps(const lod_params* p, const void* K, const void* V, const int64_t* kv, const lod_index* ix,
+                     lod::TcMaps* m) {
+  const cuuint64_t rows = (cuuint64_t)p->B * p->Hkv * (p->Tmax / p->chunk) * p->clusters;
+  const cuuint64_t gdims[2] = {(cuuint64_t)p->d, rows};
+  const cuuint64_t gstr[1] = {(cuuint64_t)p->d * 2};
+  int32_t rc = encode_map(&m->gK, ix->gK, 2, gdims, gstr);
+  if (!rc) rc = encode_map(&m->gV, ix->gV, 2, gdims, gstr);
+  const cuuint64_t kdims[4] = {(cuuint64_t)p->d, (cuuint64_t)p->Tmax, (cuuint64_t)p->Hkv, (cuuint64_t)p->B};
+  const cuuint64_t kstr[3] = {(cuuint64_t)kv[2] * 2, (cuuint64_t)kv[1] * 2, (cuuint64_t)kv[0] * 2};
+  if (!rc) rc = encode_map(&m->K, K, 4, kdims, kstr);
+  if (!rc) rc = encode_map(&m->V, V, 4, kdims, kstr);
+  return rc;
 }
 
 size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
   const int KG = kg_of(p);
-  size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
-  size_t cand = lod::cand_bytes() * (size_t)s.units * s.nsg * s.NQ * KG;
+  size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
+  size_t cand = lod::cand_bytes() * (size_t)s.units * s.nsplit * s.NQ * KG;
   return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((cand + 255) & ~size_t(255));
 }
 
@@ -159,13 +227,12 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   a.sinks = p->sinks;
   a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
   a.NP = s.NP;
-  a.nsg = s.nsg;
-  a.nsw = s.nsw;
+  a.nsplit = s.nsplit;
   a.units = s.units;
   char* w = static_cast<char*>(ws);
   a.status = reinterpret_cast<uint32_t*>(w);
   const int KG = kg_of(p);
-  size_t part = sizeof(float) * (size_t)s.units * (s.nsg + s.nsw) * s.NQ * (p->d + 2);
+  size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
   part = (part + 255) & ~size_t(255);
   a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
   a.cand = w + lod::kWsHeader + part;
@@ -285,7 +352,12 @@ int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void
   a.lse = lse;
   a.sel_groups = sel_groups;
   a.sel_pages = sel_pages;
-  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, (cudaStream_t)stream);
+  lod::TcMaps maps;
+  if (s.tc) {
+    rc = make_tc_maps(p, K, V, kv_strides, index, &maps);
+    if (rc) return rc;
+  }
+  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, s.tc ? &maps : nullptr, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_err[0] = 0;
   return LOD_OK;
@@ -324,6 +396,11 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   a.lse = lse;
   a.sel_groups = sel_groups;
   a.sel_pages = sel_pages;
+  lod::TcMaps maps;
+  if (s.tc) {
+    rc = make_tc_maps(p, K, V, kv_strides, index, &maps);
+    if (rc) return rc;
+  }
   const int64_t nw = p->window / p->chunk;
   for (int64_t lo = 0; lo < Tq; lo += p->chunk) {
     const int64_t hi = lo + p->chunk < Tq ? lo + p->chunk : Tq;
@@ -331,10 +408,11 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     const int64_t wb = bt - nw + 1 > 0 ? bt - nw + 1 : 0;
     a.pos_lo = lo;
     a.pos_hi = hi;
-    a.nsg = (int)cdiv(wb * p->clusters, lod::kScanRows);
     a.units = (int64_t)p->B * p->Hkv * cdiv(hi - lo, s.NP);
+    const int want = split_for(p, s.tc, a.units, wb * p->clusters + p->window);
+    a.nsplit = want < s.nsplit ? want : s.nsplit;
     // part/cand keep the worst-case layout of fill_attend; a chunk uses a prefix
-    cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, st);
+    cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, s.tc ? &maps : nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   }
   g_err[0] = 0;
@@ -442,7 +520,12 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
   a.lse = lse;
   a.sel_groups = sel_groups;
   a.sel_pages = sel_pages;
-  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, st);
+  lod::TcMaps maps;
+  if (s.tc) {
+    rc = make_tc_maps(p, K, V, kv_strides, index, &maps);
+    if (rc) return rc;
+  }
+  cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, s.tc ? &maps : nullptr, st);
   if (e != cudaSuccess) return cuda_fail(e, "no-alloc decode launch");
   g_err[0] = 0;
   return LOD_OK;

@@ -106,50 +106,60 @@ struct Cand {
 
 // ------------------------------------------------------------------ scan
 
+constexpr int kSlab = 64;    // rows per pipeline stage
+constexpr int kStages = 3;   // TMA ring depth
+
 template <typename T, int D, int NQ>
 struct ScanSmem {
-  static constexpr int R = kScanRows;
-  static constexpr size_t kv_bytes = (size_t)R * D * sizeof(T);
-  static constexpr size_t off_V = kv_bytes;
-  static constexpr size_t off_S = 2 * kv_bytes;                        // float [NQ][R]
-  static constexpr size_t off_P = off_S + sizeof(float) * NQ * R;      // float [R][NQ]
-  static constexpr size_t off_lnc = off_P + sizeof(float) * NQ * R;    // float [R]
-  static constexpr size_t off_pos = off_lnc + sizeof(float) * R;       // int64 [R]
-  static constexpr size_t off_m = off_pos + sizeof(int64_t) * R;       // float [NQ]
-  static constexpr size_t off_l = off_m + sizeof(float) * 16;          // float [NQ]
-  static constexpr size_t off_bar = off_l + sizeof(float) * 16;        // uint64 [2]
-  static constexpr size_t bytes = off_bar + 16;
-  static_assert(sizeof(float) * kWarps * NQ * D <= kv_bytes, "reduction scratch reuses the K stage");
+  static constexpr size_t stage_bytes = (size_t)kSlab * D * sizeof(T);      // K or V of one slab
+  static constexpr size_t off_K = 0;                                        // [kStages][kSlab][D]
+  static constexpr size_t off_V = kStages * stage_bytes;                    // [kStages][kSlab][D]
+  static constexpr size_t off_S = 2 * kStages * stage_bytes;                // float [NQ][kSlab]
+  static constexpr size_t off_P = off_S + sizeof(float) * NQ * kSlab;       // float [kSlab][NQ]
+  static constexpr size_t off_lnc = off_P + sizeof(float) * NQ * kSlab;     // float [kStages][kSlab]
+  static constexpr size_t off_pos = off_lnc + sizeof(float) * kStages * kSlab;  // int64 [kStages][kSlab]
+  static constexpr size_t off_corr = off_pos + sizeof(int64_t) * kStages * kSlab;  // float [16]
+  static constexpr size_t off_bar = off_corr + sizeof(float) * 16;          // uint64 [kStages]
+  static constexpr size_t bytes = off_bar + 8 * kStages;
+  // the final cross-warp reduction reuses the K ring
+  static_assert(sizeof(float) * kWarps * NQ * D <= kStages * stage_bytes, "reduction scratch");
 };
+
+// Row e of a unit's row list: e < G_vis -> group summary e; then the sinks;
+// then the window [ws, t_max].  Returns the token position (-1 for a group).
+__device__ __forceinline__ int64_t row_pos(int64_t e, int64_t G_vis, int64_t ns, int64_t ws) {
+  if (e < G_vis) return -1;
+  e -= G_vis;
+  return e < ns ? e : ws + (e - ns);
+}
 
 template <typename T, int D, int NQ, int KG>
 __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   constexpr int EPL = 16 / sizeof(T);  // elements per lane per 16-byte load
   constexpr int LPR = D / EPL;         // lanes per row
   constexpr int RPI = 32 / LPR;        // rows per warp per step
-  constexpr int R = kScanRows;
   constexpr int ROWB = D * sizeof(T);
+  constexpr int SHIFT = ilog2(LPR) - ilog2(NQ);
   using SM = ScanSmem<T, D, NQ>;
   static_assert(NQ <= LPR, "each query row's score must land on its own lanes");
+  static_assert(kSlab % (kWarps * RPI) == 0, "a slab is a whole number of warp steps");
 
   const int64_t u = blockIdx.x;
   const int s = blockIdx.y;
-  const int nsplit = a.nsg + a.nsw;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int li = lane % LPR, sub = lane / LPR;
   const UnitInfo ui = unit_info(a, u);
 
   extern __shared__ __align__(128) unsigned char smem[];
-  T* Ks = reinterpret_cast<T*>(smem);
-  T* Vs = reinterpret_cast<T*>(smem + SM::off_V);
+  T* Kr = reinterpret_cast<T*>(smem + SM::off_K);
+  T* Vr = reinterpret_cast<T*>(smem + SM::off_V);
   float* S_s = reinterpret_cast<float*>(smem + SM::off_S);
   float* P_s = reinterpret_cast<float*>(smem + SM::off_P);
   float* lnc_s = reinterpret_cast<float*>(smem + SM::off_lnc);
   int64_t* pos_s = reinterpret_cast<int64_t*>(smem + SM::off_pos);
-  float* m_s = reinterpret_cast<float*>(smem + SM::off_m);
-  float* l_s = reinterpret_cast<float*>(smem + SM::off_l);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM::off_bar);
-  float* red = reinterpret_cast<float*>(smem);  // [kWarps][NQ][D], after pass 1
+  float* corr_s = reinterpret_cast<float*>(smem + SM::off_corr);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::off_bar);
+  float* red = reinterpret_cast<float*>(smem);  // [kWarps][NQ][D] at the end
 
   // ---- the unit's query rows: positions and validity
   int64_t t_row[NQ];
@@ -170,307 +180,329 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   }
   if (a.seq_lens && t_max < 0 && s == 0 && tid == 0) set_status(a.status, LOD_ST_BAD_SEQLEN);
 
-  // ---- rows of this split
+  // ---- this split's slice of the unit's row list
   const int64_t unit_kv = (int64_t)ui.b * a.Hkv + ui.kvh;
-  const bool is_group = s < a.nsg;
-  int64_t lo = 0, ws = 0;
-  int nrows = 0, ns = 0;
-  int64_t wb = 0;
+  int64_t G_vis = 0, ns = 0, ws = 0, e0 = 0, e1 = 0;
   if (t_max >= 0) {
     const int64_t bt = t_max / kChunk;
     const int64_t nw = a.window / kChunk;
-    wb = bt - nw + 1 > 0 ? bt - nw + 1 : 0;  // visible chunks [0, wb)
-    ws = wb * kChunk;                        // window start
-    if (is_group) {
-      const int64_t G_vis = wb * a.k;
-      const int64_t per = (G_vis + a.nsg - 1) / a.nsg;
-      lo = s * per;
-      const int64_t hi = lo + per < G_vis ? lo + per : G_vis;
-      nrows = hi > lo ? (int)(hi - lo) : 0;
-    } else {
-      // window list: the sinks, then [ws, t_max]
-      const int64_t nsk = a.sinks < ws ? a.sinks : ws;
-      const int64_t total = nsk + (t_max - ws + 1);
-      const int64_t per = (total + a.nsw - 1) / a.nsw;
-      const int64_t e0 = (int64_t)(s - a.nsg) * per;
-      const int64_t e1 = e0 + per < total ? e0 + per : total;
-      nrows = e1 > e0 ? (int)(e1 - e0) : 0;
-      lo = e0;       // first list index
-      ns = (int)nsk; // list indices < ns are sinks
-    }
+    const int64_t wb = bt - nw + 1 > 0 ? bt - nw + 1 : 0;  // visible chunks [0, wb)
+    ws = wb * kChunk;
+    G_vis = wb * a.k;
+    ns = 0;  // the sinks are exact tokens added by the refine kernel
+    const int64_t total = G_vis + ns + (t_max - ws + 1);
+    const int64_t per = (total + a.nsplit - 1) / a.nsplit;
+    e0 = s * per < total ? s * per : total;
+    e1 = e0 + per < total ? e0 + per : total;
   }
+  const int nslab = (int)((e1 - e0 + kSlab - 1) / kSlab);
   const T* Kb = static_cast<const T*>(a.K) + ui.b * a.sb + ui.kvh * a.sh;
   const T* Vb = static_cast<const T*>(a.V) + ui.b * a.sb + ui.kvh * a.sh;
   const T* gK = static_cast<const T*>(a.gK) + unit_kv * a.Cmax * a.k * D;
   const T* gV = static_cast<const T*>(a.gV) + unit_kv * a.Cmax * a.k * D;
   const int32_t* gC = a.gCnt + unit_kv * a.Cmax * a.k;
+  const bool contiguous = a.st == D;
 
-  // ---- stage the rows in shared memory: two pipeline stages of TMA bulk copies
-  const int n0 = nrows < R / 2 ? nrows : R / 2;
-  if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (warp == 0 && nrows > 0) {
-    for (int st = 0; st < 2; ++st) {
-      const int r0 = st ? n0 : 0, r1 = st ? nrows : n0;
-      if (r1 <= r0) continue;
-      if (lane == 0) mbar_arrive_expect(&bar[st], (uint32_t)(r1 - r0) * 2u * ROWB);
-      __syncwarp();
-      if (is_group) {
+  // producer: stage slab i (rows [e0 + 64 i, ...)) into ring slot i % kStages
+  auto issue = [&](int i) {
+    const int st = i % kStages;
+    const int64_t r0 = e0 + (int64_t)i * kSlab;
+    const int64_t r1 = r0 + kSlab < e1 ? r0 + kSlab : e1;
+    const int n = (int)(r1 - r0);
+    T* kd = Kr + (size_t)st * kSlab * D;
+    T* vd = Vr + (size_t)st * kSlab * D;
+    if (lane == 0) mbar_arrive_expect(&full[st], (uint32_t)n * 2u * ROWB);
+    __syncwarp();
+    // group summaries: one contiguous run
+    const int64_t g1 = r1 < G_vis ? r1 : G_vis;
+    if (r0 < g1 && lane == 0) {
+      bulk_g2s(kd, gK + r0 * D, (uint32_t)(g1 - r0) * ROWB, &full[st]);
+      bulk_g2s(vd, gV + r0 * D, (uint32_t)(g1 - r0) * ROWB, &full[st]);
+    }
+    // tokens (sinks, then the window): runs of consecutive positions
+    const int64_t t0 = r0 > G_vis ? r0 : G_vis;
+    if (t0 < r1) {
+      if (contiguous) {
         if (lane == 0) {
-          bulk_g2s(Ks + r0 * D, gK + (lo + r0) * D, (uint32_t)(r1 - r0) * ROWB, &bar[st]);
-          bulk_g2s(Vs + r0 * D, gV + (lo + r0) * D, (uint32_t)(r1 - r0) * ROWB, &bar[st]);
+          // at most two runs: sinks [.., ns) and window [ws, ..)
+          int64_t e = t0;
+          while (e < r1) {
+            const int64_t p = row_pos(e, G_vis, ns, ws);
+            int64_t run_end = e - G_vis < ns ? G_vis + ns : r1;
+            if (run_end > r1) run_end = r1;
+            const uint32_t bytes = (uint32_t)(run_end - e) * ROWB;
+            bulk_g2s(kd + (e - r0) * D, Kb + p * D, bytes, &full[st]);
+            bulk_g2s(vd + (e - r0) * D, Vb + p * D, bytes, &full[st]);
+            e = run_end;
+          }
         }
       } else {
-        for (int r = r0 + lane; r < r1; r += 32) {
-          const int64_t e = lo + r;
-          const int64_t pos = e < ns ? e : ws + (e - ns);
-          bulk_g2s(Ks + r * D, Kb + pos * a.st, ROWB, &bar[st]);
-          bulk_g2s(Vs + r * D, Vb + pos * a.st, ROWB, &bar[st]);
+        for (int64_t e = t0 + lane; e < r1; e += 32) {
+          const int64_t p = row_pos(e, G_vis, ns, ws);
+          bulk_g2s(kd + (e - r0) * D, Kb + p * a.st, ROWB, &full[st]);
+          bulk_g2s(vd + (e - r0) * D, Vb + p * a.st, ROWB, &full[st]);
         }
       }
     }
-  }
-  // per-row log-count (group rows) and position (window rows), -inf = skip
-  for (int r = tid; r < R; r += kThreads) {
+  };
+  // row metadata of slab i (log count, -inf = skip; token position or -1)
+  auto meta = [&](int i, int r) {
+    const int st = i % kStages;
+    const int64_t e = e0 + (int64_t)i * kSlab + r;
     float lc = -INFINITY;
-    int64_t pos = -1;
-    if (r < nrows) {
-      if (is_group) {
-        const int cnt = gC[lo + r];
+    int64_t p = -1;
+    if (e < e1) {
+      if (e < G_vis) {
+        const int cnt = gC[e];
         if (cnt > 0 && cnt <= kChunk) lc = __logf((float)cnt);
         else if (cnt > kChunk) set_status(a.status, LOD_ST_BAD_COUNT);
       } else {
-        const int64_t e = lo + r;
-        pos = e < ns ? e : ws + (e - ns);
+        p = row_pos(e, G_vis, ns, ws);
         lc = 0.f;
       }
     }
-    lnc_s[r] = lc;
-    pos_s[r] = pos;
-  }
+    lnc_s[st * kSlab + r] = lc;
+    pos_s[st * kSlab + r] = p;
+  };
 
-  // ---- the query rows (pre-scaled): this lane's EPL dims of each
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0)
+    for (int i = 0; i < kStages - 1 && i < nslab; ++i) issue(i);
+  for (int i = 0; i < kStages - 1 && i < nslab; ++i)
+    for (int r = tid; r < kSlab; r += kThreads) meta(i, r);
+
+  // ---- the query rows (pre-scaled), this lane's EPL dims of each.  Row slot
+  // j of this lane holds query row (j ^ perm): every reduce-scatter step then
+  // keeps the low half of the live slots and sends the high half, with no
+  // per-lane selects.
+  const int perm = (li >> SHIFT) & (NQ - 1);
   float2 q2[NQ][EPL / 2];
 #pragma unroll
-  for (int r = 0; r < NQ; ++r) {
+  for (int j = 0; j < NQ; ++j) {
     float f[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) f[e] = 0.f;
-    if (ok[r]) {
+    const int r = j ^ perm;
+    bool okr = false;
+#pragma unroll
+    for (int x = 0; x < NQ; ++x)
+      if (x == r) okr = ok[x];
+    if (okr) {
       const int hq = ui.kvh * a.g + (r % a.g);
       const int64_t pi = a.seq_lens ? 0 : a.pos_lo + ui.blk * a.NP + r / a.g;
       const T* qp = static_cast<const T*>(a.q) + (((int64_t)ui.b * a.Hq + hq) * a.Tq + pi) * D;
       load_f<T, EPL>(qp + li * EPL, f);
     }
 #pragma unroll
-    for (int e = 0; e < EPL; e += 2) q2[r][e / 2] = make_float2(f[e] * a.scale, f[e + 1] * a.scale);
-  }
-  __syncthreads();
-
-  // ---- pass 1: scores.  Lanes of a row own EPL dims each; a reduce-scatter
-  // over the row's LPR lanes leaves query row h's score on lanes
-  // h * (LPR/NQ) .. (h+1) * (LPR/NQ) - 1.
-  bool ok_stage[2] = {true, true};
-  for (int base = 0; base < nrows; base += kWarps * RPI) {
-    const int row = base + warp * RPI + sub;
-    const int st = base >= n0 ? 1 : 0;
-    if (!ok_stage[st]) break;
-    if (!mbar_wait(&bar[st], 0, a.status)) {
-      ok_stage[st] = false;
-      break;
-    }
-    const bool valid = row < nrows;
-    float k[EPL];
-    if (valid) {
-      uint4 raw = *reinterpret_cast<const uint4*>(Ks + row * D + li * EPL);
-      unpack16<T>(raw, k);
-    } else {
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) k[e] = 0.f;
-    }
-    float part[NQ];
-#pragma unroll
-    for (int r = 0; r < NQ; ++r) {
-      float2 acc2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < EPL; e += 2) acc2 = ffma2(q2[r][e / 2], make_float2(k[e], k[e + 1]), acc2);
-      part[r] = acc2.x + acc2.y;
-    }
-#pragma unroll
-    for (int step = 0; step < ilog2(LPR); ++step) {
-      const int m = LPR >> (step + 1);
-      constexpr int dummy = 0;
-      (void)dummy;
-      const int n = NQ >> step;  // live values before this step
-      if (n > 1) {
-        const bool upper = (li & m) != 0;
-#pragma unroll
-        for (int i = 0; i < NQ / 2; ++i) {
-          if (i < n / 2) {
-            const float send = upper ? part[i] : part[i + n / 2];
-            const float keep = upper ? part[i + n / 2] : part[i];
-            part[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-          }
-        }
-      } else {
-        part[0] += __shfl_xor_sync(0xffffffffu, part[0], m);
-      }
-    }
-    constexpr int SHIFT = ilog2(LPR) - ilog2(NQ);
-    if (valid && (li & ((1 << SHIFT) - 1)) == 0) S_s[(li >> SHIFT) * R + row] = part[0];
-  }
-  // every thread must see both stages complete before pass 2 and before exit
-  for (int st = 0; st < 2; ++st) {
-    const bool used = st ? nrows > n0 : nrows > 0;
-    if (used && ok_stage[st] && !mbar_wait(&bar[st], 0, a.status)) ok_stage[st] = false;
-  }
-  const bool staged = ok_stage[0] && ok_stage[1];
-  __syncthreads();
-
-  // ---- per query row: max logit, and (group slices) the local top-KG
-  if (warp < NQ) {
-    const int r = warp;
-    float mx = -INFINITY;
-    for (int e = lane; e < nrows; e += 32) {
-      const bool live = ok[r] && staged && lnc_s[e] != -INFINITY && (is_group || pos_s[e] <= t_row[r]);
-      if (live) mx = fmaxf(mx, S_s[r * R + e] + lnc_s[e]);
-    }
-    mx = warp_max(mx);
-    if (lane == 0) m_s[r] = mx;
-    if (is_group) {
-      constexpr int PER = R / 32;
-      float cs[PER];
-      int cid[PER];
-#pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int e = lane + 32 * j;
-        const bool live = ok[r] && staged && e < nrows && lnc_s[e] != -INFINITY;
-        cs[j] = live ? S_s[r * R + e] : -INFINITY;
-        cid[j] = live ? (int)(lo + e) : 0x7fffffff;
-      }
-      Cand* out = reinterpret_cast<Cand*>(a.cand) + ((u * a.nsg + s) * NQ + r) * KG;
-      for (int rank = 0; rank < KG; ++rank) {
-        float bs = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < PER; ++j)
-          if (cand_better(cs[j], cid[j], bs, bi)) {
-            bs = cs[j];
-            bi = cid[j];
-          }
-        warp_best(bs, bi);
-#pragma unroll
-        for (int j = 0; j < PER; ++j)
-          if (cid[j] == bi) {
-            cs[j] = -INFINITY;
-            cid[j] = 0x7fffffff;
-          }
-        if (lane == rank) {
-          Cand c;
-          if (bi == 0x7fffffff) {
-            c.s = -INFINITY;
-            c.id = -1;
-            c.pages = 0;
-            c.cnt = 0;
-          } else {
-            const int64_t ch = bi / a.k;
-            const int j = bi % a.k;
-            const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + ch * (a.k + 1) + j;
-            c.s = bs;
-            c.id = bi;
-            c.pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
-            c.cnt = gC[bi];
-          }
-          out[rank] = c;
-        }
-      }
-    }
-  }
-  __syncthreads();
-
-  // ---- softmax weights of every (row, query row) pair
-  for (int idx = tid; idx < R * NQ; idx += kThreads) {
-    const int e = idx / NQ, r = idx % NQ;
-    float p = 0.f;
-    if (e < nrows && ok[r] && staged && lnc_s[e] != -INFINITY && (is_group || pos_s[e] <= t_row[r]))
-      p = __expf(S_s[r * R + e] + lnc_s[e] - m_s[r]);
-    P_s[e * NQ + r] = p;
-  }
-  __syncthreads();
-  if (warp < NQ) {
-    float sum = 0.f;
-    for (int e = lane; e < nrows; e += 32) sum += P_s[e * NQ + warp];
-    sum = warp_sum(sum);
-    if (lane == 0) l_s[warp] = sum;
+    for (int e = 0; e < EPL; e += 2) q2[j][e / 2] = make_float2(f[e] * a.scale, f[e + 1] * a.scale);
   }
 
-  // ---- pass 2: acc[r][:] += P[row][r] * V[row][:]
-  float2 acc[NQ][EPL / 2];
+  // running state: query row `warp` (warp < NQ) keeps (m, l) and its top-KG in lanes 0..KG-1
+  float m_run = -INFINITY, l_run = 0.f;
+  float c_s = -INFINITY;  // lane j < KG: j-th best score so far
+  int c_i = 0x7fffffff;   //                and its group id
+  float thr_s = -INFINITY;
+  int thr_i = 0x7fffffff;
+  // P.V accumulators: one value row per warp step, lane owns DPL = d/32 dims
+  constexpr int DPL = D / 32;
+  float2 acc[NQ][DPL / 2];
 #pragma unroll
   for (int r = 0; r < NQ; ++r)
 #pragma unroll
-    for (int e = 0; e < EPL / 2; ++e) acc[r][e] = make_float2(0.f, 0.f);
-  if (staged) {
-    for (int base = 0; base < nrows; base += kWarps * RPI) {
-      const int row = base + warp * RPI + sub;
-      if (row < nrows && lnc_s[row] != -INFINITY) {
-        float v[EPL];
-        uint4 raw = *reinterpret_cast<const uint4*>(Vs + row * D + li * EPL);
-        unpack16<T>(raw, v);
-        float p[NQ];
+    for (int e = 0; e < DPL / 2; ++e) acc[r][e] = make_float2(0.f, 0.f);
+  bool alive = true;  // false after a copy timed out
+
+  for (int i = 0; i < nslab && alive; ++i) {
+    const int st = i % kStages;
+    const int64_t r0 = e0 + (int64_t)i * kSlab;
+    const int n = (int)((e1 - r0) < kSlab ? (e1 - r0) : kSlab);
+    const T* Ks = Kr + (size_t)st * kSlab * D;
+    const T* Vs = Vr + (size_t)st * kSlab * D;
+    if (!mbar_wait(&full[st], (uint32_t)(i / kStages) & 1u, a.status)) alive = false;
+    // ---- scores of this slab
+    if (alive) {
 #pragma unroll
-        for (int r = 0; r < NQ; r += 4) {
-          if constexpr (NQ % 4 == 0) {
-            const float4 pp = *reinterpret_cast<const float4*>(P_s + row * NQ + r);
-            p[r] = pp.x;
-            p[r + 1] = pp.y;
-            p[r + 2] = pp.z;
-            p[r + 3] = pp.w;
-          } else {
+      for (int base = 0; base < kSlab; base += kWarps * RPI) {
+        const int row = base + warp * RPI + sub;
+        float k[EPL];
+        if (row < n) {
+          uint4 raw = *reinterpret_cast<const uint4*>(Ks + row * D + li * EPL);
+          unpack16<T>(raw, k);
+        } else {
 #pragma unroll
-            for (int x = 0; x < 4 && r + x < NQ; ++x) p[r + x] = P_s[row * NQ + r + x];
-          }
+          for (int e = 0; e < EPL; ++e) k[e] = 0.f;
+        }
+        float part[NQ];
+#pragma unroll
+        for (int j = 0; j < NQ; ++j) {
+          float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < EPL; e += 2) s2 = ffma2(q2[j][e / 2], make_float2(k[e], k[e + 1]), s2);
+          part[j] = s2.x + s2.y;
         }
 #pragma unroll
-        for (int r = 0; r < NQ; ++r)
+        for (int step = 0; step < ilog2(LPR); ++step) {
+          const int msk = LPR >> (step + 1);
+          const int live = NQ >> step;
+          if (live > 1) {
 #pragma unroll
-          for (int e = 0; e < EPL; e += 2)
-            acc[r][e / 2] = ffma2(make_float2(p[r], p[r]), make_float2(v[e], v[e + 1]), acc[r][e / 2]);
+            for (int j = 0; j < NQ / 2; ++j)
+              if (j < live / 2) part[j] += __shfl_xor_sync(0xffffffffu, part[j + live / 2], msk);
+          } else {
+            part[0] += __shfl_xor_sync(0xffffffffu, part[0], msk);
+          }
+        }
+        if (row < n && (li & ((1 << SHIFT) - 1)) == 0) S_s[perm * kSlab + row] = part[0];
       }
     }
-  }
-  // the warp's rows-per-step slices hold separate sums: fold them
+    if (!__syncthreads_and(alive)) {
+      alive = false;
+      break;
+    }
+    // the ring slot of slab i-1 is free now: stage slab i + kStages - 1
+    if (i + kStages - 1 < nslab) {
+      if (warp == 0) issue(i + kStages - 1);
+      for (int r = tid; r < kSlab; r += kThreads) meta(i + kStages - 1, r);
+    }
+    // ---- per query row: running max, weights, running sum, top-KG
+    if (warp < NQ) {
+      const int r = warp;
+      float lg[kSlab / 32], sc[kSlab / 32];
+      bool live[kSlab / 32];
+      float smax = -INFINITY;
 #pragma unroll
-  for (int m = LPR; m < 32; m <<= 1)
-#pragma unroll
-    for (int r = 0; r < NQ; ++r)
-#pragma unroll
-      for (int e = 0; e < EPL / 2; ++e) {
-        acc[r][e].x += __shfl_xor_sync(0xffffffffu, acc[r][e].x, m);
-        acc[r][e].y += __shfl_xor_sync(0xffffffffu, acc[r][e].y, m);
+      for (int x = 0; x < kSlab / 32; ++x) {
+        const int row = lane + 32 * x;
+        const float lc = row < n ? lnc_s[st * kSlab + row] : -INFINITY;
+        const int64_t p = pos_s[st * kSlab + row];
+        live[x] = ok[r] && lc != -INFINITY && (p < 0 || p <= t_row[r]);
+        sc[x] = S_s[r * kSlab + row];
+        lg[x] = live[x] ? sc[x] + lc : -INFINITY;
+        smax = fmaxf(smax, lg[x]);
       }
-  __syncthreads();  // the K stage becomes the cross-warp reduction buffer
-  if (sub == 0) {
+      smax = warp_max(smax);
+      const float mn = fmaxf(m_run, smax);
+      const float corr = (m_run == -INFINITY || mn == -INFINITY) ? (m_run == -INFINITY ? 0.f : 1.f)
+                                                                  : __expf(m_run - mn);
+      float psum = 0.f;
+#pragma unroll
+      for (int x = 0; x < kSlab / 32; ++x) {
+        const float p = live[x] ? __expf(lg[x] - mn) : 0.f;
+        P_s[(lane + 32 * x) * NQ + r] = p;
+        psum += p;
+      }
+      psum = warp_sum(psum);
+      l_run = l_run * corr + psum;
+      m_run = mn;
+      if (lane == 0) corr_s[r] = corr;
+      // top-KG by score (group rows only)
+      float ns[kSlab / 32];
+      int ni[kSlab / 32];
+#pragma unroll
+      for (int x = 0; x < kSlab / 32; ++x) {
+        const int row = lane + 32 * x;
+        const bool isg = live[x] && pos_s[st * kSlab + row] < 0;
+        ns[x] = isg ? sc[x] : -INFINITY;
+        ni[x] = isg ? (int)(r0 + row) : 0x7fffffff;
+      }
+      topk_merge<KG, kSlab / 32>(ns, ni, c_s, c_i, thr_s, thr_i);
+    }
+    __syncthreads();
+    // ---- acc[r] = acc[r] * corr[r] + P[:, r] . V   (warp w: rows w, w+8, ...)
+    float cr[NQ];
+#pragma unroll
+    for (int r = 0; r < NQ; ++r) cr[r] = corr_s[r];
 #pragma unroll
     for (int r = 0; r < NQ; ++r)
 #pragma unroll
-      for (int e = 0; e < EPL; e += 4)
-        *reinterpret_cast<float4*>(red + (warp * NQ + r) * D + li * EPL + e) =
-            make_float4(acc[r][e / 2].x, acc[r][e / 2].y, acc[r][e / 2 + 1].x, acc[r][e / 2 + 1].y);
+      for (int e = 0; e < DPL / 2; ++e) acc[r][e] = make_float2(acc[r][e].x * cr[r], acc[r][e].y * cr[r]);
+#pragma unroll 2
+    for (int row = warp; row < n; row += kWarps) {
+      if (lnc_s[st * kSlab + row] == -INFINITY) continue;
+      float v[DPL];
+      if constexpr (sizeof(T) == 2 && DPL == 4) {
+        const uint2 rw = *reinterpret_cast<const uint2*>(Vs + row * D + lane * DPL);
+        v[0] = __uint_as_float(rw.x << 16);
+        v[1] = __uint_as_float(rw.x & 0xffff0000u);
+        v[2] = __uint_as_float(rw.y << 16);
+        v[3] = __uint_as_float(rw.y & 0xffff0000u);
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) v[i] = Elem<T>::to_f(Vs[row * D + lane * DPL + i]);
+      }
+      float p[NQ];
+      if constexpr (NQ % 4 == 0) {
+#pragma unroll
+        for (int r = 0; r < NQ; r += 4) {
+          const float4 pp = *reinterpret_cast<const float4*>(P_s + row * NQ + r);
+          p[r] = pp.x;
+          p[r + 1] = pp.y;
+          p[r + 2] = pp.z;
+          p[r + 3] = pp.w;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < NQ; ++r) p[r] = P_s[row * NQ + r];
+      }
+#pragma unroll
+      for (int r = 0; r < NQ; ++r)
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2)
+          acc[r][e / 2] = ffma2(make_float2(p[r], p[r]), make_float2(v[e], v[e + 1]), acc[r][e / 2]);
+    }
+  }
+  // drain: no copy may still be in flight when the CTA exits
+  if (!alive) {
+    for (int i = 0; i < nslab && i < kStages; ++i) (void)mbar_wait(&full[i], 0, a.status);
+  }
+
+  // ---- reduce the warps' accumulators
+  __syncthreads();  // the K ring becomes the reduction buffer
+#pragma unroll
+  for (int r = 0; r < NQ; ++r)
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2)
+      *reinterpret_cast<float2*>(red + (warp * NQ + r) * D + lane * DPL + e) = acc[r][e / 2];
+  if (warp < NQ && lane == 0) {
+    corr_s[warp] = alive ? m_run : -INFINITY;
+  }
+  float* lsh = P_s;  // l per query row
+  if (warp < NQ && lane == 0) lsh[warp] = alive ? l_run : 0.f;
+  // candidates (all splits keep KG records per query row)
+  if (warp < NQ) {
+    Cand* out = reinterpret_cast<Cand*>(a.cand) + ((u * a.nsplit + s) * NQ + warp) * KG;
+    if (lane < KG) {
+      Cand c;
+      if (!alive || c_i == 0x7fffffff) {
+        c.s = -INFINITY;
+        c.id = -1;
+        c.pages = 0;
+        c.cnt = 0;
+      } else {
+        const int64_t ch = c_i / a.k;
+        const int j = c_i % a.k;
+        const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + ch * (a.k + 1) + j;
+        c.s = c_s;
+        c.id = c_i;
+        c.pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
+        c.cnt = gC[c_i];
+      }
+      out[lane] = c;
+    }
   }
   __syncthreads();
-  float* part = a.part + ((u * nsplit + s) * NQ) * (int64_t)(D + 2);
+  float* part = a.part + ((u * a.nsplit + s) * NQ) * (int64_t)(D + 2);
   for (int idx = tid; idx < NQ * (D + 2); idx += kThreads) {
     const int r = idx / (D + 2), c = idx % (D + 2);
     float v;
     if (c == 0) {
-      v = m_s[r];
+      v = corr_s[r];
     } else if (c == 1) {
-      v = l_s[r];
+      v = lsh[r];
     } else {
       v = 0.f;
 #pragma unroll
@@ -490,21 +522,68 @@ struct RefineSmem {
   static constexpr size_t off_V = 0;                                     // [kWarps][kRows][D] T
   static constexpr size_t off_perm = (size_t)kWarps * kRows * ROWB;      // int16 [kWarps][kChunk]
   static constexpr size_t off_q = off_perm + 2 * kWarps * kChunk;        // float [D]
-  static constexpr size_t off_g = off_q + sizeof(float) * D;            // float [D+2]
-  static constexpr size_t off_w = off_g + sizeof(float) * (D + 4);      // float [kWarps][D+2]
-  static constexpr size_t off_d = off_w + sizeof(float) * kWarps * (D + 4);  // float [kWarps][D+2]
-  static constexpr size_t off_c = off_d + sizeof(float) * kWarps * (D + 4);  // Cand [kMaxTopGroups]
+  static constexpr size_t off_g = off_q + sizeof(float) * D;            // float [D+4]
+  // per-warp final states reuse the value buffers (used only after the group loop)
+  static constexpr size_t off_w = off_V;                                // float [kWarps][D+4]
+  static constexpr size_t off_d = off_V + sizeof(float) * kWarps * (D + 4);  // float [kWarps][D+4]
+  static_assert(2 * sizeof(float) * kWarps * (D + 4) <= off_perm, "final states fit the value buffers");
+  static constexpr size_t off_sc = off_g + sizeof(float) * (D + 4);     // float [kWarps][64]
+  static constexpr size_t off_pos = off_sc + sizeof(float) * kWarps * 64;     // int64 [kWarps][32]
+  static constexpr size_t off_c = off_pos + sizeof(int64_t) * kWarps * 32;    // Cand [kMaxTopGroups]
   static constexpr size_t off_bar = off_c + sizeof(Cand) * kMaxTopGroups + 16;
   static constexpr size_t bytes = off_bar + 8 * kWarps + 16;
 };
 
+// Scores of up to 32 d-rows against q, loaded with coalesced 16-byte loads:
+// each half (or quarter) of the warp reads one whole row per step and the
+// row's score is reduced over its lanes.  rowptr(i) gives row i (valid for
+// i < n).  Writes score i to out[i].
+template <typename T, int D, typename RowPtr>
+__device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const float (&qv)[16 / sizeof(T)],
+                                                   float* out) {
+  constexpr int EPL = 16 / sizeof(T);
+  constexpr int LPR = D / EPL;
+  constexpr int RPI = 32 / LPR;
+  constexpr int STEPS = 8;  // loads in flight per lane per round
+  const int lane = threadIdx.x & 31;
+  const int li = lane % LPR, sub = lane / LPR;
+  for (int base = 0; base < n; base += STEPS * RPI) {
+  uint4 raw[STEPS];
+#pragma unroll
+  for (int it = 0; it < STEPS; ++it) {
+    const int i = base + it * RPI + sub;
+    if (i < n) raw[it] = __ldg(reinterpret_cast<const uint4*>(rowptr(i) + li * EPL));
+  }
+#pragma unroll
+  for (int it = 0; it < STEPS; ++it) {
+    if (base + it * RPI >= n) break;
+    const int i = base + it * RPI + sub;
+    float f[EPL];
+    if (i < n) {
+      unpack16<T>(raw[it], f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) f[e] = 0.f;
+    }
+    float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) s2 = ffma2(make_float2(qv[e], qv[e + 1]), make_float2(f[e], f[e + 1]), s2);
+    float sc = s2.x + s2.y;
+#pragma unroll
+    for (int msk = LPR / 2; msk > 0; msk >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, msk);
+    if (li == 0 && i < n) out[i] = sc;
+  }
+  }
+}
+
 template <typename T, int D, int NQ, int KG>
 __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   constexpr int DPL = D / 32;
+  constexpr int EPL = 16 / sizeof(T);
+  constexpr int LPR = D / EPL;
   constexpr int ROWB = D * sizeof(T);
   using SM = RefineSmem<T, D>;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nsplit = a.nsg + a.nsw;
   const int64_t npos = a.seq_lens ? 1 : a.pos_hi - a.pos_lo;
   const int64_t row = blockIdx.x;
   const int b = (int)(row / (a.Hq * npos));
@@ -533,6 +612,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   float* gstate = reinterpret_cast<float*>(smem + SM::off_g);
   float* wstate = reinterpret_cast<float*>(smem + SM::off_w);
   float* dstate = reinterpret_cast<float*>(smem + SM::off_d);
+  float* sc_s = reinterpret_cast<float*>(smem + SM::off_sc);
+  int64_t* posm_s = reinterpret_cast<int64_t*>(smem + SM::off_pos);
   Cand* win = reinterpret_cast<Cand*>(smem + SM::off_c);
   int* nwin_s = reinterpret_cast<int*>(smem + SM::off_c + sizeof(Cand) * kMaxTopGroups);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM::off_bar);
@@ -559,10 +640,11 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   if (tid == 0) fence_mbar_init();
   pdl_wait();  // the scan's partial states and candidates are visible from here on
 
-  // ---- global top-G over the group splits' candidates (warp 0)
+  const int nsplit = a.nsplit;
+  // ---- global top-G over the splits' candidates (warp 0)
   if (warp == 0) {
-    const int ncand = a.nsg * KG;
-    const Cand* src = reinterpret_cast<const Cand*>(a.cand) + (u * a.nsg * NQ) * (int64_t)KG;
+    const int ncand = nsplit * KG;
+    const Cand* src = reinterpret_cast<const Cand*>(a.cand) + (u * nsplit * NQ) * (int64_t)KG;
     float lastS = INFINITY;
     int lastI = -1;
     int nwin = 0;
@@ -571,15 +653,15 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       int bi = 0x7fffffff, bidx = -1;
       for (int e = lane; e < ncand; e += 32) {
         const int sp = e / KG, j = e % KG;
-        const Cand* c = src + ((int64_t)sp * NQ + r) * KG + j;
-        const int id = c->id;
+        const int64_t off = ((int64_t)sp * NQ + r) * KG + j;
+        const int id = src[off].id;
         if (id < 0) continue;
-        const float sc = c->s;
+        const float sc = src[off].s;
         const bool after = rank == 0 || cand_better(lastS, lastI, sc, id);
         if (after && cand_better(sc, id, bs, bi)) {
           bs = sc;
           bi = id;
-          bidx = (int)(((int64_t)sp * NQ + r) * KG + j);
+          bidx = (int)off;
         }
       }
       float ws_ = bs;
@@ -615,6 +697,11 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   const int nwin = *nwin_s;
   const float M = gstate[0];
 
+  // this lane's slice of q in the coalesced layout (dims (lane % LPR) * EPL ..)
+  float qv[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) qv[e] = qs[(lane % LPR) * EPL + e];
+
   // ---- per opened group (warp w: groups w, w + 8, ...)
   float m = -INFINITY, l = 0.f, acc[DPL];
   float dl = 0.f, dacc[DPL];  // the opened groups' coarse terms, to remove (relative to M)
@@ -630,7 +717,73 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   const T* Vb = static_cast<const T*>(a.V) + b * a.sb + kvh * a.sh;
   T* myV = Vst + warp * SM::kRows * D;
   int16_t* myperm = perm_s + warp * kChunk;
+  float* mysc = sc_s + warp * 64;
+  int64_t* mypos = posm_s + warp * 32;
   uint32_t phase = 0;
+  // One batch of up to 32 exact tokens (lane e: `ev`, position `pos`) and up
+  // to 32 coarse entries (lane p: `cvb`, logit `lgc`, value row `crow`): the
+  // value rows are staged in shared memory by TMA while the key rows are
+  // scored with coalesced loads, then everything enters the warp's online
+  // softmax state.
+  auto batch = [&](bool ev, int64_t pos, bool cvb, float lgc, const T* crow) {
+    const unsigned vm = __ballot_sync(0xffffffffu, ev);
+    const unsigned cmb = __ballot_sync(0xffffffffu, cvb);
+    if (!(vm | cmb)) return;
+    if (lane == 0) mbar_arrive_expect(&bar[warp], (uint32_t)(__popc(vm) + __popc(cmb)) * ROWB);
+    __syncwarp();
+    if (ev) bulk_g2s(myV + lane * D, Vb + pos * a.st, ROWB, &bar[warp]);
+    if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
+    // members are packed: lanes 0..nvalid-1 hold the valid ones in order
+    const int nvalid = __popc(vm);
+    const int my_rank = __popc(vm & ((1u << lane) - 1u));
+    if (ev) mypos[my_rank] = pos;
+    __syncwarp();
+    rows_dot_coalesced<T, D>(nvalid, [&](int i) { return Kb + mypos[i] * a.st; }, qv, mysc + 32);
+    __syncwarp();
+    const float lge = ev ? mysc[32 + my_rank] : -INFINITY;
+    const float lgcb = cvb ? lgc : -INFINITY;
+    const float bm = warp_max(fmaxf(lge, lgcb));
+    const float mn = fmaxf(m, bm);
+    const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    const float pe = ev ? __expf(lge - mn) : 0.f;
+    const float pc = cvb ? __expf(lgcb - mn) : 0.f;
+    l = l * corr + warp_sum(pe + pc);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] *= corr;
+    m = mn;
+    const bool okw = mbar_wait(&bar[warp], phase, a.status);
+    phase ^= 1u;
+    if (!okw) {
+      (void)mbar_wait(&bar[warp], phase ^ 1u, a.status);  // drain before the buffer is reused
+      __syncwarp();
+      return;
+    }
+    for (int j = 0; j < 64; ++j) {
+      const bool on = j < 32 ? ((vm >> j) & 1u) : ((cmb >> (j - 32)) & 1u);
+      if (!on) continue;
+      const float pj = __shfl_sync(0xffffffffu, j < 32 ? pe : pc, j & 31);
+      float v[DPL];
+      if constexpr (sizeof(T) == 2 && DPL == 4) {
+        const uint2 rw = *reinterpret_cast<const uint2*>(myV + j * D + lane * DPL);
+        v[0] = __uint_as_float(rw.x << 16);
+        v[1] = __uint_as_float(rw.x & 0xffff0000u);
+        v[2] = __uint_as_float(rw.y << 16);
+        v[3] = __uint_as_float(rw.y & 0xffff0000u);
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) v[i] = Elem<T>::to_f(myV[j * D + lane * DPL + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, v[i], acc[i]);
+    }
+    __syncwarp();
+  };
+  // the sink tokens [0, min(sinks, window start)) are exact entries (last warp)
+  if (warp == kWarps - 1) {
+    const int64_t wsq = (t / kChunk - a.window / kChunk + 1) > 0 ? (t / kChunk - a.window / kChunk + 1) * kChunk : 0;
+    const int64_t nsk = a.sinks < wsq ? a.sinks : wsq;
+    for (int64_t e0 = 0; e0 < nsk; e0 += 32) batch(e0 + lane < nsk, e0 + lane, false, 0.f, pV);
+  }
   for (int w = warp; w < nwin; w += kWarps) {
     const Cand cw = win[w];
     const int64_t c = cw.id / a.k;
@@ -653,23 +806,24 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       if (lane == 0) set_status(a.status, LOD_ST_BAD_PAGE);
     } else {
       const int np = p1 - p0;
-      // the chunk's member list, and lane p's page summary score
+      // the chunk's member list, page counts/offsets, and the page summary scores
       *reinterpret_cast<uint4*>(myperm + lane * 8) =
           __ldg(reinterpret_cast<const uint4*>(pm + c * kChunk) + lane);
-      float sc = -INFINITY;
       int cntp = 0, begp = 0;
       if (lane < np) {
         cntp = pC[c * a.P + p0 + lane];
         begp = pB[c * a.P + p0 + lane];
-        sc = row_dot<T, D>(pK + (c * a.P + p0 + lane) * D, qs);
       }
+      const T* pKc = pK + (c * a.P + p0) * D;
+      rows_dot_coalesced<T, D>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
       __syncwarp();
+      const float sc = lane < np ? mysc[lane] : -INFINITY;
       // top-TP pages by (score desc, slot asc)
       float s2 = sc;
       int sl2 = lane < np ? p0 + lane : 0x7fffffff;
       int nopen = 0;
       for (int x = 0; x < a.TP && x < np; ++x) {
-        float bs = s2;  // (the chunk-member list is in shared memory after the __syncwarp above)
+        float bs = s2;
         int bi = sl2;
         warp_best(bs, bi);
         open_slot[x] = bi;
@@ -709,54 +863,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
           set_status(a.status, LOD_ST_BAD_MEMBER);
           ev = false;
         }
-        const int64_t pos = c * kChunk + off;
-        const bool cvb = bt == 0 && cv;
-        const unsigned vm = __ballot_sync(0xffffffffu, ev);
-        const unsigned cmb = bt == 0 ? cm : 0u;
-        // value rows (exact tokens and coarse page means) go to shared memory by
-        // TMA while the key rows are dotted in registers
-        if (lane == 0 && (vm | cmb)) mbar_arrive_expect(&bar[warp], (uint32_t)(__popc(vm) + __popc(cmb)) * ROWB);
-        __syncwarp();
-        if (ev) bulk_g2s(myV + lane * D, Vb + pos * a.st, ROWB, &bar[warp]);
-        if (cvb) bulk_g2s(myV + (32 + lane) * D, pV + (c * a.P + p0 + lane) * D, ROWB, &bar[warp]);
-        const float lge = ev ? row_dot<T, D>(Kb + pos * a.st, qs) : -INFINITY;
-        const float lgcb = cvb ? lgc : -INFINITY;
-        const float bm = warp_max(fmaxf(lge, lgcb));
-        if (bm == -INFINITY) continue;  // nothing staged in this batch
-        const float mn = fmaxf(m, bm);
-        const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
-        const float pe = ev ? __expf(lge - mn) : 0.f;
-        const float pc = cvb ? __expf(lgcb - mn) : 0.f;
-        l = l * corr + warp_sum(pe + pc);
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] *= corr;
-        m = mn;
-        const bool okw = mbar_wait(&bar[warp], phase, a.status);
-        phase ^= 1u;
-        if (!okw) {
-          (void)mbar_wait(&bar[warp], phase ^ 1u, a.status);  // drain before the buffer is reused
-          __syncwarp();
-          continue;
-        }
-        for (int j = 0; j < 64; ++j) {
-          const bool on = j < 32 ? ((vm >> j) & 1u) : ((cmb >> (j - 32)) & 1u);
-          if (!on) continue;
-          const float pj = __shfl_sync(0xffffffffu, j < 32 ? pe : pc, j & 31);
-          float v[DPL];
-          if constexpr (sizeof(T) == 2 && DPL == 4) {
-            const uint2 rw = *reinterpret_cast<const uint2*>(myV + j * D + lane * DPL);
-            v[0] = __uint_as_float(rw.x << 16);
-            v[1] = __uint_as_float(rw.x & 0xffff0000u);
-            v[2] = __uint_as_float(rw.y << 16);
-            v[3] = __uint_as_float(rw.y & 0xffff0000u);
-          } else {
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) v[i] = Elem<T>::to_f(myV[j * D + lane * DPL + i]);
-          }
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, v[i], acc[i]);
-        }
-        __syncwarp();
+        batch(ev, c * kChunk + off, bt == 0 && cv, lgc, pV + (c * a.P + p0 + lane) * D);
       }
     }
     if (a.sel_pages && lane < a.TP) {
@@ -769,6 +876,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   }
 
   // ---- final merge: scan state (max M) + per-warp fine states + removals
+  // (the value staging buffers are free now and hold the per-warp states)
+  __syncthreads();
   float* ws_ = wstate + warp * (D + 4);
   float* ds_ = dstate + warp * (D + 4);
   if (lane == 0) {
@@ -812,18 +921,24 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 }
 
 template <typename T, int D, int NQ, int KG>
-cudaError_t launch_t(const AttendArgs& a, cudaStream_t stream) {
-  const int nsplit = a.nsg + a.nsw;
+cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t stream) {
+  const int nsplit = a.nsplit;
   const int64_t npos = a.seq_lens ? 1 : a.pos_hi - a.pos_lo;
   const int64_t rows = (int64_t)a.B * a.Hq * npos;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   if (a.units > 0 && nsplit > 0) {
-    auto sk = scan_kernel<T, D, NQ, KG>;
-    const size_t smem = ScanSmem<T, D, NQ>::bytes;
-    e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    sk<<<dim3((unsigned)a.units, (unsigned)nsplit), kThreads, smem, stream>>>(a);
-    e = cudaGetLastError();
+    if (maps) {
+      e = launch_scan_tc(a, *maps, NQ, stream);
+    } else if constexpr (NQ <= 8) {
+      auto sk = scan_kernel<T, D, NQ, KG>;
+      const size_t smem = ScanSmem<T, D, NQ>::bytes;
+      e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      sk<<<dim3((unsigned)a.units, (unsigned)nsplit), kThreads, smem, stream>>>(a);
+      e = cudaGetLastError();
+    } else {
+      return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
   }
   if (rows > 0) {
@@ -847,17 +962,23 @@ cudaError_t launch_t(const AttendArgs& a, cudaStream_t stream) {
 }
 
 template <typename T, int D, int NQ>
-cudaError_t launch_kg(const AttendArgs& a, cudaStream_t stream) {
-  return a.G <= 8 ? launch_t<T, D, NQ, 8>(a, stream) : launch_t<T, D, NQ, 16>(a, stream);
+cudaError_t launch_kg(const AttendArgs& a, const TcMaps* maps, cudaStream_t stream) {
+  return a.G <= 8 ? launch_t<T, D, NQ, 8>(a, maps, stream) : launch_t<T, D, NQ, 16>(a, maps, stream);
 }
 
 template <typename T, int D>
-cudaError_t launch_nq(const AttendArgs& a, int NQ, cudaStream_t stream) {
+cudaError_t launch_nq(const AttendArgs& a, int NQ, const TcMaps* maps, cudaStream_t stream) {
   switch (NQ) {
-    case 1: return launch_kg<T, D, 1>(a, stream);
-    case 2: return launch_kg<T, D, 2>(a, stream);
-    case 4: return launch_kg<T, D, 4>(a, stream);
-    case 8: return launch_kg<T, D, 8>(a, stream);
+    case 1: return launch_kg<T, D, 1>(a, maps, stream);
+    case 2: return launch_kg<T, D, 2>(a, maps, stream);
+    case 4: return launch_kg<T, D, 4>(a, maps, stream);
+    case 8: return launch_kg<T, D, 8>(a, maps, stream);
+    case 16:
+      // sixteen query rows per unit exist only on the tensor-core scan
+      if constexpr (sizeof(T) == 2 && D == 128) {
+        if (maps) return launch_kg<T, D, 16>(a, maps, stream);
+      }
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -866,11 +987,12 @@ cudaError_t launch_nq(const AttendArgs& a, int NQ, cudaStream_t stream) {
 
 size_t cand_bytes() { return sizeof(Cand); }
 
-cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, cudaStream_t stream) {
+cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, const TcMaps* maps,
+                          cudaStream_t stream) {
   if (dtype == LOD_DTYPE_F32)
-    return d == 64 ? launch_nq<float, 64>(a, NQ, stream) : launch_nq<float, 128>(a, NQ, stream);
-  return d == 64 ? launch_nq<__nv_bfloat16, 64>(a, NQ, stream)
-                 : launch_nq<__nv_bfloat16, 128>(a, NQ, stream);
+    return d == 64 ? launch_nq<float, 64>(a, NQ, nullptr, stream) : launch_nq<float, 128>(a, NQ, nullptr, stream);
+  return d == 64 ? launch_nq<__nv_bfloat16, 64>(a, NQ, nullptr, stream)
+                 : launch_nq<__nv_bfloat16, 128>(a, NQ, maps, stream);
 }
 
 }  // namespace lod

@@ -2,6 +2,8 @@
 // translation units (not part of the public ABI).
 #pragma once
 
+#include <cuda.h>
+
 #include "lod_common.cuh"
 
 namespace lod {
@@ -29,8 +31,10 @@ struct BuildArgs {
   int16_t* perm;
 };
 
-// Rows streamed by one scan CTA.
-constexpr int kScanRows = 128;
+// Scan CTAs a decode call aims for: two resident CTAs on each of the B200's 148 SMs.
+constexpr int kTargetCtas = 2 * 148;
+// Rows of one scan pipeline stage (a split streams whole stages).
+constexpr int kScanSlab = 64;
 
 // A batch of query rows handled by one scan/refine launch pair.
 //  decode:  unit = (b, kvh); the unit's NQ = g rows are its query heads, all
@@ -60,10 +64,10 @@ struct AttendArgs {
   int64_t Tmax, Cmax;
   int k, P, G, TP, window, sinks;
   float scale;
-  int nsg, nsw;             // group splits and window splits per unit
+  int nsplit;               // splits of each unit's row list (groups, sinks, window)
   int64_t units;            // scan units in this launch
-  float* part;              // [units][nsg+nsw][NQ][d+2]  (m, l, acc)
-  void* cand;               // [units][nsg][NQ][KG] candidate records (cand_bytes() each)
+  float* part;              // [units][nsplit][NQ][d+2]  (m, l, acc)
+  void* cand;               // [units][nsplit][NQ][KG] candidate records (cand_bytes() each)
   void* out;                // [B][Hq][Tq][d]
   float* lse;               // [B][Hq][Tq] or null
   int32_t* sel_groups;      // [B][Hq][Tq][G] or null
@@ -71,9 +75,20 @@ struct AttendArgs {
   uint32_t* status;
 };
 
+// TMA tensor maps of the tensor-core scan: group summaries (2-D, rows x d)
+// and the KV cache (4-D, d x t x kv-head x sequence), 64 x 128 boxes, 128B swizzle.
+struct __align__(64) TcMaps {
+  CUtensorMap gK, gV, K, V;
+};
+
 cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
                          cudaStream_t stream);
-cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, cudaStream_t stream);
+// maps == nullptr selects the CUDA-core scan; otherwise bf16, d = 128 run the
+// tensor-core scan.
+cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, const TcMaps* maps,
+                          cudaStream_t stream);
+cudaError_t launch_scan_tc(const AttendArgs& a, const TcMaps& maps, int NQ, cudaStream_t stream);
+size_t scan_tc_smem_bytes();
 size_t cand_bytes();
 
 }  // namespace lod

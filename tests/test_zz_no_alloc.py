@@ -32,12 +32,12 @@ def _call(L, p, q, Kd, Vd, st, sl, ix, out, lse, sg, sp, status=None):
 
 def test_shapes_beyond_the_built_in_scratch_are_rejected_without_touching_a_gpu():
     L = _lib.load()
-    # 64 sequences x 8 KV heads at 1M tokens need far more than the built-in array
-    p = api.Params(B=64, Hq=64, Hkv=8, d=128, Tmax=1 << 20)
+    # 512 sequences x 8 KV heads need more split states than the built-in array holds
+    p = api.Params(B=512, Hq=64, Hkv=8, d=128, Tmax=1 << 20)
     assert api.workspace_bytes(p, _lib.LOD_OP_DECODE) > _lib.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(1 << 20)
     full = _lib.lod_index(*([1 << 20] * 9))
-    st = (ctypes.c_int64 * 3)(8 * (1 << 20) * 128, (1 << 20) * 128, 128)
+    st = (ctypes.c_int64 * 3)(8 * (1 << 20) * 128, (1 << 20) * 128, 128)  # fake, never used
     rc = L.lod_decode_noalloc(ctypes.byref(p.c()), fake, fake, fake, st, fake, ctypes.byref(full), fake,
                               None, None, None, None, None)
     assert rc == _lib.LOD_EINVAL
