@@ -145,7 +145,7 @@ AttendShape decode_shape(const lod_params* p) {
 AttendShape prefill_shape(const lod_params* p) {
   AttendShape s;
   s.tc = use_tc(p);
-  s.NP = (s.tc ? 16 : nq_max(p)) / g_of(p);
+  s.NP = nq_max(p) / g_of(p);
   s.NQ = s.NP * g_of(p);
   s.units = (int64_t)p->B * p->Hkv * cdiv(p->chunk, s.NP);
   s.nsplit = split_for(p, s.tc, s.units, max_rows(p));

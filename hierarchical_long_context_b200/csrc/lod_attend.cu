@@ -758,9 +758,10 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       __syncwarp();
       return;
     }
-    for (int j = 0; j < 64; ++j) {
-      const bool on = j < 32 ? ((vm >> j) & 1u) : ((cmb >> (j - 32)) & 1u);
-      if (!on) continue;
+    unsigned long long rest = (unsigned long long)vm | ((unsigned long long)cmb << 32);
+    while (rest) {
+      const int j = __ffsll((long long)rest) - 1;
+      rest &= rest - 1;
       const float pj = __shfl_sync(0xffffffffu, j < 32 ? pe : pc, j & 31);
       float v[DPL];
       if constexpr (sizeof(T) == 2 && DPL == 4) {
@@ -973,12 +974,6 @@ cudaError_t launch_nq(const AttendArgs& a, int NQ, const TcMaps* maps, cudaStrea
     case 2: return launch_kg<T, D, 2>(a, maps, stream);
     case 4: return launch_kg<T, D, 4>(a, maps, stream);
     case 8: return launch_kg<T, D, 8>(a, maps, stream);
-    case 16:
-      // sixteen query rows per unit exist only on the tensor-core scan
-      if constexpr (sizeof(T) == 2 && D == 128) {
-        if (maps) return launch_kg<T, D, 16>(a, maps, stream);
-      }
-      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }

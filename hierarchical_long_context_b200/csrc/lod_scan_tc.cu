@@ -48,7 +48,9 @@ struct TcSmem {
   static constexpr size_t off_S = off_P + 2 * N * 128;                  // float [16][128] scores
   static constexpr size_t off_lnc = off_S + sizeof(float) * N * TROWS;  // float [128]
   static constexpr size_t off_corr = off_lnc + sizeof(float) * TROWS;   // float [16]
-  static constexpr size_t off_bar = off_corr + sizeof(float) * N;       // uint64 [kTcStages + 2]
+  static constexpr size_t off_pmax = off_corr + sizeof(float) * N;      // float [2][16] pair maxima
+  static constexpr size_t off_meta = off_pmax + sizeof(float) * 2 * N;  // int [2][128]: count, page range
+  static constexpr size_t off_bar = off_meta + sizeof(int) * 2 * TROWS;  // uint64 [kTcStages + 2]
   static constexpr size_t off_tmem = off_bar + 8 * (kTcStages + 2);
   static constexpr size_t bytes = off_tmem + 16 + 1024;  // + alignment slack
 };
@@ -63,7 +65,7 @@ struct Cand {
 template <int NQ, int KG>
 __global__ void __launch_bounds__(kTcThreads, 1)
     scan_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ AttendArgs a) {
-  static_assert(NQ <= N, "query rows per unit");
+  static_assert(NQ <= 8, "query rows per unit (two warps per row)");
   const int64_t u = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -78,6 +80,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* S_s = reinterpret_cast<float*>(sm + TcSmem::off_S);
   float* lnc_s = reinterpret_cast<float*>(sm + TcSmem::off_lnc);
   float* corr_s = reinterpret_cast<float*>(sm + TcSmem::off_corr);
+  float* pmax_s = reinterpret_cast<float*>(sm + TcSmem::off_pmax);
+  int* cnt_s = reinterpret_cast<int*>(sm + TcSmem::off_meta);      // group size of row r
+  int* pgs_s = cnt_s + TROWS;                                      // page range of row r
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + TcSmem::off_bar);
   uint64_t* bar_s = full + kTcStages;
   uint64_t* bar_o = full + kTcStages + 1;
@@ -133,33 +138,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int64_t grow0 = unit_kv * a.Cmax * a.k;  // this unit's first summary row
   const int32_t* gC = a.gCnt + grow0;
 
-  // ---- set-up: barriers, TMEM, the query operand
+  // ---- set-up: barriers, first tiles in flight, TMEM, the query operand
   if (tid == 0) {
     for (int i = 0; i < kTcStages + 2; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
-  if (warp == 0) tc::tmem_alloc(tmem_slot, 32);
-  for (int i = tid; i < N * D; i += kTcThreads) {
-    const int r = i / D, c = i % D;
-    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
-    bool okr = false;
-#pragma unroll
-    for (int x = 0; x < NQ; ++x)
-      if (x == r) okr = ok[x];
-    if (r < NQ && okr) {
-      const int hq = kvh * a.g + (r % a.g);
-      const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
-      v = static_cast<const __nv_bfloat16*>(a.q)[(((int64_t)b * a.Hq + hq) * a.Tq + pi) * D + c];
-    }
-    *reinterpret_cast<__nv_bfloat16*>(Qs + tc::sw128_offset(r, c, N)) = v;
-    *reinterpret_cast<__nv_bfloat16*>(Ps + tc::sw128_offset(r, c, N)) = __float2bfloat16_rn(0.f);
-  }
-  tc::fence_proxy_async();
-  tc::fence_before_sync();
   __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-
   auto issue = [&](int i) {  // by thread 0: tile t0 + i into ring slot i % kTcStages
     const int st = i % kTcStages;
     const int64_t tile = t0 + i;
@@ -182,14 +166,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
   if (tid == 0)
     for (int i = 0; i < kTcStages - 1 && i < ntile; ++i) issue(i);
+  if (warp == 0) tc::tmem_alloc(tmem_slot, 32);
+  // the query rows, 16-byte chunks into the swizzled K-major layout; P zeroed
+  if (tid < N * (D / 8)) {
+    const int r = tid / (D / 8), c = tid % (D / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    bool okr = false;
+#pragma unroll
+    for (int x = 0; x < NQ; ++x)
+      if (x == r) okr = ok[x];
+    if (r < NQ && okr) {
+      const int hq = kvh * a.g + (r % a.g);
+      const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
+      v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
+    }
+    const uint32_t off = (uint32_t)((c >> 3) * (N * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+    *reinterpret_cast<uint4*>(Qs + off) = v;
+    *reinterpret_cast<uint4*>(Ps + off) = make_uint4(0, 0, 0, 0);
+  }
+  tc::fence_proxy_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
 
-  // running state: warp j owns query row j -- (m, l) and its top-KG list
-  // (lane k < KG holds entry k)
-  float m_run = -INFINITY, l_run = 0.f, c_s = -INFINITY, thr_s = -INFINITY;
-  int c_i = 0x7fffffff, thr_i = 0x7fffffff;
+  // running state: query row j is shared by warps j and j + 8, each taking 64
+  // rows of every tile; each keeps (m, l) over its rows (m is common to the
+  // pair).  Every lane keeps a private sorted top-KG of the group rows it sees
+  // (score, id, page range, count); the lists are merged once, at the end.
+  float m_run = -INFINITY, l_run = 0.f;
+  float ls[KG];
+  int lid[KG], lpg[KG], lcn[KG];
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    ls[k] = -INFINITY;
+    lid[k] = 0x7fffffff;
+    lpg[k] = lcn[k] = 0;
+  }
   const int quad = warp & 3, cgrp = warp >> 2;  // TMEM lane quadrant, column group
-  int cnt_next = 0;  // row `tid` (< 128) count in the next group tile
-  if (ntile > 0 && t0 < gt && tid < TROWS && tid < (int)(G_vis - t0 * TROWS)) cnt_next = gC[t0 * TROWS + tid];
+  // row `tid` (< 128) of the next group tile: count and page range, prefetched
+  const int16_t* gP = a.gPage + unit_kv * a.Cmax * (a.k + 1);
+  auto fetch_meta = [&](int64_t tile, int& cnt, int& pg) {
+    cnt = 0;
+    pg = 0;
+    if (tile < gt && tid < TROWS && tile * TROWS + tid < G_vis) {
+      const int64_t gid = tile * TROWS + tid;
+      cnt = gC[gid];
+      const int16_t* gp = gP + (gid / a.k) * (a.k + 1) + gid % a.k;
+      pg = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
+    }
+  };
+  int cnt_next = 0, pg_next = 0;
+  if (ntile > 0) fetch_meta(t0, cnt_next, pg_next);
   float acc[4];  // dim 32 quad + lane, query rows 4 cgrp .. +3
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j] = 0.f;
@@ -204,9 +233,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nvalid = (int)((is_group ? G_vis : ws + wn) - r0 < TROWS ? (is_group ? G_vis : ws + wn) - r0 : TROWS);
     if (tid == 0 && i + kTcStages - 1 < ntile) issue(i + kTcStages - 1);
     // row metadata (log count; -inf = not a row); counts of the next tile prefetched
-    const int cnt = cnt_next;
-    if (i + 1 < ntile && t0 + i + 1 < gt && tid < TROWS && tid < (int)(G_vis - (t0 + i + 1) * TROWS))
-      cnt_next = gC[(t0 + i + 1) * TROWS + tid];
+    const int cnt = cnt_next, pg = pg_next;
+    if (i + 1 < ntile) fetch_meta(t0 + i + 1, cnt_next, pg_next);
     float lc = -INFINITY;
     if (tid < nvalid) {
       if (is_group) {
@@ -216,7 +244,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         lc = 0.f;
       }
     }
-    if (tid < TROWS) lnc_s[tid] = lc;
+    if (tid < TROWS) {
+      lnc_s[tid] = lc;
+      cnt_s[tid] = cnt;
+      pgs_s[tid] = pg;
+    }
     if (!mbar_wait(&full[st], (uint32_t)(i / kTcStages) & 1u, a.status)) alive = false;
     // a row that is not part of the softmax must not feed NaN/Inf into MMA 2
     if (alive && tid < TROWS && lc == -INFINITY) {
@@ -255,9 +287,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < 4; ++c) S_s[(4 * cgrp + c) * TROWS + 32 * quad + lane] = sv[c] * a.scale;
     }
     __syncthreads();
-    // ---- query row j = warp: tile max, weights, running sum, top-KG
-    if (warp < NQ) {
-      const int j = warp;
+    // ---- query row j (warps j and j + 8, 64 rows each): tile max, weights, sums, top-KG
+    if ((warp & 7) < NQ) {
+      const int j = warp & 7, half = warp >> 3;
       bool okj = false;
       int64_t tj = 0;
 #pragma unroll
@@ -266,11 +298,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           okj = ok[y];
           tj = t_row[y];
         }
-      float sc[TROWS / 32], lg[TROWS / 32];
+      float sc[2], lg[2];
       float tmx = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < TROWS / 32; ++q) {
-        const int row = lane + 32 * q;
+      for (int q = 0; q < 2; ++q) {
+        const int row = 64 * half + lane + 32 * q;
         const float lcr = lnc_s[row];
         const bool live = okj && lcr != -INFINITY && (is_group || r0 + row <= tj);
         sc[q] = S_s[j * TROWS + row];
@@ -278,12 +310,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmx = fmaxf(tmx, lg[q]);
       }
       tmx = warp_max(tmx);
+      if (lane == 0) pmax_s[half * N + j] = tmx;
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + j) : "memory");  // the pair of warps of row j
+      tmx = fmaxf(pmax_s[j], pmax_s[N + j]);
       const float mn = fmaxf(m_run, tmx);
       const float corr = m_run == -INFINITY ? 0.f : (mn == -INFINITY ? 1.f : __expf(m_run - mn));
       float psum = 0.f;
 #pragma unroll
-      for (int q = 0; q < TROWS / 32; ++q) {
-        const int row = lane + 32 * q;
+      for (int q = 0; q < 2; ++q) {
+        const int row = 64 * half + lane + 32 * q;
         const float p = lg[q] == -INFINITY ? 0.f : __expf(lg[q] - mn);
         psum += p;
         *reinterpret_cast<__nv_bfloat16*>(Ps + tc::sw128_offset(j, row, N)) = __float2bfloat16_rn(p);
@@ -291,17 +326,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       psum = warp_sum(psum);
       l_run = l_run * corr + psum;
       m_run = mn;
-      if (lane == 0) corr_s[j] = corr;
+      if (lane == 0 && half == 0) corr_s[j] = corr;
       if (is_group) {
-        float ns[TROWS / 32];
-        int ni[TROWS / 32];
 #pragma unroll
-        for (int q = 0; q < TROWS / 32; ++q) {
-          const bool live = lg[q] != -INFINITY;
-          ns[q] = live ? sc[q] : -INFINITY;
-          ni[q] = live ? (int)(r0 + lane + 32 * q) : 0x7fffffff;
+        for (int q = 0; q < 2; ++q) {
+          const int row = 64 * half + lane + 32 * q;
+          float ns = lg[q] != -INFINITY ? sc[q] : -INFINITY;
+          int ni = (int)(r0 + row);
+          if (ns != -INFINITY && cand_better(ns, ni, ls[KG - 1], lid[KG - 1])) {
+            int np = pgs_s[row], nc = cnt_s[row];
+#pragma unroll
+            for (int k = 0; k < KG; ++k) {
+              if (cand_better(ns, ni, ls[k], lid[k])) {
+                const float ts = ls[k];
+                const int ti = lid[k], tp = lpg[k], tcn = lcn[k];
+                ls[k] = ns;
+                lid[k] = ni;
+                lpg[k] = np;
+                lcn[k] = nc;
+                ns = ts;
+                ni = ti;
+                np = tp;
+                nc = tcn;
+              }
+            }
+          }
         }
-        topk_merge<KG, TROWS / 32>(ns, ni, c_s, c_i, thr_s, thr_i);
       }
     }
     tc::fence_proxy_async();  // the weights feed MMA 2 through the async proxy
@@ -346,29 +396,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int j = 4 * cgrp + c;
     if (j < NQ) part[j * (D + 2) + 2 + 32 * quad + lane] = alive ? acc[c] : 0.f;
   }
+  // each query warp merges its lanes' lists (KG rounds of warp argmax over the
+  // list heads); the second warp of each pair hands sum and list to the first
+  float c_s = -INFINITY;
+  int c_i = 0x7fffffff, c_pg = 0, c_cn = 0;
+  if ((warp & 7) < NQ) {
+    for (int k = 0; k < KG; ++k) {
+      float bs = ls[0];
+      int bi = lid[0];
+      warp_best(bs, bi);
+      const unsigned who = __ballot_sync(0xffffffffu, lid[0] == bi && bi != 0x7fffffff);
+      const int src = who ? __ffs(who) - 1 : 0;
+      const int bp = __shfl_sync(0xffffffffu, lpg[0], src);
+      const int bc = __shfl_sync(0xffffffffu, lcn[0], src);
+      if (lane == k) {
+        c_s = bs;
+        c_i = bi;
+        c_pg = bp;
+        c_cn = bc;
+      }
+      if (who && lane == src) {  // pop the winner's head
+#pragma unroll
+        for (int x = 0; x + 1 < KG; ++x) {
+          ls[x] = ls[x + 1];
+          lid[x] = lid[x + 1];
+          lpg[x] = lpg[x + 1];
+          lcn[x] = lcn[x + 1];
+        }
+        ls[KG - 1] = -INFINITY;
+        lid[KG - 1] = 0x7fffffff;
+      }
+    }
+  }
+  float* xl = S_s;                                         // float [16] sums
+  float* xs = S_s + N;                                     // float [16][KG] scores
+  int* xi = reinterpret_cast<int*>(S_s + N + N * KG);      // int   [16][KG] ids
+  int* xp = xi + N * KG;                                   // int   [16][KG] page ranges
+  int* xc = xp + N * KG;                                   // int   [16][KG] counts
+  __syncthreads();
+  if (warp >= 8 && (warp & 7) < NQ) {
+    const int j = warp & 7;
+    if (lane == 0) xl[j] = l_run;
+    if (lane < KG) {
+      xs[j * KG + lane] = c_s;
+      xi[j * KG + lane] = c_i;
+      xp[j * KG + lane] = c_pg;
+      xc[j * KG + lane] = c_cn;
+    }
+  }
+  __syncthreads();
   if (warp < NQ) {
     const int j = warp;
+    // the two sorted lists sit in lanes 0..KG-1 (this warp) and KG..2KG-1 (partner)
+    float hs = c_s;
+    int hi = c_i, hp = c_pg, hc = c_cn;
+    if (lane >= KG && lane < 2 * KG) {
+      hs = xs[j * KG + lane - KG];
+      hi = xi[j * KG + lane - KG];
+      hp = xp[j * KG + lane - KG];
+      hc = xc[j * KG + lane - KG];
+    } else if (lane >= 2 * KG) {
+      hs = -INFINITY;
+      hi = 0x7fffffff;
+    }
+    float os = -INFINITY;
+    int oi = 0x7fffffff, op = 0, oc = 0;
+    for (int k = 0; k < KG; ++k) {
+      float bs = hs;
+      int bi = hi;
+      warp_best(bs, bi);
+      const unsigned who = __ballot_sync(0xffffffffu, hi == bi && bi != 0x7fffffff);
+      const int src = who ? __ffs(who) - 1 : 0;
+      const int bp = __shfl_sync(0xffffffffu, hp, src);
+      const int bc = __shfl_sync(0xffffffffu, hc, src);
+      if (lane == k) {
+        os = bs;
+        oi = bi;
+        op = bp;
+        oc = bc;
+      }
+      if (who && lane == src) {
+        hs = -INFINITY;
+        hi = 0x7fffffff;
+      }
+    }
     if (lane == 0) {
       part[j * (D + 2) + 0] = alive ? m_run : -INFINITY;
-      part[j * (D + 2) + 1] = alive ? l_run : 0.f;
+      part[j * (D + 2) + 1] = alive ? l_run + xl[j] : 0.f;
     }
     Cand* out = reinterpret_cast<Cand*>(a.cand) + ((u * a.nsplit + s) * NQ + j) * KG;
     if (lane < KG) {
       Cand c;
-      if (!alive || c_i == 0x7fffffff) {
-        c.s = -INFINITY;
-        c.id = -1;
-        c.pages = 0;
-        c.cnt = 0;
-      } else {
-        const int64_t ch = c_i / a.k;
-        const int jj = c_i % a.k;
-        const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + ch * (a.k + 1) + jj;
-        c.s = c_s;
-        c.id = c_i;
-        c.pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
-        c.cnt = gC[c_i];
-      }
+      const bool none = !alive || oi == 0x7fffffff;
+      c.s = none ? -INFINITY : os;
+      c.id = none ? -1 : oi;
+      c.pages = none ? 0 : op;
+      c.cnt = none ? 0 : oc;
       out[lane] = c;
     }
   }
@@ -396,7 +519,6 @@ cudaError_t launch_scan_tc(const AttendArgs& a, const TcMaps& maps, int NQ, cuda
     case 2: return launch_nq<2>(a, maps, stream);
     case 4: return launch_nq<4>(a, maps, stream);
     case 8: return launch_nq<8>(a, maps, stream);
-    case 16: return launch_nq<16>(a, maps, stream);
     default: return cudaErrorInvalidValue;
   }
 }
