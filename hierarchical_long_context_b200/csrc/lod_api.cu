@@ -240,7 +240,7 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
-                 int64_t c1, const lod_index* ix, cudaStream_t stream) {
+                 int64_t c1, const lod_index* ix, void* ws, cudaStream_t stream) {
   lod::BuildArgs a;
   memset(&a, 0, sizeof(a));
   a.K = K;
@@ -265,6 +265,7 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.pBeg = ix->pBeg;
   a.gPage = ix->gPage;
   a.perm = ix->perm;
+  a.status = static_cast<uint32_t*>(ws);
   cudaError_t e = lod::launch_build(a, p->dtype, p->d, c1 - c0, p->B, stream);
   if (e != cudaSuccess) return cuda_fail(e, "index build launch");
   return LOD_OK;
@@ -322,7 +323,7 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V, const
   if (chunk_end - chunk_begin > 0x7fffffff) return fail(LOD_EINVAL, "chunk range too large");
   if (!ws || !aligned16(ws) || ws_bytes < lod::kWsHeader)
     return fail(LOD_EINVAL, "workspace too small or misaligned");
-  rc = do_build(p, K, V, kv_strides, chunk_begin, chunk_end, index, (cudaStream_t)stream);
+  rc = do_build(p, K, V, kv_strides, chunk_begin, chunk_end, index, ws, (cudaStream_t)stream);
   if (!rc) g_err[0] = 0;
   return rc;
 }
@@ -382,7 +383,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   // 1) index of every chunk completed inside the query range (a pure function of K/V)
   const int64_t c0 = q_begin / p->chunk, c1 = (q_begin + Tq) / p->chunk;
   if (c1 > c0) {
-    rc = do_build(p, K, V, kv_strides, c0, c1, index, st);
+    rc = do_build(p, K, V, kv_strides, c0, c1, index, ws, st);
     if (rc) return rc;
   }
   // 2) attention, one launch pair per query chunk

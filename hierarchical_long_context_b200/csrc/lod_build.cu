@@ -2,19 +2,24 @@
 // Attention", How It Works, paragraph 1): per 256-token chunk, k-means groups,
 // 16-key pages, and their mean keys, mean values and counts.
 //
-// One CTA of 256 threads per (chunk, KV head, sequence); thread i owns the
-// chunk's i-th clustered key and keeps it in registers as fp32.  Centroids
-// live in shared memory and are read as warp-uniform (broadcast) float4
-// loads, so the assignment step is one FMA per (key, centroid, dimension)
-// in the expanded form ||c||^2 - 2 k.c (the ||k||^2 term is common to all
-// centroids of a key and cannot change its argmin).
+// One CTA of 256 threads per (chunk, KV head, sequence).
+// The chunk's keys are staged in shared memory by one TMA bulk copy; thread i
+// also keeps key i in registers in the cache's packed form.  Centroids live
+// in shared memory as fp32 pairs, interleaved by cluster, and are read as
+// warp-uniform (broadcast) loads, so the assignment step is one packed fp32x2
+// FMA per (key, centroid, two dimensions) in the expanded form
+// ||c||^2 - 2 k.c (the ||k||^2 term is common to all centroids of a key).
 //
 // The update step is deterministic: members are counting-sorted by cluster
-// (stable, ascending position) and every (cluster, dimension) sum is taken by
-// one thread in that order.  Hence an iteration whose assignment equals the
-// previous one reproduces the previous centroids bit for bit, every later
-// round would repeat it, and the loop may stop there with an unchanged
-// result.
+// (stable, ascending position) and every (cluster, dimension) sum is taken in
+// a fixed order.  An iteration whose assignment equals the previous one
+// therefore reproduces the previous centroids bit for bit, every later round
+// would repeat it, and the loop stops there with an unchanged result.
+//
+// Summaries: each warp sums whole pages (its V rows read with coalesced
+// loads, all in flight), writes the page means and keeps the page sums in
+// shared memory; a group's mean value is the sum of its pages' sums, and its
+// mean key is the final centroid.
 #include "lod_internal.cuh"
 
 namespace lod {
@@ -22,8 +27,9 @@ namespace lod {
 namespace {
 
 constexpr int kBuildThreads = 256;
+constexpr int kBuildWarps = kBuildThreads / 32;
 
-template <int N>
+template <int NW>
 __device__ __forceinline__ void block_argmax(float v, int idx, float* red_s, int* red_i, float& out_v,
                                              int& out_i) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -43,8 +49,8 @@ __device__ __forceinline__ void block_argmax(float v, int idx, float* red_s, int
   }
   __syncthreads();
   if (warp == 0) {
-    v = lane < N ? red_s[lane] : -INFINITY;
-    idx = lane < N ? red_i[lane] : 0x7fffffff;
+    v = lane < NW ? red_s[lane] : -INFINITY;
+    idx = lane < NW ? red_i[lane] : 0x7fffffff;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       float v2 = __shfl_xor_sync(0xffffffffu, v, o);
@@ -55,20 +61,52 @@ __device__ __forceinline__ void block_argmax(float v, int idx, float* red_s, int
       }
     }
     if (lane == 0) {
-      red_s[N] = v;
-      red_i[N] = idx;
+      red_s[NW] = v;
+      red_i[NW] = idx;
     }
   }
   __syncthreads();
-  out_v = red_s[N];
-  out_i = red_i[N];
+  out_v = red_s[NW];
+  out_i = red_i[NW];
   __syncthreads();
 }
 
+// Element pair p (dims 2p, 2p+1) of a key held as packed 32-bit words.
+template <typename T>
+__device__ __forceinline__ float2 pair_of(const uint32_t* w, int p) {
+  if constexpr (sizeof(T) == 2) {
+    return make_float2(__uint_as_float(w[p] << 16), __uint_as_float(w[p] & 0xffff0000u));
+  } else {
+    return make_float2(__uint_as_float(w[2 * p]), __uint_as_float(w[2 * p + 1]));
+  }
+}
+
 template <typename T, int D, int KMAX>
-__global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
-  constexpr int NW = kBuildThreads / 32;
-  constexpr int ROW_BYTES = D * (int)sizeof(T) + 16;  // padded row: conflict-free per-thread rows
+struct BuildSmem {
+  static constexpr int PMAX = kChunk / kPage + KMAX;  // page slots per chunk
+  static constexpr size_t off_x = 0;                                        // T [256][D]
+  static constexpr size_t off_cen = (size_t)kChunk * D * sizeof(T);         // float2 [D/2][KMAX]
+  static constexpr size_t off_psum = off_cen + sizeof(float) * D * KMAX;    // float [PMAX][D] value sums
+  static constexpr size_t off_cn = off_psum + sizeof(float) * PMAX * D;     // float [KMAX]
+  static constexpr size_t off_red = off_cn + sizeof(float) * KMAX;          // float/int [NW+1] x 2
+  static constexpr size_t off_wc = off_red + 8 * (kBuildWarps + 1);         // int [NW][KMAX]
+  static constexpr size_t off_cnt = off_wc + 4 * kBuildWarps * KMAX;        // int [KMAX]
+  static constexpr size_t off_off = off_cnt + 4 * KMAX;                     // int [KMAX+1]
+  static constexpr size_t off_ps = off_off + 4 * (KMAX + 1);                // int [KMAX+1]
+  static constexpr size_t off_perm = off_ps + 4 * (KMAX + 1);               // int [256]
+  static constexpr size_t off_bar = (off_perm + 4 * kChunk + 7) & ~size_t(7);
+  static constexpr size_t bytes = off_bar + 8;
+};
+
+// Keys of 256 bytes stay in registers at one CTA per SM; smaller ones fit two.
+template <typename T, int D, int KMAX>
+__global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1) kmeans_kernel(BuildArgs a) {
+  constexpr int NW = kBuildWarps;
+  constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int NWORD = D * (int)sizeof(T) / 4;  // packed 32-bit words per key
+  constexpr int NP = D / 2;                      // dimension pairs
+  using SM = BuildSmem<T, D, KMAX>;
+  constexpr int PMAX = SM::PMAX;
   const int64_t c = a.chunk_begin + blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t unit = (int64_t)b * a.Hkv + h;
@@ -77,40 +115,56 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
   const int n = kChunk - first;
   const int k = a.k;
 
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* cen = reinterpret_cast<float*>(smem_raw);              // [KMAX][D]
-  float* cnorm = cen + KMAX * D;                                // [KMAX]
-  float* red_s = cnorm + KMAX;                                  // [NW + 1]
-  int* red_i = reinterpret_cast<int*>(red_s + NW + 1);          // [NW + 1]
-  int* wcnt = red_i + NW + 1;                                   // [NW][KMAX]
-  int* cnt = wcnt + NW * KMAX;                                  // [KMAX]
-  int* off = cnt + KMAX;                                        // [KMAX + 1]
-  int* pstart = off + KMAX + 1;                                 // [KMAX + 1]
-  int* perm_s = pstart + KMAX + 1;                              // [kChunk]
-  unsigned char* xs = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(perm_s + kChunk) + 15) & ~uintptr_t(15));  // [kChunk][ROW_BYTES]
+  extern __shared__ __align__(128) unsigned char smem[];
+  T* xs = reinterpret_cast<T*>(smem + SM::off_x);
+  float2* cen2 = reinterpret_cast<float2*>(smem + SM::off_cen);
+  float* psum = reinterpret_cast<float*>(smem + SM::off_psum);
+  float* cnorm = reinterpret_cast<float*>(smem + SM::off_cn);
+  float* red_s = reinterpret_cast<float*>(smem + SM::off_red);
+  int* red_i = reinterpret_cast<int*>(red_s + NW + 1);
+  int* wcnt = reinterpret_cast<int*>(smem + SM::off_wc);
+  int* cnt = reinterpret_cast<int*>(smem + SM::off_cnt);
+  int* off = reinterpret_cast<int*>(smem + SM::off_off);
+  int* pstart = reinterpret_cast<int*>(smem + SM::off_ps);
+  int* perm_s = reinterpret_cast<int*>(smem + SM::off_perm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM::off_bar);
 
   const T* Kc = static_cast<const T*>(a.K) + b * a.sb + h * a.sh + c * kChunk * a.st;
   const T* Vc = static_cast<const T*>(a.V) + b * a.sb + h * a.sh + c * kChunk * a.st;
 
-  // ---- own key into registers (fp32) and into the padded shared-memory copy
-  float x[D];
-  if (tid < n) {
-    const T* row = Kc + (int64_t)(first + tid) * a.st;
-    constexpr int VEC = 16 / sizeof(T);
-#pragma unroll
-    for (int i = 0; i < D; i += VEC) {
-      uint4 raw = __ldg(reinterpret_cast<const uint4*>(row + i));
-      *reinterpret_cast<uint4*>(xs + tid * ROW_BYTES + i * sizeof(T)) = raw;
-      float f[VEC];
-      load_f<T, VEC>(row + i, f);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) x[i + e] = f[e];
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < D; ++i) x[i] = 0.f;
+  // ---- stage the chunk's keys in shared memory (TMA) and own key in registers
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
   }
+  __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect(bar, (uint32_t)kChunk * ROWB);
+    __syncwarp();
+    if (a.st == D) {
+      if (lane == 0) bulk_g2s(xs, Kc, (uint32_t)kChunk * ROWB, bar);
+    } else {
+      for (int r = lane; r < kChunk; r += 32) bulk_g2s(xs + r * D, Kc + (int64_t)r * a.st, ROWB, bar);
+    }
+  }
+  uint32_t kw[NWORD];
+  {
+    const uint4* row = reinterpret_cast<const uint4*>(Kc + (int64_t)(tid < n ? first + tid : first) * a.st);
+#pragma unroll
+    for (int v = 0; v < NWORD / 4; ++v) {
+      const uint4 r = __ldg(row + v);
+      kw[4 * v] = r.x;
+      kw[4 * v + 1] = r.y;
+      kw[4 * v + 2] = r.z;
+      kw[4 * v + 3] = r.w;
+    }
+  }
+  const bool staged = mbar_wait(bar, 0, a.status);
+  if (!__syncthreads_and(staged)) {  // copy timed out: leave this chunk unwritten
+    if (tid == 0) (void)mbar_wait(bar, 0, a.status);
+    return;
+  }
+  auto xval = [&](int row, int d) { return Elem<T>::to_f(xs[row * D + d]); };
 
   // ---- seeded farthest-first initialisation
   float mind = tid < n ? INFINITY : -INFINITY;
@@ -123,32 +177,35 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
       float bv;
       block_argmax<NW>(tid < n ? mind : -INFINITY, tid, red_s, red_i, bv, pick);
     }
-    if (tid == pick) {
-#pragma unroll
-      for (int i = 0; i < D; ++i) cen[j * D + i] = x[i];
-    }
+    for (int p = tid; p < NP; p += kBuildThreads)
+      cen2[p * KMAX + j] = make_float2(xval(first + pick, 2 * p), xval(first + pick, 2 * p + 1));
     __syncthreads();
     if (tid < n) {
       float dd = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; i += 4) {
-        float4 cc = *reinterpret_cast<const float4*>(cen + j * D + i);
-        float t0 = x[i] - cc.x, t1 = x[i + 1] - cc.y, t2 = x[i + 2] - cc.z, t3 = x[i + 3] - cc.w;
+      for (int p = 0; p < NP; ++p) {
+        const float2 x = pair_of<T>(kw, p);
+        const float2 cc = cen2[p * KMAX + j];
+        const float t0 = x.x - cc.x, t1 = x.y - cc.y;
         dd = fmaf(t0, t0, dd);
         dd = fmaf(t1, t1, dd);
-        dd = fmaf(t2, t2, dd);
-        dd = fmaf(t3, t3, dd);
       }
       mind = fminf(mind, dd);
     }
   }
-  // centroid norms
-  for (int j = warp; j < k; j += NW) {
-    float s = 0.f;
-    for (int i = lane; i < D; i += 32) s = fmaf(cen[j * D + i], cen[j * D + i], s);
-    s = warp_sum(s);
-    if (lane == 0) cnorm[j] = s;
-  }
+  auto norms = [&]() {
+    for (int j = warp; j < k; j += NW) {
+      float s = 0.f;
+      for (int p = lane; p < NP; p += 32) {
+        const float2 cc = cen2[p * KMAX + j];
+        s = fmaf(cc.x, cc.x, s);
+        s = fmaf(cc.y, cc.y, s);
+      }
+      s = warp_sum(s);
+      if (lane == 0) cnorm[j] = s;
+    }
+  };
+  norms();
   __syncthreads();
 
   // ---- Lloyd rounds
@@ -156,27 +213,21 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
   for (int it = 0; it < a.iters; ++it) {
     int a_new = 0;
     if (tid < n) {
-      float dot[KMAX];
+      float2 dot[KMAX];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) dot[j] = 0.f;
+      for (int j = 0; j < KMAX; ++j) dot[j] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < D; i += 4) {
+      for (int p = 0; p < NP; ++p) {
+        const float2 x = pair_of<T>(kw, p);
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          if (j < k) {
-            float4 cc = *reinterpret_cast<const float4*>(cen + j * D + i);
-            dot[j] = fmaf(x[i], cc.x, dot[j]);
-            dot[j] = fmaf(x[i + 1], cc.y, dot[j]);
-            dot[j] = fmaf(x[i + 2], cc.z, dot[j]);
-            dot[j] = fmaf(x[i + 3], cc.w, dot[j]);
-          }
-        }
+        for (int j = 0; j < KMAX; ++j)
+          if (j < k) dot[j] = ffma2(x, cen2[p * KMAX + j], dot[j]);
       }
-      float best = fmaf(-2.f, dot[0], cnorm[0]);
+      float best = fmaf(-2.f, dot[0].x + dot[0].y, cnorm[0]);
 #pragma unroll
       for (int j = 1; j < KMAX; ++j) {
         if (j < k) {
-          float dj = fmaf(-2.f, dot[j], cnorm[j]);
+          const float dj = fmaf(-2.f, dot[j].x + dot[j].y, cnorm[j]);
           if (dj < best) {  // strict: ties keep the lower cluster id
             best = dj;
             a_new = j;
@@ -191,7 +242,7 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
     // stable counting sort of members by cluster (ascending local index)
     int rank = 0;
     for (int j = 0; j < k; ++j) {
-      unsigned m = __ballot_sync(0xffffffffu, tid < n && a_new == j);
+      const unsigned m = __ballot_sync(0xffffffffu, tid < n && a_new == j);
       if (lane == 0) wcnt[warp * KMAX + j] = __popc(m);
       if (tid < n && a_new == j) rank = __popc(m & ((1u << lane) - 1u));
     }
@@ -202,7 +253,7 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
         off[j] = o;
         int cj = 0;
         for (int w = 0; w < NW; ++w) {
-          int t = wcnt[w * KMAX + j];
+          const int t = wcnt[w * KMAX + j];
           wcnt[w * KMAX + j] = o + cj;  // becomes the warp's base offset for cluster j
           cj += t;
         }
@@ -215,24 +266,34 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
     if (tid < n) perm_s[wcnt[warp * KMAX + a_new] + rank] = tid;
     __syncthreads();
 
-    // centroid := member mean (fp32, ascending member order); empty clusters keep theirs
-    for (int item = tid; item < k * D; item += kBuildThreads) {
-      const int j = item / D, i = item % D;
+    // centroid := member mean (fp32, fixed order: four interleaved partial sums);
+    // empty clusters keep theirs
+    for (int item = tid; item < k * NP; item += kBuildThreads) {
+      const int j = item / NP, p = item % NP;
       const int cj = cnt[j];
       if (cj > 0) {
-        float s = 0.f;
-        for (int m = off[j]; m < off[j] + cj; ++m)
-          s += Elem<T>::to_f(*reinterpret_cast<const T*>(xs + perm_s[m] * ROW_BYTES + i * sizeof(T)));
-        cen[j * D + i] = s / (float)cj;
+        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
+        const int m0 = off[j], m1 = off[j] + cj;
+        int m = m0;
+        for (; m + 3 < m1; m += 4) {
+          const int r0 = first + perm_s[m], r1 = first + perm_s[m + 1];
+          const int r2 = first + perm_s[m + 2], r3 = first + perm_s[m + 3];
+          s0.x += xval(r0, 2 * p); s0.y += xval(r0, 2 * p + 1);
+          s1.x += xval(r1, 2 * p); s1.y += xval(r1, 2 * p + 1);
+          s2.x += xval(r2, 2 * p); s2.y += xval(r2, 2 * p + 1);
+          s3.x += xval(r3, 2 * p); s3.y += xval(r3, 2 * p + 1);
+        }
+        for (; m < m1; ++m) {
+          const int r0 = first + perm_s[m];
+          s0.x += xval(r0, 2 * p);
+          s0.y += xval(r0, 2 * p + 1);
+        }
+        const float sx = (s0.x + s1.x) + (s2.x + s3.x), sy = (s0.y + s1.y) + (s2.y + s3.y);
+        cen2[p * KMAX + j] = make_float2(sx / (float)cj, sy / (float)cj);
       }
     }
     __syncthreads();
-    for (int j = warp; j < k; j += NW) {
-      float s = 0.f;
-      for (int i = lane; i < D; i += 32) s = fmaf(cen[j * D + i], cen[j * D + i], s);
-      s = warp_sum(s);
-      if (lane == 0) cnorm[j] = s;
-    }
+    norms();
     __syncthreads();
   }
 
@@ -261,8 +322,8 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
   perm[tid] = tid < n ? (int16_t)(first + perm_s[tid]) : (int16_t)-1;
   if (tid <= k) gPage[tid] = (int16_t)pstart[tid];
   if (tid < k) gCnt[tid] = cnt[tid];
+  const int used = pstart[k];
   if (tid < P) {
-    int used = pstart[k];
     if (tid < used) {
       int j = 0;
       while (j + 1 < k && pstart[j + 1] <= tid) ++j;
@@ -275,57 +336,72 @@ __global__ void __launch_bounds__(kBuildThreads, 1) kmeans_kernel(BuildArgs a) {
     }
   }
 
-  // summaries: one thread per (group, dimension, K-or-V), fp32 sums in member order
-  for (int item = tid; item < 2 * k * D; item += kBuildThreads) {
-    const int isv = item / (k * D);
-    const int j = (item / D) % k, i = item % D;
-    const int cj = cnt[j];
-    T* gdst = isv ? gV : gK;
-    T* pdst = isv ? pV : pK;
-    if (cj == 0) {
-      gdst[j * D + i] = Elem<T>::from_f(0.f);
-      continue;
-    }
-    float gs = 0.f, ps = 0.f;
-    int inpage = 0, slot = pstart[j];
-    for (int m = off[j]; m < off[j] + cj; ++m) {
-      const int loc = perm_s[m];
-      float v = isv ? Elem<T>::to_f(Vc[(int64_t)(first + loc) * a.st + i])
-                    : Elem<T>::to_f(*reinterpret_cast<const T*>(xs + loc * ROW_BYTES + i * sizeof(T)));
-      gs += v;
-      ps += v;
-      if (++inpage == kPage) {
-        pdst[slot * D + i] = Elem<T>::from_f(ps / (float)kPage);
-        ++slot;
-        ps = 0.f;
-        inpage = 0;
+  // page sums: warp w takes pages w, w + NW, ...; lane owns DPL dims
+  constexpr int DPL = D / 32;
+  for (int pg = warp; pg < used; pg += NW) {
+    int j = 0;
+    while (j + 1 < k && pstart[j + 1] <= pg) ++j;
+    const int m0 = off[j] + (pg - pstart[j]) * kPage;
+    const int pc = min(kPage, cnt[j] - (pg - pstart[j]) * kPage);
+    float vv[kPage][DPL];
+#pragma unroll
+    for (int r = 0; r < kPage; ++r) {
+      if (r < pc) {
+        load_f<T, DPL>(Vc + (int64_t)(first + perm_s[m0 + r]) * a.st + lane * DPL, vv[r]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) vv[r][i] = 0.f;
       }
     }
-    if (inpage > 0) pdst[slot * D + i] = Elem<T>::from_f(ps / (float)inpage);
-    // the group key mean is the final centroid: the same fp32 sum / count
-    gdst[j * D + i] = Elem<T>::from_f(isv ? gs / (float)cj : cen[j * D + i]);
+    float sk[DPL], sv[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) sk[i] = sv[i] = 0.f;
+#pragma unroll
+    for (int r = 0; r < kPage; ++r) {
+      if (r < pc) {
+        const int row = first + perm_s[m0 + r];
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) {
+          sk[i] += xval(row, lane * DPL + i);
+          sv[i] += vv[r][i];
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      pK[pg * D + lane * DPL + i] = Elem<T>::from_f(sk[i] / (float)pc);
+      pV[pg * D + lane * DPL + i] = Elem<T>::from_f(sv[i] / (float)pc);
+      psum[pg * D + lane * DPL + i] = sv[i];
+    }
   }
   // unused page slots hold zeros
-  for (int item = tid; item < (int)(P - pstart[k]) * D; item += kBuildThreads) {
-    const int slot = pstart[k] + item / D, i = item % D;
+  for (int item = tid; item < (int)(P - used) * D; item += kBuildThreads) {
+    const int slot = used + item / D, i = item % D;
     pK[slot * D + i] = Elem<T>::from_f(0.f);
     pV[slot * D + i] = Elem<T>::from_f(0.f);
   }
-}
-
-template <int D, int KMAX>
-size_t kmeans_smem_bytes(size_t elem) {
-  constexpr int NW = kBuildThreads / 32;
-  size_t s = sizeof(float) * (KMAX * D + KMAX + NW + 1) + sizeof(int) * (NW + 1 + NW * KMAX + KMAX +
-                                                                          2 * (KMAX + 1) + kChunk);
-  s = (s + 15) & ~size_t(15);
-  s += (size_t)kChunk * (D * elem + 16);
-  return s;
+  __syncthreads();
+  // group means: key = the final centroid; value = its pages' sums in page order
+  for (int item = tid; item < k * D; item += kBuildThreads) {
+    const int j = item / D, i = item % D;
+    const int cj = cnt[j];
+    if (cj == 0) {
+      gK[j * D + i] = Elem<T>::from_f(0.f);
+      gV[j * D + i] = Elem<T>::from_f(0.f);
+      continue;
+    }
+    float s = 0.f;
+    for (int pg = pstart[j]; pg < pstart[j + 1]; ++pg) s += psum[pg * D + i];
+    const float2 cc = cen2[(i / 2) * KMAX + j];
+    gK[j * D + i] = Elem<T>::from_f((i & 1) ? cc.y : cc.x);
+    gV[j * D + i] = Elem<T>::from_f(s / (float)cj);
+  }
+  static_assert(PMAX >= kChunk / kPage, "page slots");
 }
 
 template <typename T, int D, int KMAX>
 cudaError_t launch_kmeans_t(const BuildArgs& a, int64_t nchunks, int B, cudaStream_t stream) {
-  const size_t smem = kmeans_smem_bytes<D, KMAX>(sizeof(T));
+  const size_t smem = BuildSmem<T, D, KMAX>::bytes;
   auto kern = kmeans_kernel<T, D, KMAX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -29,6 +29,7 @@ struct BuildArgs {
   int16_t* pBeg;
   int16_t* gPage;
   int16_t* perm;
+  uint32_t* status;    // device status word (workspace header)
 };
 
 // Scan CTAs a decode call aims for: two resident CTAs on each of the B200's 148 SMs.
