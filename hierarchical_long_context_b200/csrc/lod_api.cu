@@ -190,10 +190,9 @@ int32_t make_tc_maps(const lod_params* p, const void* K, const void* V, const in
 }
 
 size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
-  const int KG = kg_of(p);
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
-  size_t cand = lod::cand_bytes() * (size_t)s.units * s.nsplit * s.NQ * KG;
-  return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((cand + 255) & ~size_t(255));
+  size_t gsc = sizeof(float) * (size_t)s.units * s.NQ * (size_t)(p->Tmax / p->chunk) * p->clusters;
+  return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((gsc + 255) & ~size_t(255));
 }
 
 void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, const void* K,
@@ -231,12 +230,10 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   a.units = s.units;
   char* w = static_cast<char*>(ws);
   a.status = reinterpret_cast<uint32_t*>(w);
-  const int KG = kg_of(p);
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
   part = (part + 255) & ~size_t(255);
   a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
-  a.cand = w + lod::kWsHeader + part;
-  (void)KG;
+  a.gsc = reinterpret_cast<float*>(w + lod::kWsHeader + part);
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
@@ -412,7 +409,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.units = (int64_t)p->B * p->Hkv * cdiv(hi - lo, s.NP);
     const int want = split_for(p, s.tc, a.units, wb * p->clusters + p->window);
     a.nsplit = want < s.nsplit ? want : s.nsplit;
-    // part/cand keep the worst-case layout of fill_attend; a chunk uses a prefix
+    // part/gsc keep the worst-case layout of fill_attend; a chunk uses a prefix
     cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, s.tc ? &maps : nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   }
@@ -442,7 +439,7 @@ int32_t lod_get_status(void* ws, lod_stream_t stream, uint32_t* status) {
 // while a CUDA graph or a latency-critical step is being recorded, or a
 // plugin host that gives its kernels only their input and output buffers.
 // For them this entry point keeps the decode scratch (split partial states,
-// candidate records and the status word) in a fixed array compiled into the
+// group scores and the status word) in a fixed array compiled into the
 // library.  The array is `static __device__`, so each GPU that loads this
 // library holds its kLodNoallocScratchBytes until the process exits.  Host
 // code cannot use the array's name as an address; the device address is
@@ -502,7 +499,7 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
   rc = noalloc_scratch(&ws);
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  // The partial states and candidates are fully rewritten by every call; only
+  // The partial states and group scores are fully rewritten by every call; only
   // the status word must start from zero when no caller word is given.
   if (!status) {
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), st);

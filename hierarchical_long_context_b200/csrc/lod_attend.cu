@@ -9,13 +9,13 @@
 //          TMA bulk copies -- either visible group summaries (mean key, mean
 //          value, count) or exact window/sink tokens -- and computes
 //            pass 1  the scores of all its rows against the NQ queries,
-//            then    per query row the max logit (score + ln count) and, for
-//                    group slices, the local top-KG groups by score,
+//            then    per query row the max logit (score + ln count), and the
+//                    group scores go to the workspace's score array,
 //            pass 2  the weighted sum of its values,
 //          leaving a partial softmax state (max, sum, acc[d]) over ALL its rows.
 //  refine  one CTA per query row, launched as a programmatic dependent of the
-//          scan.  It merges the split states, picks the global top
-//          `top_groups` groups from the local candidates, removes those groups'
+//          scan.  It merges the split states, picks the top `top_groups`
+//          groups from the unit's score array, removes those groups'
 //          coarse terms (they are replaced by finer entries), scores each
 //          opened group's page summaries, opens the top `top_pages` pages and
 //          adds their tokens exactly (values staged by TMA), adds the other
@@ -96,10 +96,10 @@ __device__ __forceinline__ UnitInfo unit_info(const AttendArgs& a, int64_t u) {
   return ui;
 }
 
-// Candidate record written by the scan and read by the refine kernel.
+// An opened group (refine kernel).
 struct Cand {
   float s;     // scale * q.mean_k
-  int id;      // global group id (chunk * k + slot), -1 = none
+  int id;      // group id within the unit (chunk * k + slot), -1 = none
   int pages;   // first page slot | (last page slot + 1) << 16
   int cnt;     // group size
 };
@@ -133,7 +133,7 @@ __device__ __forceinline__ int64_t row_pos(int64_t e, int64_t G_vis, int64_t ns,
   return e < ns ? e : ws + (e - ns);
 }
 
-template <typename T, int D, int NQ, int KG>
+template <typename T, int D, int NQ>
 __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   constexpr int EPL = 16 / sizeof(T);  // elements per lane per 16-byte load
   constexpr int LPR = D / EPL;         // lanes per row
@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   const T* gK = static_cast<const T*>(a.gK) + unit_kv * a.Cmax * a.k * D;
   const T* gV = static_cast<const T*>(a.gV) + unit_kv * a.Cmax * a.k * D;
   const int32_t* gC = a.gCnt + unit_kv * a.Cmax * a.k;
+  const int64_t gcap = a.Cmax * a.k;
   const bool contiguous = a.st == D;
 
   // producer: stage slab i (rows [e0 + 64 i, ...)) into ring slot i % kStages
@@ -301,12 +302,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
     for (int e = 0; e < EPL; e += 2) q2[j][e / 2] = make_float2(f[e] * a.scale, f[e + 1] * a.scale);
   }
 
-  // running state: query row `warp` (warp < NQ) keeps (m, l) and its top-KG in lanes 0..KG-1
+  // running state: query row `warp` (warp < NQ) keeps (m, l)
   float m_run = -INFINITY, l_run = 0.f;
-  float c_s = -INFINITY;  // lane j < KG: j-th best score so far
-  int c_i = 0x7fffffff;   //                and its group id
-  float thr_s = -INFINITY;
-  int thr_i = 0x7fffffff;
   // P.V accumulators: one value row per warp step, lane owns DPL = d/32 dims
   constexpr int DPL = D / 32;
   float2 acc[NQ][DPL / 2];
@@ -368,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
       if (warp == 0) issue(i + kStages - 1);
       for (int r = tid; r < kSlab; r += kThreads) meta(i + kStages - 1, r);
     }
-    // ---- per query row: running max, weights, running sum, top-KG
+    // ---- per query row: running max, weights, running sum, group scores
     if (warp < NQ) {
       const int r = warp;
       float lg[kSlab / 32], sc[kSlab / 32];
@@ -399,17 +396,13 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
       l_run = l_run * corr + psum;
       m_run = mn;
       if (lane == 0) corr_s[r] = corr;
-      // top-KG by score (group rows only)
-      float ns[kSlab / 32];
-      int ni[kSlab / 32];
+      // group scores (-inf: not in this query row's softmax)
+      float* gsr = a.gsc + (u * NQ + r) * gcap;
 #pragma unroll
       for (int x = 0; x < kSlab / 32; ++x) {
         const int row = lane + 32 * x;
-        const bool isg = live[x] && pos_s[st * kSlab + row] < 0;
-        ns[x] = isg ? sc[x] : -INFINITY;
-        ni[x] = isg ? (int)(r0 + row) : 0x7fffffff;
+        if (row < n && pos_s[st * kSlab + row] < 0) gsr[r0 + row] = live[x] ? sc[x] : -INFINITY;
       }
-      topk_merge<KG, kSlab / 32>(ns, ni, c_s, c_i, thr_s, thr_i);
     }
     __syncthreads();
     // ---- acc[r] = acc[r] * corr[r] + P[:, r] . V   (warp w: rows w, w+8, ...)
@@ -472,28 +465,6 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   }
   float* lsh = P_s;  // l per query row
   if (warp < NQ && lane == 0) lsh[warp] = alive ? l_run : 0.f;
-  // candidates (all splits keep KG records per query row)
-  if (warp < NQ) {
-    Cand* out = reinterpret_cast<Cand*>(a.cand) + ((u * a.nsplit + s) * NQ + warp) * KG;
-    if (lane < KG) {
-      Cand c;
-      if (!alive || c_i == 0x7fffffff) {
-        c.s = -INFINITY;
-        c.id = -1;
-        c.pages = 0;
-        c.cnt = 0;
-      } else {
-        const int64_t ch = c_i / a.k;
-        const int j = c_i % a.k;
-        const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + ch * (a.k + 1) + j;
-        c.s = c_s;
-        c.id = c_i;
-        c.pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
-        c.cnt = gC[c_i];
-      }
-      out[lane] = c;
-    }
-  }
   __syncthreads();
   float* part = a.part + ((u * a.nsplit + s) * NQ) * (int64_t)(D + 2);
   for (int idx = tid; idx < NQ * (D + 2); idx += kThreads) {
@@ -530,8 +501,12 @@ struct RefineSmem {
   static constexpr size_t off_sc = off_g + sizeof(float) * (D + 4);     // float [kWarps][64]
   static constexpr size_t off_pos = off_sc + sizeof(float) * kWarps * 64;     // int64 [kWarps][32]
   static constexpr size_t off_c = off_pos + sizeof(int64_t) * kWarps * 32;    // Cand [kMaxTopGroups]
-  static constexpr size_t off_bar = off_c + sizeof(Cand) * kMaxTopGroups + 16;
+  static constexpr size_t off_key = off_c + sizeof(Cand) * kMaxTopGroups + 16;  // uint64 [kWarps][32]
+  static constexpr size_t off_wb = off_key + 8 * kWarps * 32;                  // uint64 [kWarps]
+  static constexpr size_t off_bar = off_wb + 8 * kWarps + 16;
   static constexpr size_t bytes = off_bar + 8 * kWarps + 16;
+  // group selection: the survivors of the bound reuse the value buffers
+  static constexpr int kSurvCap = (int)(off_perm / 8);
 };
 
 // Scores of up to 32 d-rows against q, loaded with coalesced 16-byte loads:
@@ -576,7 +551,39 @@ __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const f
   }
 }
 
-template <typename T, int D, int NQ, int KG>
+// Orderable 64-bit key of group `id` with score s: a larger key is a better
+// group (higher score, then smaller id); 0 = no group (score -inf).
+__device__ __forceinline__ uint64_t group_key(float s, int64_t id) {
+  if (s == -INFINITY) return 0;
+  uint32_t b = __float_as_uint(s);
+  b ^= (b & 0x80000000u) ? 0xffffffffu : 0x80000000u;
+  return ((uint64_t)b << 32) | (uint32_t)(0xffffffffu - (uint32_t)id);
+}
+__device__ __forceinline__ float key_score(uint64_t k) {
+  uint32_t b = (uint32_t)(k >> 32);
+  b = (b & 0x80000000u) ? (b ^ 0x80000000u) : ~b;
+  return __uint_as_float(b);
+}
+__device__ __forceinline__ int key_id(uint64_t k) { return (int)(0xffffffffu - (uint32_t)k); }
+
+// Largest key over the CTA (every thread receives it); red: [kWarps] scratch.
+__device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = x > v ? x : v;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  uint64_t r = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) r = red[w] > r ? red[w] : r;
+  return r;
+}
+
+template <typename T, int D, int NQ>
 __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   constexpr int DPL = D / 32;
   constexpr int EPL = 16 / sizeof(T);
@@ -616,6 +623,10 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   int64_t* posm_s = reinterpret_cast<int64_t*>(smem + SM::off_pos);
   Cand* win = reinterpret_cast<Cand*>(smem + SM::off_c);
   int* nwin_s = reinterpret_cast<int*>(smem + SM::off_c + sizeof(Cand) * kMaxTopGroups);
+  int* nsurv_s = nwin_s + 1;
+  uint64_t* keys_s = reinterpret_cast<uint64_t*>(smem + SM::off_key);
+  uint64_t* wb_s = reinterpret_cast<uint64_t*>(smem + SM::off_wb);
+  uint64_t* surv = reinterpret_cast<uint64_t*>(smem + SM::off_V);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM::off_bar);
 
   // ---- prologue (overlaps the scan's tail): position, q, barriers
@@ -641,46 +652,99 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   pdl_wait();  // the scan's partial states and candidates are visible from here on
 
   const int nsplit = a.nsplit;
-  // ---- global top-G over the splits' candidates (warp 0)
-  if (warp == 0) {
-    const int ncand = nsplit * KG;
-    const Cand* src = reinterpret_cast<const Cand*>(a.cand) + (u * nsplit * NQ) * (int64_t)KG;
-    float lastS = INFINITY;
-    int lastI = -1;
-    int nwin = 0;
-    for (int rank = 0; rank < a.G; ++rank) {
-      float bs = -INFINITY;
-      int bi = 0x7fffffff, bidx = -1;
-      for (int e = lane; e < ncand; e += 32) {
-        const int sp = e / KG, j = e % KG;
-        const int64_t off = ((int64_t)sp * NQ + r) * KG + j;
-        const int id = src[off].id;
-        if (id < 0) continue;
-        const float sc = src[off].s;
-        const bool after = rank == 0 || cand_better(lastS, lastI, sc, id);
-        if (after && cand_better(sc, id, bs, bi)) {
-          bs = sc;
-          bi = id;
-          bidx = (int)off;
+  // ---- the top-G groups of this row from the unit's score array.  A bound
+  // that G distinct groups reach (the G-th best of a warp's per-thread best
+  // keys; the largest such bound over the warps), the groups at or above it
+  // (at most G threads per warp hold any), then their exact ranks.
+  {
+    const int64_t wbq = t / kChunk - a.window / kChunk + 1;
+    const int64_t Gq = wbq > 0 ? wbq * a.k : 0;  // visible groups of this row
+    const float* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
+    uint64_t tb = 0;
+#pragma unroll 4
+    for (int64_t i = tid; i < Gq; i += kThreads) {
+      const uint64_t kk = group_key(srow[i], i);
+      tb = kk > tb ? kk : tb;
+    }
+    keys_s[tid] = tb;
+    if (tid == 0) *nsurv_s = 0;
+    __syncwarp();
+    int rk = 0;
+    const ulonglong2* kw = reinterpret_cast<const ulonglong2*>(keys_s + warp * 32);
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const ulonglong2 pq = kw[x];
+      rk += (pq.x > tb ? 1 : 0) + (pq.y > tb ? 1 : 0);
+    }
+    const unsigned at = __ballot_sync(0xffffffffu, tb != 0 && rk == a.G - 1);
+    if (lane == 0) wb_s[warp] = at ? keys_s[warp * 32 + __ffs(at) - 1] : 0;
+    __syncthreads();
+    uint64_t lo = 1;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) lo = wb_s[w] > lo ? wb_s[w] : lo;
+    for (int64_t i0 = 0; i0 < Gq; i0 += kThreads) {
+      const int64_t i = i0 + tid;
+      const uint64_t kk = i < Gq ? group_key(srow[i], i) : 0;
+      const bool keep = kk >= lo;
+      const unsigned msk = __ballot_sync(0xffffffffu, keep);
+      if (msk) {
+        const int lead = __ffs(msk) - 1;
+        int base = 0;
+        if (lane == lead) base = atomicAdd(nsurv_s, __popc(msk));
+        base = __shfl_sync(0xffffffffu, base, lead);
+        const int pos = base + __popc(msk & ((1u << lane) - 1u));
+        if (keep && pos < SM::kSurvCap) surv[pos] = kk;
+      }
+    }
+    __syncthreads();
+    const int n = *nsurv_s;
+    const int nwin = n < a.G ? n : a.G;
+    if (n <= SM::kSurvCap) {
+      for (int x = tid; x < n; x += kThreads) {
+        const uint64_t kx = surv[x];
+        int rx = 0, y = 0;
+        for (; y + 1 < n; y += 2) {
+          const ulonglong2 pq = *reinterpret_cast<const ulonglong2*>(surv + y);
+          rx += (pq.x > kx ? 1 : 0) + (pq.y > kx ? 1 : 0);
+        }
+        if (y < n) rx += surv[y] > kx ? 1 : 0;
+        if (rx < nwin) {
+          win[rx].s = key_score(kx);
+          win[rx].id = key_id(kx);
         }
       }
-      float ws_ = bs;
-      int wi_ = bi;
-      warp_best(ws_, wi_);
-      if (wi_ == 0x7fffffff) break;
-      if (bi == wi_) win[rank] = src[bidx];
-      lastS = ws_;
-      lastI = wi_;
-      ++nwin;
+    } else {  // more survivors than the buffer holds: one rank at a time
+      uint64_t last = ~0ull;
+      for (int x = 0; x < nwin; ++x) {
+        uint64_t bk = 0;
+        for (int64_t i = tid; i < Gq; i += kThreads) {
+          const uint64_t kk = group_key(srow[i], i);
+          if (kk < last && kk > bk) bk = kk;
+        }
+        bk = block_max_key(bk, wb_s);
+        if (tid == 0) {
+          win[x].s = key_score(bk);
+          win[x].id = key_id(bk);
+        }
+        last = bk;
+      }
     }
-    if (lane == 0) *nwin_s = nwin;
-  } else {
+    if (tid == 0) *nwin_s = nwin;
+    __syncthreads();
+    if (tid < nwin) {  // the winners' sizes and page ranges
+      const int id = win[tid].id;
+      win[tid].cnt = a.gCnt[unit_kv * a.Cmax * a.k + id];
+      const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + (id / a.k) * (a.k + 1) + id % a.k;
+      win[tid].pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
+    }
+  }
+  {
     // ---- merge the split states (thread c owns component c: m, l, acc[])
     const float* ps = a.part + (u * nsplit * NQ + r) * (int64_t)(D + 2);
     const int64_t stride = (int64_t)NQ * (D + 2);
     float M = -INFINITY;
     for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, ps[sp * stride]);
-    for (int c = tid - 32; c < D + 2; c += kThreads - 32) {
+    for (int c = tid; c < D + 2; c += kThreads) {
       float v = 0.f;
       if (c == 0) {
         v = M;
@@ -921,7 +985,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     for (int i = nwin * a.TP + tid; i < a.G * a.TP; i += kThreads) a.sel_pages[orow * a.G * a.TP + i] = -1;
 }
 
-template <typename T, int D, int NQ, int KG>
+template <typename T, int D, int NQ>
 cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t stream) {
   const int nsplit = a.nsplit;
   const int64_t npos = a.seq_lens ? 1 : a.pos_hi - a.pos_lo;
@@ -931,7 +995,7 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
     if (maps) {
       e = launch_scan_tc(a, *maps, NQ, stream);
     } else if constexpr (NQ <= 8) {
-      auto sk = scan_kernel<T, D, NQ, KG>;
+      auto sk = scan_kernel<T, D, NQ>;
       const size_t smem = ScanSmem<T, D, NQ>::bytes;
       e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
@@ -943,7 +1007,7 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
     if (e != cudaSuccess) return e;
   }
   if (rows > 0) {
-    auto rk = refine_kernel<T, D, NQ, KG>;
+    auto rk = refine_kernel<T, D, NQ>;
     const size_t smem = RefineSmem<T, D>::bytes;
     e = cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -962,25 +1026,19 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
-template <typename T, int D, int NQ>
-cudaError_t launch_kg(const AttendArgs& a, const TcMaps* maps, cudaStream_t stream) {
-  return a.G <= 8 ? launch_t<T, D, NQ, 8>(a, maps, stream) : launch_t<T, D, NQ, 16>(a, maps, stream);
-}
-
 template <typename T, int D>
 cudaError_t launch_nq(const AttendArgs& a, int NQ, const TcMaps* maps, cudaStream_t stream) {
   switch (NQ) {
-    case 1: return launch_kg<T, D, 1>(a, maps, stream);
-    case 2: return launch_kg<T, D, 2>(a, maps, stream);
-    case 4: return launch_kg<T, D, 4>(a, maps, stream);
-    case 8: return launch_kg<T, D, 8>(a, maps, stream);
+    case 1: return launch_t<T, D, 1>(a, maps, stream);
+    case 2: return launch_t<T, D, 2>(a, maps, stream);
+    case 4: return launch_t<T, D, 4>(a, maps, stream);
+    case 8: return launch_t<T, D, 8>(a, maps, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-size_t cand_bytes() { return sizeof(Cand); }
 
 cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, const TcMaps* maps,
                           cudaStream_t stream) {

@@ -68,7 +68,8 @@ struct AttendArgs {
   int nsplit;               // splits of each unit's row list (groups, sinks, window)
   int64_t units;            // scan units in this launch
   float* part;              // [units][nsplit][NQ][d+2]  (m, l, acc)
-  void* cand;               // [units][nsplit][NQ][KG] candidate records (cand_bytes() each)
+  float* gsc;               // [units][NQ][Cmax * k] group scores scale * q . mean k of the
+                            // unit's visible groups (-inf: not in that query row's softmax)
   void* out;                // [B][Hq][Tq][d]
   float* lse;               // [B][Hq][Tq] or null
   int32_t* sel_groups;      // [B][Hq][Tq][G] or null
@@ -90,6 +91,5 @@ cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, const T
                           cudaStream_t stream);
 cudaError_t launch_scan_tc(const AttendArgs& a, const TcMaps& maps, int NQ, cudaStream_t stream);
 size_t scan_tc_smem_bytes();
-size_t cand_bytes();
 
 }  // namespace lod
