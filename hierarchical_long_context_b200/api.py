@@ -53,11 +53,11 @@ class Params:
 
 
 class Index:
-    """The nine device arrays of lod_index, as torch tensors."""
+    """The eleven device arrays of lod_index, as torch tensors."""
 
     def __init__(self, params: Params, device="cuda"):
         lib = load()
-        sizes = (ctypes.c_size_t * 9)()
+        sizes = (ctypes.c_size_t * len(_lib.INDEX_FIELDS))()
         check("lod_index_sizes", lib.lod_index_sizes(ctypes.byref(params.c()), sizes))
         p = params
         Cmax, k, P, d = p.Tmax // p.chunk, p.clusters, p.page_slots, p.d
@@ -71,6 +71,8 @@ class Index:
         self.pBeg = torch.zeros(*u, Cmax * P, dtype=torch.int16, device=device)
         self.gPage = torch.zeros(*u, Cmax * (k + 1), dtype=torch.int16, device=device)
         self.perm = torch.full((*u, Cmax * p.chunk), -1, dtype=torch.int16, device=device)
+        self.mK = torch.zeros(*u, Cmax * p.chunk, d, dtype=p.dtype, device=device)
+        self.mV = torch.zeros_like(self.mK)
         for i, f in enumerate(_lib.INDEX_FIELDS):
             t = getattr(self, f)
             assert t.numel() * t.element_size() == sizes[i], (f, t.numel() * t.element_size(), sizes[i])

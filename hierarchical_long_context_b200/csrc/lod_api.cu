@@ -81,10 +81,11 @@ int32_t validate_kv(const lod_params* p, const void* K, const void* V, const int
 
 int32_t validate_index(const lod_index* ix) {
   if (!ix) return fail(LOD_EINVAL, "index is NULL");
-  const void* ptrs[9] = {ix->gK, ix->gV, ix->gCnt, ix->pK, ix->pV, ix->pCnt, ix->pBeg, ix->gPage, ix->perm};
-  for (int i = 0; i < 9; ++i) {
+  const void* ptrs[LOD_INDEX_ARRAYS] = {ix->gK,   ix->gV,    ix->gCnt, ix->pK, ix->pV, ix->pCnt,
+                                        ix->pBeg, ix->gPage, ix->perm, ix->mK, ix->mV};
+  for (int i = 0; i < LOD_INDEX_ARRAYS; ++i) {
     if (!ptrs[i]) return fail(LOD_EINVAL, "index field %d is NULL", i);
-    if (i == 0 || i == 1 || i == 3 || i == 4) {
+    if (i == 0 || i == 1 || i == 3 || i == 4 || i == 9 || i == 10) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index summary %d must be 16-byte aligned", i);
     } else if (i == 8) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index member list (perm) must be 16-byte aligned");
@@ -212,6 +213,8 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   a.pBeg = ix->pBeg;
   a.gPage = ix->gPage;
   a.perm = ix->perm;
+  a.mK = ix->mK;
+  a.mV = ix->mV;
   a.B = p->B;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
@@ -262,6 +265,8 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.pBeg = ix->pBeg;
   a.gPage = ix->gPage;
   a.perm = ix->perm;
+  a.mK = ix->mK;
+  a.mV = ix->mV;
   a.status = static_cast<uint32_t*>(ws);
   cudaError_t e = lod::launch_build(a, p->dtype, p->d, c1 - c0, p->B, stream);
   if (e != cudaSuccess) return cuda_fail(e, "index build launch");
@@ -276,7 +281,7 @@ int32_t lod_version(void) { return 100; }
 
 const char* lod_last_error(void) { return g_err; }
 
-int32_t lod_index_sizes(const lod_params* p, size_t bytes[9]) {
+int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]) {
   int32_t rc = validate(p);
   if (rc) return rc;
   if (!bytes) return fail(LOD_EINVAL, "bytes is NULL");
@@ -289,6 +294,7 @@ int32_t lod_index_sizes(const lod_params* p, size_t bytes[9]) {
   bytes[6] = units * Cmax * P * sizeof(int16_t);
   bytes[7] = units * Cmax * (k + 1) * sizeof(int16_t);
   bytes[8] = units * Cmax * p->chunk * sizeof(int16_t);
+  bytes[9] = bytes[10] = units * Cmax * p->chunk * d * e;
   g_err[0] = 0;
   return LOD_OK;
 }

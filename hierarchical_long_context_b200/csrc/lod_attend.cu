@@ -491,35 +491,35 @@ struct RefineSmem {
   static constexpr int ROWB = D * sizeof(T);
   static constexpr int kRows = 48;  // per warp: 32 exact tokens + 16 coarse page means
   static constexpr size_t off_V = 0;                                     // [kWarps][kRows][D] T
-  static constexpr size_t off_perm = (size_t)kWarps * kRows * ROWB;      // int16 [kWarps][kChunk]
-  static constexpr size_t off_q = off_perm + 2 * kWarps * kChunk;        // float [D]
+  static constexpr size_t off_q = (size_t)kWarps * kRows * ROWB;        // float [D]
   static constexpr size_t off_g = off_q + sizeof(float) * D;            // float [D+4]
   // per-warp final states reuse the value buffers (used only after the group loop)
   static constexpr size_t off_w = off_V;                                // float [kWarps][D+4]
   static constexpr size_t off_d = off_V + sizeof(float) * kWarps * (D + 4);  // float [kWarps][D+4]
-  static_assert(2 * sizeof(float) * kWarps * (D + 4) <= off_perm, "final states fit the value buffers");
+  static_assert(2 * sizeof(float) * kWarps * (D + 4) <= off_q, "final states fit the value buffers");
   static constexpr size_t off_sc = off_g + sizeof(float) * (D + 4);     // float [kWarps][64]
   static constexpr size_t off_pos = off_sc + sizeof(float) * kWarps * 64;     // int64 [kWarps][32]
   static constexpr size_t off_c = off_pos + sizeof(int64_t) * kWarps * 32;    // Cand [kMaxTopGroups]
   static constexpr size_t off_key = off_c + sizeof(Cand) * kMaxTopGroups + 16;  // uint64 [kWarps][32]
   static constexpr size_t off_wb = off_key + 8 * kWarps * 32;                  // uint64 [kWarps]
-  static constexpr size_t off_bar = off_wb + 8 * kWarps + 16;
+  static constexpr size_t off_pc = off_wb + 8 * kWarps;                      // int [2][kWarps][32]
+  static constexpr size_t off_bar = off_pc + 4 * 2 * kWarps * 32 + 16;
   static constexpr size_t bytes = off_bar + 8 * kWarps + 16;
   // group selection: the survivors of the bound reuse the value buffers
-  static constexpr int kSurvCap = (int)(off_perm / 8);
+  static constexpr int kSurvCap = (int)(off_q / 8);
+  static_assert(ROWB > 256 || bytes <= 113 * 1024, "two CTAs per SM for rows of up to 256 bytes");
 };
 
 // Scores of up to 32 d-rows against q, loaded with coalesced 16-byte loads:
 // each half (or quarter) of the warp reads one whole row per step and the
 // row's score is reduced over its lanes.  rowptr(i) gives row i (valid for
 // i < n).  Writes score i to out[i].
-template <typename T, int D, typename RowPtr>
+template <typename T, int D, int STEPS, typename RowPtr>
 __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const float (&qv)[16 / sizeof(T)],
                                                    float* out) {
   constexpr int EPL = 16 / sizeof(T);
   constexpr int LPR = D / EPL;
-  constexpr int RPI = 32 / LPR;
-  constexpr int STEPS = 8;  // loads in flight per lane per round
+  constexpr int RPI = 32 / LPR;  // STEPS: loads in flight per lane per round
   const int lane = threadIdx.x & 31;
   const int li = lane % LPR, sub = lane / LPR;
   for (int base = 0; base < n; base += STEPS * RPI) {
@@ -552,10 +552,11 @@ __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const f
 }
 
 // Orderable 64-bit key of group `id` with score s: a larger key is a better
-// group (higher score, then smaller id); 0 = no group (score -inf).
+// group (higher score, then smaller id; the same order as comparing the
+// floats); 0 = no group (score -inf).
 __device__ __forceinline__ uint64_t group_key(float s, int64_t id) {
   if (s == -INFINITY) return 0;
-  uint32_t b = __float_as_uint(s);
+  uint32_t b = s == 0.f ? 0u : __float_as_uint(s);  // -0 orders as +0
   b ^= (b & 0x80000000u) ? 0xffffffffu : 0x80000000u;
   return ((uint64_t)b << 32) | (uint32_t)(0xffffffffu - (uint32_t)id);
 }
@@ -614,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 
   extern __shared__ __align__(128) unsigned char smem[];
   T* Vst = reinterpret_cast<T*>(smem + SM::off_V);
-  int16_t* perm_s = reinterpret_cast<int16_t*>(smem + SM::off_perm);
   float* qs = reinterpret_cast<float*>(smem + SM::off_q);
   float* gstate = reinterpret_cast<float*>(smem + SM::off_g);
   float* wstate = reinterpret_cast<float*>(smem + SM::off_w);
@@ -623,7 +623,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   int64_t* posm_s = reinterpret_cast<int64_t*>(smem + SM::off_pos);
   Cand* win = reinterpret_cast<Cand*>(smem + SM::off_c);
   int* nwin_s = reinterpret_cast<int*>(smem + SM::off_c + sizeof(Cand) * kMaxTopGroups);
-  int* nsurv_s = nwin_s + 1;
   uint64_t* keys_s = reinterpret_cast<uint64_t*>(smem + SM::off_key);
   uint64_t* wb_s = reinterpret_cast<uint64_t*>(smem + SM::off_wb);
   uint64_t* surv = reinterpret_cast<uint64_t*>(smem + SM::off_V);
@@ -652,52 +651,121 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   pdl_wait();  // the scan's partial states and candidates are visible from here on
 
   const int nsplit = a.nsplit;
-  // ---- the top-G groups of this row from the unit's score array.  A bound
-  // that G distinct groups reach (the G-th best of a warp's per-thread best
-  // keys; the largest such bound over the warps), the groups at or above it
-  // (at most G threads per warp hold any), then their exact ranks.
+  // the split states this thread merges (component c = tid of each), loaded
+  // now so that the loads overlap the group selection
+  constexpr int kPre = 8;
+  const float* ps = a.part + (u * nsplit * NQ + r) * (int64_t)(D + 2);
+  const int64_t pstride = (int64_t)NQ * (D + 2);
+  float pre_m[kPre], pre_v[kPre];
+#pragma unroll
+  for (int sp = 0; sp < kPre; ++sp) {
+    pre_m[sp] = -INFINITY;
+    pre_v[sp] = 0.f;
+    if (sp < nsplit && tid < D + 2) {
+      pre_m[sp] = ps[sp * pstride];
+      pre_v[sp] = ps[sp * pstride + tid];
+    }
+  }
+  // ---- the top-G groups of this row from the unit's score array (higher
+  // score first, then smaller id).  A bound that G distinct groups reach (the
+  // G-th best of a warp's per-thread best groups; the best such bound over the
+  // warps), the groups at or above it (at most G threads per warp hold any),
+  // then their exact ranks.
   {
     const int64_t wbq = t / kChunk - a.window / kChunk + 1;
-    const int64_t Gq = wbq > 0 ? wbq * a.k : 0;  // visible groups of this row
+    const int Gq = wbq > 0 ? (int)(wbq * a.k) : 0;  // visible groups of this row
     const float* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
-    uint64_t tb = 0;
-#pragma unroll 4
-    for (int64_t i = tid; i < Gq; i += kThreads) {
-      const uint64_t kk = group_key(srow[i], i);
-      tb = kk > tb ? kk : tb;
+    constexpr int kSel = 16;  // scores per thread kept in registers (up to 4096 groups)
+    const bool in_regs = Gq <= kSel * kThreads;
+    float sv[kSel];
+    float bs = -INFINITY;
+    int bi = 0x7fffffff;
+    if (in_regs) {
+#pragma unroll
+      for (int e = 0; e < kSel; ++e) {
+        const int i = tid + e * kThreads;
+        sv[e] = i < Gq ? srow[i] : -INFINITY;
+      }
+#pragma unroll
+      for (int e = 0; e < kSel; ++e)
+        if (sv[e] > bs) {  // first occurrence: the smaller id wins a tie
+          bs = sv[e];
+          bi = tid + e * kThreads;
+        }
+    } else {
+      for (int i = tid; i < Gq; i += kThreads) {
+        const float si = srow[i];
+        if (si > bs) {
+          bs = si;
+          bi = i;
+        }
+      }
     }
-    keys_s[tid] = tb;
-    if (tid == 0) *nsurv_s = 0;
+    const uint64_t tk = group_key(bs, bi);
+    keys_s[tid] = tk;
     __syncwarp();
     int rk = 0;
     const ulonglong2* kw = reinterpret_cast<const ulonglong2*>(keys_s + warp * 32);
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
       const ulonglong2 pq = kw[x];
-      rk += (pq.x > tb ? 1 : 0) + (pq.y > tb ? 1 : 0);
+      rk += (pq.x > tk ? 1 : 0) + (pq.y > tk ? 1 : 0);
     }
-    const unsigned at = __ballot_sync(0xffffffffu, tb != 0 && rk == a.G - 1);
+    const unsigned at = __ballot_sync(0xffffffffu, tk != 0 && rk == a.G - 1);
     if (lane == 0) wb_s[warp] = at ? keys_s[warp * 32 + __ffs(at) - 1] : 0;
     __syncthreads();
-    uint64_t lo = 1;
+    uint64_t lo = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) lo = wb_s[w] > lo ? wb_s[w] : lo;
-    for (int64_t i0 = 0; i0 < Gq; i0 += kThreads) {
-      const int64_t i = i0 + tid;
-      const uint64_t kk = i < Gq ? group_key(srow[i], i) : 0;
-      const bool keep = kk >= lo;
-      const unsigned msk = __ballot_sync(0xffffffffu, keep);
-      if (msk) {
-        const int lead = __ffs(msk) - 1;
-        int base = 0;
-        if (lane == lead) base = atomicAdd(nsurv_s, __popc(msk));
-        base = __shfl_sync(0xffffffffu, base, lead);
-        const int pos = base + __popc(msk & ((1u << lane) - 1u));
-        if (keep && pos < SM::kSurvCap) surv[pos] = kk;
+    const float lo_s = lo ? key_score(lo) : -INFINITY;
+    const int lo_i = lo ? key_id(lo) : 0x7fffffff;
+    auto at_or_above = [&](float si, int i) { return si != -INFINITY && (si > lo_s || (si == lo_s && i <= lo_i)); };
+    // survivors, compacted by a prefix count over the CTA
+    int cnt = 0;
+    if (in_regs) {
+#pragma unroll
+      for (int e = 0; e < kSel; ++e) cnt += at_or_above(sv[e], tid + e * kThreads) ? 1 : 0;
+    } else {
+      for (int i = tid; i < Gq; i += kThreads) cnt += at_or_above(srow[i], i) ? 1 : 0;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int* wtot = reinterpret_cast<int*>(keys_s);  // the keys are no longer needed
+    __syncthreads();
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt, n = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wtot[w];
+      pos += w < warp ? c : 0;
+      n += c;
+    }
+    if (cnt) {
+      if (in_regs) {
+#pragma unroll
+        for (int e = 0; e < kSel; ++e) {
+          const int i = tid + e * kThreads;
+          if (at_or_above(sv[e], i)) {
+            if (pos < SM::kSurvCap) surv[pos] = group_key(sv[e], i);
+            ++pos;
+          }
+        }
+      } else {
+        for (int i = tid; i < Gq; i += kThreads) {
+          const float si = srow[i];
+          if (at_or_above(si, i)) {
+            if (pos < SM::kSurvCap) surv[pos] = group_key(si, i);
+            ++pos;
+          }
+        }
       }
     }
     __syncthreads();
-    const int n = *nsurv_s;
     const int nwin = n < a.G ? n : a.G;
     if (n <= SM::kSurvCap) {
       for (int x = tid; x < n; x += kThreads) {
@@ -717,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       uint64_t last = ~0ull;
       for (int x = 0; x < nwin; ++x) {
         uint64_t bk = 0;
-        for (int64_t i = tid; i < Gq; i += kThreads) {
+        for (int i = tid; i < Gq; i += kThreads) {
           const uint64_t kk = group_key(srow[i], i);
           if (kk < last && kk > bk) bk = kk;
         }
@@ -730,32 +798,26 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       }
     }
     if (tid == 0) *nwin_s = nwin;
-    __syncthreads();
-    if (tid < nwin) {  // the winners' sizes and page ranges
-      const int id = win[tid].id;
-      win[tid].cnt = a.gCnt[unit_kv * a.Cmax * a.k + id];
-      const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + (id / a.k) * (a.k + 1) + id % a.k;
-      win[tid].pages = ((int)(uint16_t)gp[0]) | ((int)(uint16_t)gp[1] << 16);
-    }
   }
-  {
+  if (tid < D + 2) {
     // ---- merge the split states (thread c owns component c: m, l, acc[])
-    const float* ps = a.part + (u * nsplit * NQ + r) * (int64_t)(D + 2);
-    const int64_t stride = (int64_t)NQ * (D + 2);
     float M = -INFINITY;
-    for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, ps[sp * stride]);
-    for (int c = tid; c < D + 2; c += kThreads) {
-      float v = 0.f;
-      if (c == 0) {
-        v = M;
-      } else {
-        for (int sp = 0; sp < nsplit; ++sp) {
-          const float ms = ps[sp * stride];
-          if (ms != -INFINITY) v = fmaf(ps[sp * stride + c], __expf(ms - M), v);
-        }
+#pragma unroll
+    for (int sp = 0; sp < kPre; ++sp) M = fmaxf(M, pre_m[sp]);
+    for (int sp = kPre; sp < nsplit; ++sp) M = fmaxf(M, ps[sp * pstride]);
+    float v = 0.f;
+    if (tid == 0) {
+      v = M;
+    } else {
+#pragma unroll
+      for (int sp = 0; sp < kPre; ++sp)
+        if (pre_m[sp] != -INFINITY) v = fmaf(pre_v[sp], __expf(pre_m[sp] - M), v);
+      for (int sp = kPre; sp < nsplit; ++sp) {
+        const float ms = ps[sp * pstride];
+        if (ms != -INFINITY) v = fmaf(ps[sp * pstride + tid], __expf(ms - M), v);
       }
-      gstate[c] = v;
     }
+    gstate[tid] = v;
   }
   __syncthreads();
   const int nwin = *nwin_s;
@@ -776,33 +838,37 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   const T* pV = static_cast<const T*>(a.pV) + unit_kv * a.Cmax * a.P * D;
   const int32_t* pC = a.pCnt + unit_kv * a.Cmax * a.P;
   const int16_t* pB = a.pBeg + unit_kv * a.Cmax * a.P;
-  const int16_t* pm = a.perm + unit_kv * a.Cmax * kChunk;
+  const T* mK = static_cast<const T*>(a.mK) + unit_kv * a.Cmax * kChunk * D;
+  const T* mV = static_cast<const T*>(a.mV) + unit_kv * a.Cmax * kChunk * D;
   const T* Kb = static_cast<const T*>(a.K) + b * a.sb + kvh * a.sh;
   const T* Vb = static_cast<const T*>(a.V) + b * a.sb + kvh * a.sh;
   T* myV = Vst + warp * SM::kRows * D;
-  int16_t* myperm = perm_s + warp * kChunk;
   float* mysc = sc_s + warp * 64;
-  int64_t* mypos = posm_s + warp * 32;
+  const T** mykp = reinterpret_cast<const T**>(posm_s) + warp * 32;
+  int* mycnt = reinterpret_cast<int*>(smem + SM::off_pc) + warp * 32;
+  int* mybeg = mycnt + kWarps * 32;
   uint32_t phase = 0;
-  // One batch of up to 32 exact tokens (lane e: `ev`, position `pos`) and up
-  // to 32 coarse entries (lane p: `cvb`, logit `lgc`, value row `crow`): the
-  // value rows are staged in shared memory by TMA while the key rows are
-  // scored with coalesced loads, then everything enters the warp's online
-  // softmax state.
-  auto batch = [&](bool ev, int64_t pos, bool cvb, float lgc, const T* crow) {
+  // member key rows scored per round: all 32 of a batch for bf16 rows
+  constexpr int kMemberSteps = 8;
+  // One batch of up to 32 exact tokens (lane e: `ev`, key and value rows
+  // `krow`, `vrow`) and up to 32 coarse entries (lane p: `cvb`, logit `lgc`,
+  // value row `crow`): the value rows are staged in shared memory by TMA
+  // while the key rows are scored with coalesced loads, then everything
+  // enters the warp's online softmax state.
+  auto batch = [&](bool ev, const T* krow, const T* vrow, bool cvb, float lgc, const T* crow) {
     const unsigned vm = __ballot_sync(0xffffffffu, ev);
     const unsigned cmb = __ballot_sync(0xffffffffu, cvb);
     if (!(vm | cmb)) return;
     if (lane == 0) mbar_arrive_expect(&bar[warp], (uint32_t)(__popc(vm) + __popc(cmb)) * ROWB);
     __syncwarp();
-    if (ev) bulk_g2s(myV + lane * D, Vb + pos * a.st, ROWB, &bar[warp]);
+    if (ev) bulk_g2s(myV + lane * D, vrow, ROWB, &bar[warp]);
     if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
     // members are packed: lanes 0..nvalid-1 hold the valid ones in order
     const int nvalid = __popc(vm);
     const int my_rank = __popc(vm & ((1u << lane) - 1u));
-    if (ev) mypos[my_rank] = pos;
+    if (ev) mykp[my_rank] = krow;
     __syncwarp();
-    rows_dot_coalesced<T, D>(nvalid, [&](int i) { return Kb + mypos[i] * a.st; }, qv, mysc + 32);
+    rows_dot_coalesced<T, D, kMemberSteps>(nvalid, [&](int i) { return mykp[i]; }, qv, mysc + 32);
     __syncwarp();
     const float lge = ev ? mysc[32 + my_rank] : -INFINITY;
     const float lgcb = cvb ? lgc : -INFINITY;
@@ -847,20 +913,33 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   if (warp == kWarps - 1) {
     const int64_t wsq = (t / kChunk - a.window / kChunk + 1) > 0 ? (t / kChunk - a.window / kChunk + 1) * kChunk : 0;
     const int64_t nsk = a.sinks < wsq ? a.sinks : wsq;
-    for (int64_t e0 = 0; e0 < nsk; e0 += 32) batch(e0 + lane < nsk, e0 + lane, false, 0.f, pV);
+    for (int64_t e0 = 0; e0 < nsk; e0 += 32)
+      batch(e0 + lane < nsk, Kb + (e0 + lane) * a.st, Vb + (e0 + lane) * a.st, false, 0.f, pV);
   }
   for (int w = warp; w < nwin; w += kWarps) {
-    const Cand cw = win[w];
-    const int64_t c = cw.id / a.k;
-    const int p0 = cw.pages & 0xffff, p1 = (cw.pages >> 16) & 0xffff;
+    const float gs = win[w].s;
+    const int gid = win[w].id;
+    const int64_t c = gid / a.k;
+    // one round trip: the group's size and page range, its chunk's page
+    // counts and member runs, and its mean value
+    const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + c * (a.k + 1) + gid % a.k;
+    const int gcnt = a.gCnt[unit_kv * a.Cmax * a.k + gid];
+    const int p0 = (uint16_t)gp[0], p1 = (uint16_t)gp[1];
+    float gv[DPL];
+    load_f<T, DPL>(gV + (int64_t)gid * D + lane * DPL, gv);
+    int pcl = 0, pbl = 0;  // the chunk's page counts and member offsets (slot = lane)
+    if (lane < a.P) {
+      pcl = pC[c * a.P + lane];
+      pbl = pB[c * a.P + lane];
+    }
+    mycnt[lane] = pcl;
+    mybeg[lane] = pbl;
     int open_slot[kMaxTopPages];
 #pragma unroll
     for (int x = 0; x < kMaxTopPages; ++x) open_slot[x] = -1;
     // remove this group's coarse term: exp(s + ln n - M) * (1, gV)
-    if (cw.cnt > 0 && cw.cnt <= kChunk) {
-      const float e = __expf(cw.s + __logf((float)cw.cnt) - M);
-      float gv[DPL];
-      load_f<T, DPL>(gV + (int64_t)cw.id * D + lane * DPL, gv);
+    if (gcnt > 0 && gcnt <= kChunk) {
+      const float e = __expf(gs + __logf((float)gcnt) - M);
       dl -= e;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) dacc[i] = fmaf(-e, gv[i], dacc[i]);
@@ -871,16 +950,15 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       if (lane == 0) set_status(a.status, LOD_ST_BAD_PAGE);
     } else {
       const int np = p1 - p0;
-      // the chunk's member list, page counts/offsets, and the page summary scores
-      *reinterpret_cast<uint4*>(myperm + lane * 8) =
-          __ldg(reinterpret_cast<const uint4*>(pm + c * kChunk) + lane);
+      // page counts/offsets and the page summary scores
+      __syncwarp();
       int cntp = 0, begp = 0;
       if (lane < np) {
-        cntp = pC[c * a.P + p0 + lane];
-        begp = pB[c * a.P + p0 + lane];
+        cntp = mycnt[p0 + lane];
+        begp = mybeg[p0 + lane];
       }
       const T* pKc = pK + (c * a.P + p0) * D;
-      rows_dot_coalesced<T, D>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
+      rows_dot_coalesced<T, D, 8>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
       __syncwarp();
       const float sc = lane < np ? mysc[lane] : -INFINITY;
       // top-TP pages by (score desc, slot asc)
@@ -919,16 +997,17 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         const int n_of = __shfl_sync(0xffffffffu, cntp, sl_lane & 31);
         const int b_of = __shfl_sync(0xffffffffu, begp, sl_lane & 31);
         bool ev = x < nopen && slot >= 0 && mi < n_of;
-        if (ev && (n_of > kPage || b_of < 0 || b_of + n_of > kChunk)) {
+        if (ev && n_of > kPage) {
           set_status(a.status, LOD_ST_BAD_PAGE);
           ev = false;
         }
-        const int off = ev ? myperm[b_of + mi] : 0;
-        if (ev && (off < 0 || off >= kChunk)) {
+        if (ev && (b_of < 0 || b_of + n_of > kChunk)) {
           set_status(a.status, LOD_ST_BAD_MEMBER);
           ev = false;
         }
-        batch(ev, c * kChunk + off, bt == 0 && cv, lgc, pV + (c * a.P + p0 + lane) * D);
+        // the page's members are consecutive rows of the member-ordered copies
+        const int64_t row = c * kChunk + (ev ? b_of + mi : 0);
+        batch(ev, mK + row * D, mV + row * D, bt == 0 && cv, lgc, pV + (c * a.P + p0 + lane) * D);
       }
     }
     if (a.sel_pages && lane < a.TP) {

@@ -374,6 +374,20 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
       psum[pg * D + lane * DPL + i] = sv[i];
     }
   }
+  // member-ordered copies: row m = the token at chunk offset perm[m], so each
+  // page's members are consecutive rows (keys from shared memory, values
+  // from the rows the page sums just read)
+  {
+    constexpr int C16 = ROWB / 16;  // 16-byte pieces per row
+    uint4* mKc = reinterpret_cast<uint4*>(static_cast<T*>(a.mK) + ((unit * a.Cmax + c) * kChunk) * D);
+    uint4* mVc = reinterpret_cast<uint4*>(static_cast<T*>(a.mV) + ((unit * a.Cmax + c) * kChunk) * D);
+    for (int item = tid; item < n * C16; item += kBuildThreads) {
+      const int m = item / C16, q = item % C16;
+      const int row = first + perm_s[m];
+      mKc[item] = reinterpret_cast<const uint4*>(xs + row * D)[q];
+      mVc[item] = __ldg(reinterpret_cast<const uint4*>(Vc + (int64_t)row * a.st) + q);
+    }
+  }
   // unused page slots hold zeros
   for (int item = tid; item < (int)(P - used) * D; item += kBuildThreads) {
     const int slot = used + item / D, i = item % D;

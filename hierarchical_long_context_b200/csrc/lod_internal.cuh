@@ -29,6 +29,8 @@ struct BuildArgs {
   int16_t* pBeg;
   int16_t* gPage;
   int16_t* perm;
+  void* mK;            // member-ordered key / value copies
+  void* mV;
   uint32_t* status;    // device status word (workspace header)
 };
 
@@ -61,6 +63,8 @@ struct AttendArgs {
   const int16_t* pBeg;
   const int16_t* gPage;
   const int16_t* perm;
+  const void* mK;           // member-ordered key / value copies [..][Cmax * chunk][d]
+  const void* mV;
   int B, Hq, Hkv, g;
   int64_t Tmax, Cmax;
   int k, P, G, TP, window, sinks;

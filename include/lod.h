@@ -59,7 +59,7 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
 /* Device status bits (lod_get_status). */
 #define LOD_ST_BAD_SEQLEN 0x1u   /* seq_len outside [1, Tmax]: that row's output is zeroed */
 #define LOD_ST_BAD_PAGE 0x2u     /* page range or page slot outside the chunk's slots */
-#define LOD_ST_BAD_MEMBER 0x4u   /* member offset outside the chunk */
+#define LOD_ST_BAD_MEMBER 0x4u   /* a page's member run [pBeg, pBeg + pCnt) outside the chunk */
 #define LOD_ST_BAD_COUNT 0x8u    /* group or page count outside [0, chunk] */
 #define LOD_ST_TIMEOUT 0x10u     /* an asynchronous copy did not complete within the kernel's wait limit */
 
@@ -105,8 +105,14 @@ typedef struct lod_params {
  *   gPage   [Cmax*(k+1)]  int16 pages of group j are slots [gPage[j], gPage[j+1])
  *   perm    [Cmax*chunk]  int16 chunk-local token offsets, group-major and
  *                         ascending within a group; -1 past the last member
- * Every array is laid out [B][Hkv][...] in that order.  gK, gV, pK, pV and
- * perm must be 16-byte aligned, gCnt and pCnt 4-byte aligned.
+ *   mK, mV  [Cmax*chunk][d] member-ordered copies of the chunk's keys and
+ *                         values: row m of chunk c is the token at offset
+ *                         perm[m], so the members of a page are the
+ *                         consecutive rows [pBeg, pBeg + pCnt) and an opened
+ *                         page is read as one contiguous run (rows past the
+ *                         last member are not written)
+ * Every array is laid out [B][Hkv][...] in that order.  gK, gV, pK, pV, perm,
+ * mK and mV must be 16-byte aligned, gCnt and pCnt 4-byte aligned.
  */
 typedef struct lod_index {
   void* gK;
@@ -118,6 +124,8 @@ typedef struct lod_index {
   int16_t* pBeg;
   int16_t* gPage;
   int16_t* perm;
+  void* mK;
+  void* mV;
 } lod_index;
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -127,11 +135,12 @@ int32_t lod_version(void);
 const char* lod_last_error(void);
 
 /*
- * Byte sizes of the nine lod_index arrays, in field order (gK, gV, gCnt, pK,
- * pV, pCnt, pBeg, gPage, perm), written to bytes[0..8] (host).  Validates
- * `p` like every other entry point.
+ * Byte sizes of the eleven lod_index arrays, in field order (gK, gV, gCnt,
+ * pK, pV, pCnt, pBeg, gPage, perm, mK, mV), written to bytes[0..10] (host).
+ * Validates `p` like every other entry point.
  */
-int32_t lod_index_sizes(const lod_params* p, size_t bytes[9]);
+#define LOD_INDEX_ARRAYS 11
+int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]);
 
 /*
  * Workspace bytes needed by one call of `op` (lod_op) with parameters `p`

@@ -56,8 +56,10 @@ def unit_from_gpu(ix: api.Index, b: int, h: int, nchunks: int, p: api.Params) ->
                 perm=i(ix.perm, nchunks * C), nchunks=nchunks)
 
 
-def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params) -> None:
-    """Write an oracle-built index of one sequence into a GPU index."""
+def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params, K=None, V=None) -> None:
+    """Write an oracle-built index of one sequence into a GPU index.  K, V
+    (that sequence's cache rows, [T][d] tensors) fill the member-ordered
+    copies: row m of chunk c is the token at offset perm[m]."""
     n = u["nchunks"]
     k, P, C = p.clusters, p.page_slots, p.chunk
     dev = ix.gK.device
@@ -71,6 +73,13 @@ def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params) -> None:
     put(ix.pBeg, u["pBeg"], n * P)
     put(ix.gPage, u["gPage"], n * (k + 1))
     put(ix.perm, u["perm"], n * C)
+    if K is not None:
+        perm = torch.from_numpy(np.asarray(u["perm"][:n * C], dtype=np.int64))
+        rows = torch.arange(n * C) // C * C + perm
+        ok = perm >= 0
+        dst = torch.nonzero(ok).flatten()
+        ix.mK[b, h, dst.to(dev)] = K.to(dev)[rows[ok].to(dev)].to(ix.mK.dtype)
+        ix.mV[b, h, dst.to(dev)] = V.to(dev)[rows[ok].to(dev)].to(ix.mV.dtype)
 
 
 def assignment(u: dict, k: int, C: int = 256) -> np.ndarray:
@@ -85,6 +94,18 @@ def assignment(u: dict, k: int, C: int = 256) -> np.ndarray:
                 a[c * C + u["perm"][c * C + m]] = j
             off += cnt
     return a
+
+
+def check_member_copies(ix: api.Index, b: int, h: int, K, V, nchunks: int, p: api.Params) -> None:
+    """The member-ordered copies hold the cache rows bit for bit: row m of
+    chunk c of mK / mV is row c * chunk + perm[m] of K / V (K, V: that
+    sequence's [T][d] cache rows)."""
+    C = p.chunk
+    perm = ix.perm[b, h, :nchunks * C].long()
+    ok = perm >= 0
+    rows = torch.arange(nchunks * C, device=perm.device) // C * C + perm
+    assert torch.equal(ix.mK[b, h, :nchunks * C][ok], K.to(perm.device)[rows[ok]])
+    assert torch.equal(ix.mV[b, h, :nchunks * C][ok], V.to(perm.device)[rows[ok]])
 
 
 def check_index_consistency(u: dict, K: np.ndarray, V: np.ndarray, cfg: oracle.Config, bf16: bool):

@@ -40,7 +40,7 @@ def P(**kw):
 
 
 def _sizes(p):
-    sizes = (ctypes.c_size_t * 9)()
+    sizes = (ctypes.c_size_t * len(_lib.INDEX_FIELDS))()
     rc = _lib.load().lod_index_sizes(ctypes.byref(p.c()), sizes)
     return rc, list(sizes)
 
@@ -52,7 +52,8 @@ def test_index_sizes_match_the_documented_layout():
     Cmax, k, Pp = 4096 // 256, 4, 256 // 16 + 4
     u = 2 * 2
     assert s == [u * Cmax * k * 128 * 2] * 2 + [u * Cmax * k * 4] + [u * Cmax * Pp * 128 * 2] * 2 + \
-        [u * Cmax * Pp * 4, u * Cmax * Pp * 2, u * Cmax * (k + 1) * 2, u * Cmax * 256 * 2]
+        [u * Cmax * Pp * 4, u * Cmax * Pp * 2, u * Cmax * (k + 1) * 2, u * Cmax * 256 * 2] + \
+        [u * Cmax * 256 * 128 * 2] * 2
 
 
 @pytest.mark.parametrize("kw, code", [
@@ -109,7 +110,7 @@ def test_null_and_misaligned_pointers_fail_before_any_launch():
     rc = L.lod_build_index(ctypes.byref(p), fake, fake, bad, 0, 1, ctypes.byref(ix), fake, 256, None)
     assert rc == _lib.LOD_EINVAL
     # chunk range beyond Tmax (index pointers present, fake)
-    full = _lib.lod_index(*([1 << 20] * 9))
+    full = _lib.lod_index(*([1 << 20] * len(_lib.INDEX_FIELDS)))
     rc = L.lod_build_index(ctypes.byref(p), fake, fake, st, 0, 17, ctypes.byref(full), fake, 256, None)
     assert rc == _lib.LOD_EINVAL and b"chunk range" in L.lod_last_error()
     rc = L.lod_build_index(ctypes.byref(p), fake, fake, st, 3, 3, ctypes.byref(full), fake, 256, None)
@@ -127,7 +128,7 @@ def test_null_and_misaligned_pointers_fail_before_any_launch():
 def test_reserved_fields_must_be_zero():
     p = P().c()
     p.reserved0 = 1
-    sizes = (ctypes.c_size_t * 9)()
+    sizes = (ctypes.c_size_t * len(_lib.INDEX_FIELDS))()
     assert _lib.load().lod_index_sizes(ctypes.byref(p), sizes) == _lib.LOD_EINVAL
 
 
@@ -137,4 +138,4 @@ def test_struct_layout_matches_the_header():
     assert _lib.lod_params.scale.offset == 64
     assert _lib.lod_params.Tmax.offset == 72
     assert ctypes.sizeof(_lib.lod_params) == 80
-    assert ctypes.sizeof(_lib.lod_index) == 72
+    assert ctypes.sizeof(_lib.lod_index) == 8 * 11

@@ -111,6 +111,7 @@ def test_build_full_size(k):
         Kn, Vn = _np(K[0, h]), _np(V[0, h])
         gu = lt.unit_from_gpu(ix, 0, h, nch, p)
         lt.check_index_consistency(gu, Kn, Vn, cfg, True)
+        lt.check_member_copies(ix, 0, h, Kd[0, h], Vd[0, h], nch, p)
         ou = oracle.build_sequence(cfg, h, Kn, Vn, nch)
         st = lt.compare_builds(gu, ou, cfg, True)
         print("build k=%d kvh %d" % (k, h), st)

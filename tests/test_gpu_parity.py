@@ -61,6 +61,7 @@ def test_build_matches_oracle(name, k, T):
             K, V = _np(Kc[b, h]), _np(Vc[b, h])
             gu = lt.unit_from_gpu(ix, b, h, nch, p)
             lt.check_index_consistency(gu, K, V, cfg, w.dtype == "bf16")
+            lt.check_member_copies(ix, b, h, Kd[b, h], Vd[b, h], nch, p)
             ou = oracle.build_sequence(cfg, b * w.Hkv + h, K, V, nch)
             st = lt.compare_builds(gu, ou, cfg, w.dtype == "bf16")
             for key in tot:
@@ -135,7 +136,7 @@ def test_decode_on_oracle_index_matches_oracle():
     for b in range(w.B):
         for h in range(w.Hkv):
             ous[(b, h)] = oracle.build_sequence(cfg, b * w.Hkv + h, _np(Kc[b, h]), _np(Vc[b, h]), T // 256)
-            lt.unit_to_gpu(ix, b, h, ous[(b, h)], p)
+            lt.unit_to_gpu(ix, b, h, ous[(b, h)], p, Kd[b, h], Vd[b, h])
     rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 300], draws=4)
     st = _check_decode(w, p, Kc, Vc, ix, rows, cfg, lambda b, h, K, V, n: ous[(b, h)])
     print(st)
@@ -228,10 +229,11 @@ def test_bad_index_values_are_skipped_and_reported():
     sg = torch.empty(1, 8, p.top_groups, dtype=torch.int32, device="cuda")
     api.lod_decode(p, q, Kd, Vd, sl, ix, sel_groups=sg, ws=ws)
     assert api.lod_get_status(ws) == 0
-    # corrupt every member offset of the chunks the first head opens
+    # move every page's member run of the chunks the first head opens past the chunk end
+    P = p.page_slots
     for gid in sg[0, 0].tolist():
         c = gid // p.clusters
-        ix.perm[0, 0, c * 256:(c + 1) * 256] = 4000
+        ix.pBeg[0, 0, c * P:(c + 1) * P] = 250
     api.lod_decode(p, q, Kd, Vd, sl, ix, ws=ws)
     st = api.lod_get_status(ws)
     assert st & api._lib.LOD_ST_BAD_MEMBER

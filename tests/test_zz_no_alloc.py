@@ -36,7 +36,7 @@ def test_shapes_beyond_the_built_in_scratch_are_rejected_without_touching_a_gpu(
     p = api.Params(B=512, Hq=64, Hkv=8, d=128, Tmax=1 << 20)
     assert api.workspace_bytes(p, _lib.LOD_OP_DECODE) > _lib.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(1 << 20)
-    full = _lib.lod_index(*([1 << 20] * 9))
+    full = _lib.lod_index(*([1 << 20] * len(_lib.INDEX_FIELDS)))
     st = (ctypes.c_int64 * 3)(8 * (1 << 20) * 128, (1 << 20) * 128, 128)  # fake, never used
     rc = L.lod_decode_noalloc(ctypes.byref(p.c()), fake, fake, fake, st, fake, ctypes.byref(full), fake,
                               None, None, None, None, None)
