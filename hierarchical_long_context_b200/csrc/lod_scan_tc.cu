@@ -144,21 +144,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t grow0 = unit_kv * a.Cmax * a.k;  // this unit's first summary row
   const int32_t* gC = a.gCnt + grow0;
 
-  // ---- set-up: barriers, TMEM, the query operand, zeroed weights
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1 + 32);  // the producer's expect_tx + 32 cp.async arrivals
-      mbar_init(&empty[i], 1);
+  // producer (warp 0, all lanes): tile t0 + i into ring slot i % kStages
+  auto issue_tile = [&](int i) {
+    const int st = i % kStages;
+    const int64_t tile = t0 + i;
+    unsigned char* kd = Kring + (size_t)st * kTileBytes;
+    unsigned char* vd = Vring + (size_t)st * kTileBytes;
+    if (lane == 0) {
+      mbar_arrive_expect(&full[st], 2u * kTileBytes);
+      if (tile < gt) {
+        const int row = (int)(grow0 + tile * TROWS);
+        tc::tma_load_2d(kd, &maps.gK, 0, row, &full[st]);
+        tc::tma_load_2d(kd + kTileBytes / 2, &maps.gK, 64, row, &full[st]);
+        tc::tma_load_2d(vd, &maps.gV, 0, row, &full[st]);
+        tc::tma_load_2d(vd + kTileBytes / 2, &maps.gV, 64, row, &full[st]);
+      } else {
+        const int pos = (int)(ws + (tile - gt) * TROWS);
+        tc::tma_load_4d(kd, &maps.K, 0, pos, kvh, b, &full[st]);
+        tc::tma_load_4d(kd + kTileBytes / 2, &maps.K, 64, pos, kvh, b, &full[st]);
+        tc::tma_load_4d(vd, &maps.V, 0, pos, kvh, b, &full[st]);
+        tc::tma_load_4d(vd + kTileBytes / 2, &maps.V, 64, pos, kvh, b, &full[st]);
+      }
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&o_done[i], 1);
+    if (tile < gt) {  // member counts of the tile's groups (zero past the visible ones)
+#pragma unroll
+      for (int k4 = 0; k4 < TROWS / 32; ++k4) {
+        const int r = lane + 32 * k4;
+        const int64_t gid = tile * TROWS + r;
+        const bool v = gid < G_vis;
+        cp_async4_zfill(cnt_s + st * TROWS + r, v ? gC + gid : gC, v);
+      }
     }
-    mbar_init(fin, 1);
-    *abort_s = 0;
-    fence_mbar_init();
+    cp_async_mbar_arrive_noinc(&full[st]);
+  };
+
+  // ---- set-up: barriers and the first ring stages (warp 0), TMEM (warp 1),
+  // the query operand and zeroed weights (softmax warps)
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(&full[i], 1 + 32);  // the producer's expect_tx + 32 cp.async arrivals
+        mbar_init(&empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&s_full[i], 1);
+        mbar_init(&s_free[i], 4);
+        mbar_init(&p_full[i], 4);
+        mbar_init(&o_done[i], 1);
+      }
+      mbar_init(fin, 1);
+      *abort_s = 0;
+      fence_mbar_init();
+      tc::prefetch_tensormap(&maps.gK);
+      tc::prefetch_tensormap(&maps.gV);
+      tc::prefetch_tensormap(&maps.K);
+      tc::prefetch_tensormap(&maps.V);
+    }
+    __syncwarp();
+    for (int i = 0; i < kStages && i < ntile; ++i) issue_tile(i);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, kTmemCols);
   if (warp >= 2) {
@@ -198,45 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    if (lane == 0) {
-      tc::prefetch_tensormap(&maps.gK);
-      tc::prefetch_tensormap(&maps.gV);
-      tc::prefetch_tensormap(&maps.K);
-      tc::prefetch_tensormap(&maps.V);
-    }
-    int issued = 0;
-    for (int i = 0; i < ntile; ++i) {
-      const int st = i % kStages;
-      if (i >= kStages && !wait(&empty[st], (uint32_t)(i / kStages - 1) & 1u)) break;
-      const int64_t tile = t0 + i;
-      unsigned char* kd = Kring + (size_t)st * kTileBytes;
-      unsigned char* vd = Vring + (size_t)st * kTileBytes;
-      if (lane == 0) {
-        mbar_arrive_expect(&full[st], 2u * kTileBytes);
-        if (tile < gt) {
-          const int row = (int)(grow0 + tile * TROWS);
-          tc::tma_load_2d(kd, &maps.gK, 0, row, &full[st]);
-          tc::tma_load_2d(kd + kTileBytes / 2, &maps.gK, 64, row, &full[st]);
-          tc::tma_load_2d(vd, &maps.gV, 0, row, &full[st]);
-          tc::tma_load_2d(vd + kTileBytes / 2, &maps.gV, 64, row, &full[st]);
-        } else {
-          const int pos = (int)(ws + (tile - gt) * TROWS);
-          tc::tma_load_4d(kd, &maps.K, 0, pos, kvh, b, &full[st]);
-          tc::tma_load_4d(kd + kTileBytes / 2, &maps.K, 64, pos, kvh, b, &full[st]);
-          tc::tma_load_4d(vd, &maps.V, 0, pos, kvh, b, &full[st]);
-          tc::tma_load_4d(vd + kTileBytes / 2, &maps.V, 64, pos, kvh, b, &full[st]);
-        }
-      }
-      if (tile < gt) {  // member counts of the tile's groups (zero past the visible ones)
-#pragma unroll
-        for (int k4 = 0; k4 < TROWS / 32; ++k4) {
-          const int r = lane + 32 * k4;
-          const int64_t gid = tile * TROWS + r;
-          const bool v = gid < G_vis;
-          cp_async4_zfill(cnt_s + st * TROWS + r, v ? gC + gid : gC, v);
-        }
-      }
-      cp_async_mbar_arrive_noinc(&full[st]);
+    int issued = ntile < kStages ? ntile : kStages;  // issued during the set-up
+    for (int i = kStages; i < ntile; ++i) {
+      if (!wait(&empty[i % kStages], (uint32_t)(i / kStages - 1) & 1u)) break;
+      issue_tile(i);
       ++issued;
     }
     cp_async_wait_all();
