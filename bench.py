@@ -114,6 +114,37 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- helpers
 
+def csrc_hash() -> str:
+    """SHA-256 over the library's CUDA sources (file names and contents)."""
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "hierarchical_long_context_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kind: str, workload: str):
+    """DRAM bytes (read + write) per launch from the committed ncu summary
+    profiles/<kind>_<workload>.md, or None when that summary is missing or was
+    captured from CUDA sources other than the current ones."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kind, workload))
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as fh:
+        for line in fh:
+            for key in ("traffic_bytes_per_launch:", "csrc_sha256:"):
+                if line.strip().startswith(key):
+                    vals[key] = line.strip()[len(key):].strip().split()[0]
+    if vals.get("csrc_sha256:") != csrc_hash() or "traffic_bytes_per_launch:" not in vals:
+        return None
+    return int(vals["traffic_bytes_per_launch:"])
+
+
 def l2_flusher(dev):
     buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     return lambda: buf.zero_()
@@ -227,7 +258,7 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
         status_word=status,
         roofline=dict(bound="hbm", kernel="lod_decode (scan + refine kernels)", achieved=achieved,
                       peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved / peaks["hbm_gbs"],
-                      traffic=None, algorithmic_bytes_per_launch=touched,
+                      traffic=profiled_traffic("lod_decode", w.name), algorithmic_bytes_per_launch=touched,
                       peak_source=peaks["source"], nominal_peak_gbs=8000.0),
         e2e=dict(value=world * w.B / (e2e_ms * 1e-3), unit="queries/s",
                  h2d_bytes_per_step=qh.numel() * qh.element_size() + newkv.numel() * newkv.element_size(),

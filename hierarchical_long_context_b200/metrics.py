@@ -8,9 +8,10 @@ Decode, per (sequence b, KV head) and for its g query heads at position t:
   * every visible, non-empty group summary: mean key + mean value + count;
   * the window [ws, t] and the sinks: one K row and one V row per token;
   * for the union of the opened groups: every page mean key, the page mean
-    values of pages left unopened by some head, page counts/offsets, the
-    group's page range and the member offsets of the opened pages;
-  * the K and V rows of the union of opened pages' members;
+    values of pages left unopened by some head, page counts/offsets and the
+    group's page range;
+  * the K and V rows of the union of opened pages' members (read from the
+    member-ordered copies, one contiguous run per page);
   * the queries and outputs.
 """
 from __future__ import annotations
@@ -60,7 +61,7 @@ def decode_touched_bytes(p, index, seq_lens, sel_groups, sel_pages) -> int:
                         total += row
             for pid in opened:
                 n = int(pCnt[b, h, pid])
-                total += n * (2 + 2 * row)  # member offsets, K and V rows
+                total += n * 2 * row  # K and V rows (one contiguous run per page)
     return total
 
 
@@ -100,13 +101,15 @@ def prefill_flops(p, q_begin: int, Tq: int) -> float:
 
 
 def build_bytes(p, nchunks: int) -> int:
-    """Bytes of one lod_build_index call over nchunks chunks of every sequence:
-    read K and V once, write the summaries, counts, offsets and member lists."""
+    """Bytes of one lod_build_index call over chunks [0, nchunks) of every
+    sequence: read K and V once, write the summaries, counts, offsets, member
+    lists and the member-ordered K/V copies (every clustered token once)."""
     e = 4 if str(p.dtype).endswith("float32") else 2
     units = p.B * p.Hkv
     k, P, C, d = p.clusters, p.page_slots, p.chunk, p.d
     per_chunk = 2 * C * d * e + 2 * k * d * e + k * 4 + 2 * P * d * e + P * (4 + 2) + (k + 1) * 2 + C * 2
-    return units * nchunks * per_chunk
+    copies = 2 * (nchunks * C - (p.sinks if nchunks else 0)) * d * e
+    return units * (nchunks * per_chunk + copies)
 
 
 def build_flops(p, nchunks: int) -> float:
