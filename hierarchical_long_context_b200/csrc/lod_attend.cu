@@ -560,6 +560,12 @@ __device__ __forceinline__ uint64_t group_key(float s, int64_t id) {
   b ^= (b & 0x80000000u) ? 0xffffffffu : 0x80000000u;
   return ((uint64_t)b << 32) | (uint32_t)(0xffffffffu - (uint32_t)id);
 }
+// Orderable 32-bit key of a score (larger = better; -0 as +0); 0 = -inf.
+__device__ __forceinline__ uint32_t okey32(float s) {
+  if (s == -INFINITY) return 0u;
+  const uint32_t b = s == 0.f ? 0u : __float_as_uint(s);
+  return b ^ ((b & 0x80000000u) ? 0xffffffffu : 0x80000000u);
+}
 __device__ __forceinline__ float key_score(uint64_t k) {
   uint32_t b = (uint32_t)(k >> 32);
   b = (b & 0x80000000u) ? (b ^ 0x80000000u) : ~b;
@@ -668,9 +674,9 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   }
   // ---- the top-G groups of this row from the unit's score array (higher
   // score first, then smaller id).  A bound that G distinct groups reach (the
-  // G-th best of a warp's per-thread best groups; the best such bound over the
-  // warps), the groups at or above it (at most G threads per warp hold any),
-  // then their exact ranks.
+  // G-th largest of a warp's per-thread best scores; the largest such bound
+  // over the warps), the groups scoring at or above it (a few dozen), then
+  // their exact ranks by (score, id).
   {
     const int64_t wbq = t / kChunk - a.window / kChunk + 1;
     const int Gq = wbq > 0 ? (int)(wbq * a.k) : 0;  // visible groups of this row
@@ -701,73 +707,83 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         }
       }
     }
-    const uint64_t tk = group_key(bs, bi);
-    keys_s[tid] = tk;
-    __syncwarp();
-    int rk = 0;
-    const ulonglong2* kw = reinterpret_cast<const ulonglong2*>(keys_s + warp * 32);
-#pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      const ulonglong2 pq = kw[x];
-      rk += (pq.x > tk ? 1 : 0) + (pq.y > tk ? 1 : 0);
+    // the warp's G-th largest per-thread best (32-bit orderable score; equal
+    // scores counted with their multiplicity): G distinct groups reach it
+    const uint32_t tb32 = okey32(bs);
+    uint32_t kk = tb32, wbound = 0;
+    int cum = 0;
+    for (int it = 0; it < a.G; ++it) {
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, kk);
+      if (mx == 0u) break;
+      const unsigned eq = __ballot_sync(0xffffffffu, kk == mx);
+      cum += __popc(eq);
+      if (kk == mx) kk = 0u;
+      if (cum >= a.G) {
+        wbound = mx;
+        break;
+      }
     }
-    const unsigned at = __ballot_sync(0xffffffffu, tk != 0 && rk == a.G - 1);
-    if (lane == 0) wb_s[warp] = at ? keys_s[warp * 32 + __ffs(at) - 1] : 0;
+    uint32_t* wb32 = reinterpret_cast<uint32_t*>(wb_s);
+    int* wtot = reinterpret_cast<int*>(keys_s);
+    if (lane == 0) wb32[warp] = wbound;
     __syncthreads();
-    uint64_t lo = 0;
+    uint32_t lo = 1u;  // groups with a score at or above the bound survive
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) lo = wb_s[w] > lo ? wb_s[w] : lo;
-    const float lo_s = lo ? key_score(lo) : -INFINITY;
-    const int lo_i = lo ? key_id(lo) : 0x7fffffff;
-    auto at_or_above = [&](float si, int i) { return si != -INFINITY && (si > lo_s || (si == lo_s && i <= lo_i)); };
-    // survivors, compacted by a prefix count over the CTA
-    int cnt = 0;
+    for (int w = 0; w < kWarps; ++w) lo = max(lo, wb32[w]);
+    // survivors: per-slot ballots give each warp its count and each lane its offset
+    const uint32_t lt = (1u << lane) - 1u;
+    int n = 0;
     if (in_regs) {
+      uint32_t msk[kSel];
+      int wcount = 0;
 #pragma unroll
-      for (int e = 0; e < kSel; ++e) cnt += at_or_above(sv[e], tid + e * kThreads) ? 1 : 0;
-    } else {
-      for (int i = tid; i < Gq; i += kThreads) cnt += at_or_above(srow[i], i) ? 1 : 0;
-    }
-    int incl = cnt;
+      for (int e = 0; e < kSel; ++e) {
+        msk[e] = __ballot_sync(0xffffffffu, okey32(sv[e]) >= lo);
+        wcount += __popc(msk[e]);
+      }
+      if (lane == 0) wtot[warp] = wcount;
+      __syncthreads();
+      int base = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int* wtot = reinterpret_cast<int*>(keys_s);  // the keys are no longer needed
-    __syncthreads();
-    if (lane == 31) wtot[warp] = incl;
-    __syncthreads();
-    int pos = incl - cnt, n = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = wtot[w];
+        base += w < warp ? c : 0;
+        n += c;
+      }
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const int c = wtot[w];
-      pos += w < warp ? c : 0;
-      n += c;
-    }
-    if (cnt) {
-      if (in_regs) {
-#pragma unroll
-        for (int e = 0; e < kSel; ++e) {
-          const int i = tid + e * kThreads;
-          if (at_or_above(sv[e], i)) {
-            if (pos < SM::kSurvCap) surv[pos] = group_key(sv[e], i);
-            ++pos;
-          }
+      for (int e = 0; e < kSel; ++e) {
+        if ((msk[e] >> lane) & 1u) {
+          const int pos = base + __popc(msk[e] & lt);
+          if (pos < SM::kSurvCap) surv[pos] = group_key(sv[e], tid + e * kThreads);
         }
-      } else {
-        for (int i = tid; i < Gq; i += kThreads) {
-          const float si = srow[i];
-          if (at_or_above(si, i)) {
-            if (pos < SM::kSurvCap) surv[pos] = group_key(si, i);
-            ++pos;
-          }
+        base += __popc(msk[e]);
+      }
+    } else {
+      if (tid == 0) wtot[kWarps] = 0;
+      __syncthreads();
+      for (int i = tid; i < Gq; i += kThreads) {
+        const float si = srow[i];
+        if (okey32(si) >= lo) {
+          const int pos = atomicAdd(&wtot[kWarps], 1);
+          if (pos < SM::kSurvCap) surv[pos] = group_key(si, i);
         }
       }
     }
     __syncthreads();
+    if (!in_regs) n = wtot[kWarps];
     const int nwin = n < a.G ? n : a.G;
-    if (n <= SM::kSurvCap) {
+    if (n <= 64) {  // four threads rank each survivor
+      const int x = tid >> 2, qq = tid & 3;
+      const uint64_t kx = x < n ? surv[x] : 0ull;
+      int rx = 0;
+      for (int y = qq; y < n; y += 4) rx += surv[y] > kx ? 1 : 0;
+      rx += __shfl_xor_sync(0xffffffffu, rx, 1);
+      rx += __shfl_xor_sync(0xffffffffu, rx, 2);
+      if (x < n && qq == 0 && rx < nwin) {
+        win[rx].s = key_score(kx);
+        win[rx].id = key_id(kx);
+      }
+    } else if (n <= SM::kSurvCap) {
       for (int x = tid; x < n; x += kThreads) {
         const uint64_t kx = surv[x];
         int rx = 0, y = 0;
@@ -786,8 +802,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       for (int x = 0; x < nwin; ++x) {
         uint64_t bk = 0;
         for (int i = tid; i < Gq; i += kThreads) {
-          const uint64_t kk = group_key(srow[i], i);
-          if (kk < last && kk > bk) bk = kk;
+          const uint64_t kv = group_key(srow[i], i);
+          if (kv < last && kv > bk) bk = kv;
         }
         bk = block_max_key(bk, wb_s);
         if (tid == 0) {
