@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int li = lane % LPR, sub = lane / LPR;
+  pdl_wait();  // inputs are read only after the preceding kernel completed
+  pdl_launch_dependents();
   const UnitInfo ui = unit_info(a, u);
 
   extern __shared__ __align__(128) unsigned char smem[];
@@ -481,7 +483,6 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
     }
     part[idx] = v;
   }
-  pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------ refine
@@ -654,7 +655,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   }
   if (tid < kWarps) mbar_init(&bar[tid], 1);
   if (tid == 0) fence_mbar_init();
-  pdl_wait();  // the scan's partial states and candidates are visible from here on
+  pdl_wait();  // the scan's partial states and group scores are visible from here on
+  pdl_launch_dependents();
 
   const int nsplit = a.nsplit;
   // the split states this thread merges (component c = tid of each), loaded
@@ -1094,8 +1096,7 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
       const size_t smem = ScanSmem<T, D, NQ>::bytes;
       e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      sk<<<dim3((unsigned)a.units, (unsigned)nsplit), kThreads, smem, stream>>>(a);
-      e = cudaGetLastError();
+      e = launch_pdl(sk, dim3((unsigned)a.units, (unsigned)nsplit), dim3(kThreads), smem, stream, a);
     } else {
       return cudaErrorInvalidValue;
     }

@@ -4,6 +4,8 @@
 
 #include <cuda.h>
 
+#include <utility>
+
 #include "lod_common.cuh"
 
 namespace lod {
@@ -33,6 +35,26 @@ struct BuildArgs {
   void* mV;
   uint32_t* status;    // device status word (workspace header)
 };
+
+// Launch `kern` as a programmatic dependent of the preceding work in `stream`
+// (it may start before that work completes and must call pdl_wait before
+// reading anything it produced).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
 
 // Scan CTAs a decode call aims for: two resident CTAs on each of the B200's 148 SMs.
 constexpr int kTargetCtas = 2 * 148;

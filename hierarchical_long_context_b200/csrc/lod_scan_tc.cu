@@ -73,6 +73,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t u = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // launched as a programmatic dependent: inputs are read only after the
+  // preceding kernel has completed; the refine kernel may launch right away
+  // (it waits for this grid's completion before reading what it writes)
+  pdl_wait();
+  pdl_launch_dependents();
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -444,7 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
-  pdl_launch_dependents();
 }
 
 template <int NQ>
@@ -453,8 +457,7 @@ cudaError_t launch_nq(const AttendArgs& a, const TcMaps& maps, cudaStream_t stre
   const size_t smem = TcSmem::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((unsigned)a.units, (unsigned)a.nsplit), kThreads, smem, stream>>>(maps, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)a.units, (unsigned)a.nsplit), dim3(kThreads), smem, stream, maps, a);
 }
 
 }  // namespace
