@@ -108,92 +108,6 @@ __device__ __forceinline__ void warp_best(float& s, int& id) {
   }
 }
 
-// A warp-held sorted top-KG list: lane k < KG holds entry k (best first).
-// Merge NV new (score, id) pairs per lane (invalid ones carry id INT_MAX and
-// -inf) into it, keeping the best KG by (score desc, id asc).  Few newcomers
-// are inserted one at a time; many are merged in KG rounds of warp argmax.
-template <int KG, int NV>
-__device__ __forceinline__ void topk_merge(float (&ns)[NV], int (&ni)[NV], float& c_s, int& c_i, float& thr_s,
-                                           int& thr_i) {
-  const int lane = threadIdx.x & 31;
-  bool live[NV];
-  int n = 0;
-#pragma unroll
-  for (int q = 0; q < NV; ++q) {
-    live[q] = ni[q] != 0x7fffffff && cand_better(ns[q], ni[q], thr_s, thr_i);
-    n += __popc(__ballot_sync(0xffffffffu, live[q]));
-  }
-  if (n == 0) return;
-  if (n <= 4) {
-#pragma unroll
-    for (int q = 0; q < NV; ++q) {
-      unsigned want = __ballot_sync(0xffffffffu, live[q]);
-      while (want) {
-        const int src = __ffs(want) - 1;
-        want &= want - 1;
-        const float s = __shfl_sync(0xffffffffu, ns[q], src);
-        const int id = __shfl_sync(0xffffffffu, ni[q], src);
-        if (!cand_better(s, id, thr_s, thr_i)) continue;
-        const bool beats = lane < KG && cand_better(s, id, c_s, c_i);
-        const int at = __ffs(__ballot_sync(0xffffffffu, beats)) - 1;
-        const float up_s = __shfl_up_sync(0xffffffffu, c_s, 1);
-        const int up_i = __shfl_up_sync(0xffffffffu, c_i, 1);
-        if (lane < KG && lane > at) {
-          c_s = up_s;
-          c_i = up_i;
-        }
-        if (lane == at) {
-          c_s = s;
-          c_i = id;
-        }
-        thr_s = __shfl_sync(0xffffffffu, c_s, KG - 1);
-        thr_i = __shfl_sync(0xffffffffu, c_i, KG - 1);
-      }
-    }
-    return;
-  }
-  // KG rounds: each lane offers its best remaining (newcomers and its list entry)
-  float ls = lane < KG ? c_s : -INFINITY;
-  int lid = lane < KG ? c_i : 0x7fffffff;
-#pragma unroll
-  for (int q = 0; q < NV; ++q)
-    if (!live[q]) {
-      ns[q] = -INFINITY;
-      ni[q] = 0x7fffffff;
-    }
-  float out_s = -INFINITY;
-  int out_i = 0x7fffffff;
-  for (int k = 0; k < KG; ++k) {
-    float bs = ls;
-    int bi = lid;
-#pragma unroll
-    for (int q = 0; q < NV; ++q)
-      if (cand_better(ns[q], ni[q], bs, bi)) {
-        bs = ns[q];
-        bi = ni[q];
-      }
-    warp_best(bs, bi);
-    if (lane == k) {
-      out_s = bs;
-      out_i = bi;
-    }
-    if (lid == bi) {
-      ls = -INFINITY;
-      lid = 0x7fffffff;
-    }
-#pragma unroll
-    for (int q = 0; q < NV; ++q)
-      if (ni[q] == bi) {
-        ns[q] = -INFINITY;
-        ni[q] = 0x7fffffff;
-      }
-  }
-  c_s = out_s;
-  c_i = out_i;
-  thr_s = __shfl_sync(0xffffffffu, c_s, KG - 1);
-  thr_i = __shfl_sync(0xffffffffu, c_i, KG - 1);
-}
-
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
