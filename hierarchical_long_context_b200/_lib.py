@@ -36,7 +36,7 @@ class lod_params(ctypes.Structure):
 
 class lod_index(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("gK", "gV", "gCnt", "pK", "pV", "pCnt", "pBeg", "gPage", "perm", "mK", "mV")]
+                ("gK", "gV", "gCnt", "pK", "pV", "pCnt", "pBeg", "gPage", "perm", "mK", "mV", "gMeta")]
 
 
 INDEX_FIELDS = [f for f, _ in lod_index._fields_]

@@ -53,7 +53,7 @@ class Params:
 
 
 class Index:
-    """The eleven device arrays of lod_index, as torch tensors."""
+    """The twelve device arrays of lod_index, as torch tensors."""
 
     def __init__(self, params: Params, device="cuda"):
         lib = load()
@@ -73,6 +73,7 @@ class Index:
         self.perm = torch.full((*u, Cmax * p.chunk), -1, dtype=torch.int16, device=device)
         self.mK = torch.zeros(*u, Cmax * p.chunk, d, dtype=p.dtype, device=device)
         self.mV = torch.zeros_like(self.mK)
+        self.gMeta = torch.zeros(*u, Cmax * k, dtype=torch.int32, device=device)
         for i, f in enumerate(_lib.INDEX_FIELDS):
             t = getattr(self, f)
             assert t.numel() * t.element_size() == sizes[i], (f, t.numel() * t.element_size(), sizes[i])

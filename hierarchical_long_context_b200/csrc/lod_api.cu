@@ -82,14 +82,14 @@ int32_t validate_kv(const lod_params* p, const void* K, const void* V, const int
 int32_t validate_index(const lod_index* ix) {
   if (!ix) return fail(LOD_EINVAL, "index is NULL");
   const void* ptrs[LOD_INDEX_ARRAYS] = {ix->gK,   ix->gV,    ix->gCnt, ix->pK, ix->pV, ix->pCnt,
-                                        ix->pBeg, ix->gPage, ix->perm, ix->mK, ix->mV};
+                                        ix->pBeg, ix->gPage, ix->perm, ix->mK, ix->mV, ix->gMeta};
   for (int i = 0; i < LOD_INDEX_ARRAYS; ++i) {
     if (!ptrs[i]) return fail(LOD_EINVAL, "index field %d is NULL", i);
     if (i == 0 || i == 1 || i == 3 || i == 4 || i == 9 || i == 10) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index summary %d must be 16-byte aligned", i);
     } else if (i == 8) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index member list (perm) must be 16-byte aligned");
-    } else if ((i == 2 || i == 5) && (reinterpret_cast<uintptr_t>(ptrs[i]) & 3u)) {
+    } else if ((i == 2 || i == 5 || i == 11) && (reinterpret_cast<uintptr_t>(ptrs[i]) & 3u)) {
       return fail(LOD_EINVAL, "index field %d misaligned", i);
     } else if (reinterpret_cast<uintptr_t>(ptrs[i]) & 1u) {
       return fail(LOD_EINVAL, "index field %d misaligned", i);
@@ -192,7 +192,7 @@ int32_t make_tc_maps(const lod_params* p, const void* K, const void* V, const in
 
 size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
-  size_t gsc = sizeof(float) * (size_t)s.units * s.NQ * (size_t)(p->Tmax / p->chunk) * p->clusters;
+  size_t gsc = sizeof(float2) * (size_t)s.units * s.NQ * (size_t)(p->Tmax / p->chunk) * p->clusters;
   return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((gsc + 255) & ~size_t(255));
 }
 
@@ -215,6 +215,7 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   a.perm = ix->perm;
   a.mK = ix->mK;
   a.mV = ix->mV;
+  a.gMeta = ix->gMeta;
   a.B = p->B;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
@@ -236,7 +237,7 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
   part = (part + 255) & ~size_t(255);
   a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
-  a.gsc = reinterpret_cast<float*>(w + lod::kWsHeader + part);
+  a.gsc = reinterpret_cast<float2*>(w + lod::kWsHeader + part);
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
@@ -267,6 +268,7 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.perm = ix->perm;
   a.mK = ix->mK;
   a.mV = ix->mV;
+  a.gMeta = ix->gMeta;
   a.status = static_cast<uint32_t*>(ws);
   cudaError_t e = lod::launch_build(a, p->dtype, p->d, c1 - c0, p->B, stream);
   if (e != cudaSuccess) return cuda_fail(e, "index build launch");
@@ -295,6 +297,7 @@ int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]) {
   bytes[7] = units * Cmax * (k + 1) * sizeof(int16_t);
   bytes[8] = units * Cmax * p->chunk * sizeof(int16_t);
   bytes[9] = bytes[10] = units * Cmax * p->chunk * d * e;
+  bytes[11] = units * Cmax * k * sizeof(int32_t);
   g_err[0] = 0;
   return LOD_OK;
 }

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
   const T* Vb = static_cast<const T*>(a.V) + ui.b * a.sb + ui.kvh * a.sh;
   const T* gK = static_cast<const T*>(a.gK) + unit_kv * a.Cmax * a.k * D;
   const T* gV = static_cast<const T*>(a.gV) + unit_kv * a.Cmax * a.k * D;
-  const int32_t* gC = a.gCnt + unit_kv * a.Cmax * a.k;
+  const int32_t* gM = a.gMeta + unit_kv * a.Cmax * a.k;  // size | page range per group
   const int64_t gcap = a.Cmax * a.k;
   const bool contiguous = a.st == D;
 
@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
       }
     }
   };
-  // row metadata of slab i (log count, -inf = skip; token position or -1)
+  // row metadata of slab i (log count, -inf = skip; token position, or
+  // -2 - gMeta word for a group)
   auto meta = [&](int i, int r) {
     const int st = i % kStages;
     const int64_t e = e0 + (int64_t)i * kSlab + r;
@@ -256,9 +257,11 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
     int64_t p = -1;
     if (e < e1) {
       if (e < G_vis) {
-        const int cnt = gC[e];
+        const int mt = gM[e];
+        const int cnt = mt & 0xffff;
         if (cnt > 0 && cnt <= kChunk) lc = __logf((float)cnt);
         else if (cnt > kChunk) set_status(a.status, LOD_ST_BAD_COUNT);
+        p = -2 - (int64_t)mt;
       } else {
         p = row_pos(e, G_vis, ns, ws);
         lc = 0.f;
@@ -399,11 +402,13 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(AttendArgs a) {
       m_run = mn;
       if (lane == 0) corr_s[r] = corr;
       // group scores (-inf: not in this query row's softmax)
-      float* gsr = a.gsc + (u * NQ + r) * gcap;
+      float2* gsr = a.gsc + (u * NQ + r) * gcap;
 #pragma unroll
       for (int x = 0; x < kSlab / 32; ++x) {
         const int row = lane + 32 * x;
-        if (row < n && pos_s[st * kSlab + row] < 0) gsr[r0 + row] = live[x] ? sc[x] : -INFINITY;
+        const int64_t pr = pos_s[st * kSlab + row];
+        if (row < n && pr < 0)
+          gsr[r0 + row] = make_float2(live[x] ? sc[x] : -INFINITY, __int_as_float((int)(-2 - pr)));
       }
     }
     __syncthreads();
@@ -682,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   {
     const int64_t wbq = t / kChunk - a.window / kChunk + 1;
     const int Gq = wbq > 0 ? (int)(wbq * a.k) : 0;  // visible groups of this row
-    const float* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
+    const float2* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
     constexpr int kSel = 16;  // scores per thread kept in registers (up to 4096 groups)
     const bool in_regs = Gq <= kSel * kThreads;
     float sv[kSel];
@@ -692,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 #pragma unroll
       for (int e = 0; e < kSel; ++e) {
         const int i = tid + e * kThreads;
-        sv[e] = i < Gq ? srow[i] : -INFINITY;
+        sv[e] = i < Gq ? srow[i].x : -INFINITY;
       }
 #pragma unroll
       for (int e = 0; e < kSel; ++e)
@@ -702,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         }
     } else {
       for (int i = tid; i < Gq; i += kThreads) {
-        const float si = srow[i];
+        const float si = srow[i].x;
         if (si > bs) {
           bs = si;
           bi = i;
@@ -764,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       if (tid == 0) wtot[kWarps] = 0;
       __syncthreads();
       for (int i = tid; i < Gq; i += kThreads) {
-        const float si = srow[i];
+        const float si = srow[i].x;
         if (okey32(si) >= lo) {
           const int pos = atomicAdd(&wtot[kWarps], 1);
           if (pos < SM::kSurvCap) surv[pos] = group_key(si, i);
@@ -804,7 +809,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       for (int x = 0; x < nwin; ++x) {
         uint64_t bk = 0;
         for (int i = tid; i < Gq; i += kThreads) {
-          const uint64_t kv = group_key(srow[i], i);
+          const uint64_t kv = group_key(srow[i].x, i);
           if (kv < last && kv > bk) bk = kv;
         }
         bk = block_max_key(bk, wb_s);
@@ -938,11 +943,12 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const float gs = win[w].s;
     const int gid = win[w].id;
     const int64_t c = gid / a.k;
-    // one round trip: the group's size and page range, its chunk's page
-    // counts and member runs, and its mean value
-    const int16_t* gp = a.gPage + unit_kv * a.Cmax * (a.k + 1) + c * (a.k + 1) + gid % a.k;
-    const int gcnt = a.gCnt[unit_kv * a.Cmax * a.k + gid];
-    const int p0 = (uint16_t)gp[0], p1 = (uint16_t)gp[1];
+    // size and page range: the gMeta word the scan stored beside the score
+    const int meta = __float_as_int(a.gsc[(u * NQ + r) * (a.Cmax * a.k) + gid].y);
+    const int gcnt = meta & 0xffff;
+    const int p0 = (meta >> 16) & 0xff, p1 = (meta >> 24) & 0xff;
+    // one round trip: the chunk's page counts and member runs, the group's
+    // mean value and its pages' summary scores
     float gv[DPL];
     load_f<T, DPL>(gV + (int64_t)gid * D + lane * DPL, gv);
     int pcl = 0, pbl = 0;  // the chunk's page counts and member offsets (slot = lane)
@@ -950,6 +956,10 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       pcl = pC[c * a.P + lane];
       pbl = pB[c * a.P + lane];
     }
+    const bool prange_ok = !(p1 < p0 || p1 > a.P || p1 - p0 > 32);
+    const int np = prange_ok ? p1 - p0 : 0;
+    const T* pKc = pK + (c * a.P + (prange_ok ? p0 : 0)) * D;
+    rows_dot_coalesced<T, D, 8>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
     mycnt[lane] = pcl;
     mybeg[lane] = pbl;
     int open_slot[kMaxTopPages];
@@ -964,10 +974,9 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     } else {
       if (lane == 0) set_status(a.status, LOD_ST_BAD_COUNT);
     }
-    if (p1 < p0 || p1 > a.P || p1 - p0 > 32) {
+    if (!prange_ok) {
       if (lane == 0) set_status(a.status, LOD_ST_BAD_PAGE);
     } else {
-      const int np = p1 - p0;
       // page counts/offsets and the page summary scores
       __syncwarp();
       int cntp = 0, begp = 0;
@@ -975,9 +984,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         cntp = mycnt[p0 + lane];
         begp = mybeg[p0 + lane];
       }
-      const T* pKc = pK + (c * a.P + p0) * D;
-      rows_dot_coalesced<T, D, 8>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
-      __syncwarp();
       const float sc = lane < np ? mysc[lane] : -INFINITY;
       // top-TP pages by (score desc, slot asc)
       float s2 = sc;

@@ -321,7 +321,10 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
 
   perm[tid] = tid < n ? (int16_t)(first + perm_s[tid]) : (int16_t)-1;
   if (tid <= k) gPage[tid] = (int16_t)pstart[tid];
-  if (tid < k) gCnt[tid] = cnt[tid];
+  if (tid < k) {
+    gCnt[tid] = cnt[tid];
+    a.gMeta[unit * a.Cmax * k + c * k + tid] = cnt[tid] | (pstart[tid] << 16) | (pstart[tid + 1] << 24);
+  }
   const int used = pstart[k];
   if (tid < P) {
     if (tid < used) {

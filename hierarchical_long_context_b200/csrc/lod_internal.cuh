@@ -33,6 +33,7 @@ struct BuildArgs {
   int16_t* perm;
   void* mK;            // member-ordered key / value copies
   void* mV;
+  int32_t* gMeta;      // size | first page << 16 | end page << 24 per group
   uint32_t* status;    // device status word (workspace header)
 };
 
@@ -87,6 +88,7 @@ struct AttendArgs {
   const int16_t* perm;
   const void* mK;           // member-ordered key / value copies [..][Cmax * chunk][d]
   const void* mV;
+  const int32_t* gMeta;     // size | first page << 16 | end page << 24 per group
   int B, Hq, Hkv, g;
   int64_t Tmax, Cmax;
   int k, P, G, TP, window, sinks;
@@ -94,8 +96,9 @@ struct AttendArgs {
   int nsplit;               // splits of each unit's row list (groups, sinks, window)
   int64_t units;            // scan units in this launch
   float* part;              // [units][nsplit][NQ][d+2]  (m, l, acc)
-  float* gsc;               // [units][NQ][Cmax * k] group scores scale * q . mean k of the
-                            // unit's visible groups (-inf: not in that query row's softmax)
+  float2* gsc;              // [units][NQ][Cmax * k] (score, meta) per visible group: score =
+                            // scale * q . mean k (-inf: not in that query row's softmax),
+                            // meta = the group's gMeta word (as float bits)
   void* out;                // [B][Hq][Tq][d]
   float* lse;               // [B][Hq][Tq] or null
   int32_t* sel_groups;      // [B][Hq][Tq][G] or null

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int ntile = (int)(t1 - t0);
   const int64_t grow0 = unit_kv * a.Cmax * a.k;  // this unit's first summary row
-  const int32_t* gC = a.gCnt + grow0;
+  const int32_t* gM = a.gMeta + grow0;  // size | page range per group
 
   // producer (warp 0, all lanes): tile t0 + i into ring slot i % kStages
   auto issue_tile = [&](int i) {
@@ -171,13 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_4d(vd + kTileBytes / 2, &maps.V, 64, pos, kvh, b, &full[st]);
       }
     }
-    if (tile < gt) {  // member counts of the tile's groups (zero past the visible ones)
+    if (tile < gt) {  // the tile's groups' size and page range (zero past the visible ones)
 #pragma unroll
       for (int k4 = 0; k4 < TROWS / 32; ++k4) {
         const int r = lane + 32 * k4;
         const int64_t gid = tile * TROWS + r;
         const bool v = gid < G_vis;
-        cp_async4_zfill(cnt_s + st * TROWS + r, v ? gC + gid : gC, v);
+        cp_async4_zfill(cnt_s + st * TROWS + r, v ? gM + gid : gM, v);
       }
     }
     cp_async_mbar_arrive_noinc(&full[st]);
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l[j] = 0.f;
     }
     const int64_t gcap = a.Cmax * a.k;
-    float* gsc = a.gsc + u * NQ * gcap;  // this unit's group scores, [NQ][gcap]
+    float2* gsc = a.gsc + u * NQ * gcap;  // this unit's (group score, meta), [NQ][gcap]
     bool alive = true;
     for (int i = 0; i < ntile; ++i) {
       const int st = i % kStages, buf = i & 1;
@@ -338,8 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ln count of row r; -inf: the row is in no query row's softmax
       float lc;
+      int meta = 0;
       if (is_group) {
-        const int c = cnt_s[st * TROWS + r];
+        meta = cnt_s[st * TROWS + r];
+        const int c = meta & 0xffff;
         lc = (c > 0 && c <= kChunk) ? __logf((float)c) : -INFINITY;
         if (c > kChunk) set_status(a.status, LOD_ST_BAD_COUNT);
       } else {
@@ -412,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // group scores (-inf: not in this query row's softmax)
       if (is_group && r0 + r < G_vis) {
 #pragma unroll
-        for (int j = 0; j < NQ; ++j) gsc[j * gcap + r0 + r] = lg[j] == -INFINITY ? -INFINITY : sc[j];
+        for (int j = 0; j < NQ; ++j)
+          gsc[j * gcap + r0 + r] = make_float2(lg[j] == -INFINITY ? -INFINITY : sc[j], __int_as_float(meta));
       }
     }
     // ---------------------------------------------------------------- epilogue

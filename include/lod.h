@@ -111,8 +111,10 @@ typedef struct lod_params {
  *                         consecutive rows [pBeg, pBeg + pCnt) and an opened
  *                         page is read as one contiguous run (rows past the
  *                         last member are not written)
+ *   gMeta   [Cmax*k]      int32 gCnt and gPage of a group in one word:
+ *                         size | first page slot << 16 | end page slot << 24
  * Every array is laid out [B][Hkv][...] in that order.  gK, gV, pK, pV, perm,
- * mK and mV must be 16-byte aligned, gCnt and pCnt 4-byte aligned.
+ * mK and mV must be 16-byte aligned, gCnt, pCnt and gMeta 4-byte aligned.
  */
 typedef struct lod_index {
   void* gK;
@@ -126,6 +128,7 @@ typedef struct lod_index {
   int16_t* perm;
   void* mK;
   void* mV;
+  int32_t* gMeta;
 } lod_index;
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -135,11 +138,11 @@ int32_t lod_version(void);
 const char* lod_last_error(void);
 
 /*
- * Byte sizes of the eleven lod_index arrays, in field order (gK, gV, gCnt,
- * pK, pV, pCnt, pBeg, gPage, perm, mK, mV), written to bytes[0..10] (host).
- * Validates `p` like every other entry point.
+ * Byte sizes of the twelve lod_index arrays, in field order (gK, gV, gCnt,
+ * pK, pV, pCnt, pBeg, gPage, perm, mK, mV, gMeta), written to bytes[0..11]
+ * (host).  Validates `p` like every other entry point.
  */
-#define LOD_INDEX_ARRAYS 11
+#define LOD_INDEX_ARRAYS 12
 int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]);
 
 /*

@@ -53,7 +53,15 @@ def unit_from_gpu(ix: api.Index, b: int, h: int, nchunks: int, p: api.Params) ->
     return dict(gK=f(ix.gK, nchunks * k), gV=f(ix.gV, nchunks * k), gCnt=i(ix.gCnt, nchunks * k),
                 pK=f(ix.pK, nchunks * P), pV=f(ix.pV, nchunks * P), pCnt=i(ix.pCnt, nchunks * P),
                 pBeg=i(ix.pBeg, nchunks * P), gPage=i(ix.gPage, nchunks * (k + 1)),
-                perm=i(ix.perm, nchunks * C), nchunks=nchunks)
+                perm=i(ix.perm, nchunks * C), gMeta=i(ix.gMeta, nchunks * k), nchunks=nchunks)
+
+
+def pack_meta(u: dict, k: int) -> np.ndarray:
+    """gMeta of an index in the oracle's layout: size | first page << 16 | end page << 24."""
+    n = u["nchunks"]
+    gp = np.asarray(u["gPage"][:n * (k + 1)], dtype=np.int64).reshape(n, k + 1)
+    cnt = np.asarray(u["gCnt"][:n * k], dtype=np.int64).reshape(n, k)
+    return (cnt | (gp[:, :k] << 16) | (gp[:, 1:] << 24)).reshape(-1).astype(np.int32)
 
 
 def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params, K=None, V=None) -> None:
@@ -73,6 +81,7 @@ def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params, K=None, V
     put(ix.pBeg, u["pBeg"], n * P)
     put(ix.gPage, u["gPage"], n * (k + 1))
     put(ix.perm, u["perm"], n * C)
+    put(ix.gMeta, pack_meta(u, k), n * k)
     if K is not None:
         perm = torch.from_numpy(np.asarray(u["perm"][:n * C], dtype=np.int64))
         rows = torch.arange(n * C) // C * C + perm
@@ -113,6 +122,8 @@ def check_index_consistency(u: dict, K: np.ndarray, V: np.ndarray, cfg: oracle.C
     chunk minus the sinks, pages cut each group into runs of 16 in ascending
     order, and every summary is its members' mean (to one storage ulp)."""
     k, P, C = cfg.clusters, cfg.page_slots, cfg.chunk
+    if "gMeta" in u:
+        np.testing.assert_array_equal(u["gMeta"], pack_meta(u, k))
     for c in range(u["nchunks"]):
         first = cfg.sinks if c == 0 else 0
         perm = u["perm"][c * C:(c + 1) * C]

@@ -53,7 +53,7 @@ def test_index_sizes_match_the_documented_layout():
     u = 2 * 2
     assert s == [u * Cmax * k * 128 * 2] * 2 + [u * Cmax * k * 4] + [u * Cmax * Pp * 128 * 2] * 2 + \
         [u * Cmax * Pp * 4, u * Cmax * Pp * 2, u * Cmax * (k + 1) * 2, u * Cmax * 256 * 2] + \
-        [u * Cmax * 256 * 128 * 2] * 2
+        [u * Cmax * 256 * 128 * 2] * 2 + [u * Cmax * k * 4]
 
 
 @pytest.mark.parametrize("kw, code", [
@@ -138,4 +138,4 @@ def test_struct_layout_matches_the_header():
     assert _lib.lod_params.scale.offset == 64
     assert _lib.lod_params.Tmax.offset == 72
     assert ctypes.sizeof(_lib.lod_params) == 80
-    assert ctypes.sizeof(_lib.lod_index) == 8 * 11
+    assert ctypes.sizeof(_lib.lod_index) == 8 * 12

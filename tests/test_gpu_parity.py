@@ -241,3 +241,11 @@ def test_bad_index_values_are_skipped_and_reported():
     # a sequence length beyond the cache
     api.lod_decode(p, q, Kd, Vd, torch.tensor([T + 1], device="cuda"), ix, ws=ws)
     assert api.lod_get_status(ws) & api._lib.LOD_ST_BAD_SEQLEN
+    # page ranges past the chunk's slots in the packed group words
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    api.lod_decode(p, q, Kd, Vd, sl, ix, ws=ws)
+    assert api.lod_get_status(ws) == 0
+    ix.gMeta[0, 0] = (ix.gMeta[0, 0] & 0xffff) | (200 << 24)
+    out = api.lod_decode(p, q, Kd, Vd, sl, ix, ws=ws)
+    assert api.lod_get_status(ws) & api._lib.LOD_ST_BAD_PAGE
+    assert torch.isfinite(out.float()).all()
