@@ -274,25 +274,50 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
         status |= api.lod_get_status(r[5], stream)
     ms = ms_region if ms_region is not None else float(np.mean(ts))
     ms_max = dist_max(ms, world)
-    # end to end through the public API: pinned host q (and this token's K/V row) in, out back
-    qh = q.cpu().pin_memory()
-    newkv = torch.empty(2, w.B, w.Hkv, w.d, dtype=w.torch_dtype).pin_memory()
-    newkv[0] = K[:, :, w.T - 1]
-    newkv[1] = V[:, :, w.T - 1]
-    outh = torch.empty_like(qh).pin_memory()
-    qd = torch.empty_like(q)
+    # end to end through the public API: one pinned host buffer in (q and this
+    # token's K and V rows), out back; each step is one CUDA graph (the copy in,
+    # the cache-row writes, the decode kernels, the copy out)
+    qn, rown = q.numel(), w.B * w.Hkv * w.d
+    hin = torch.empty(qn + 2 * rown, dtype=w.torch_dtype).pin_memory()
+    hin[:qn] = q.cpu().reshape(-1)
+    hin[qn:qn + rown] = K[:, :, w.T - 1].reshape(-1)
+    hin[qn + rown:] = V[:, :, w.T - 1].reshape(-1)
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    stage = [torch.empty(qn + 2 * rown, dtype=w.torch_dtype, device=dev) for _ in range(R)]
 
-    def e2e_step(i):
-        qr, Kr, Vr, slr, ixr, wsr, outr = reps[i % R]
-        qr.copy_(qh, non_blocking=True)
-        Kr[:, :, w.T - 1].copy_(newkv[0], non_blocking=True)
-        Vr[:, :, w.T - 1].copy_(newkv[1], non_blocking=True)
-        api.lod_decode(p, qr, Kr, Vr, slr, ixr, out=outr, ws=wsr, stream=stream)
-        outh.copy_(outr, non_blocking=True)
+    def e2e_body(r, strm):
+        qr, Kr, Vr, slr, ixr, wsr, outr = reps[r]
+        st = stage[r]
+        st.copy_(hin, non_blocking=True)
+        Kr[:, :, w.T - 1].copy_(st[qn:qn + rown].view(w.B, w.Hkv, w.d))
+        Vr[:, :, w.T - 1].copy_(st[qn + rown:].view(w.B, w.Hkv, w.d))
+        api.lod_decode(p, st[:qn].view(q.shape), Kr, Vr, slr, ixr, out=outr, ws=wsr, stream=strm)
+        hout.copy_(outr, non_blocking=True)
 
-    e2e_steps = max(10, min(args.steps, 200))
-    te = time_steps(e2e_step, e2e_steps, 3, flush, stream)
-    e2e_ms = dist_max(float(np.mean(te)), world)
+    graphs = None
+    if args.graphs:
+        try:
+            graphs = []
+            for r in range(R):
+                e2e_body(r, stream)  # warm (attributes set, lazy state built) before capture
+            torch.cuda.synchronize()
+            for r in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    e2e_body(r, None)
+                graphs.append(g)
+            torch.cuda.synchronize()
+        except Exception as ex:  # capture not possible here: eager steps instead
+            print("e2e graph capture failed (%s); eager steps" % ex, file=sys.stderr)
+            graphs = None
+    e2e_step = (lambda i: graphs[i % R].replay()) if graphs else (lambda i: e2e_body(i % R, stream))
+    e2e_steps = max(10, min(args.steps, 1000))
+    if flush is None:
+        e2e_ms = dist_max(time_region(e2e_step, e2e_steps, 5, stream) / e2e_steps, world)
+    else:
+        e2e_ms = dist_max(float(np.mean(time_steps(e2e_step, e2e_steps, 3, flush, stream))), world)
+    torch.cuda.synchronize()
+    assert torch.equal(hout.to(dev), reps[(e2e_steps - 1) % R][6]), "e2e output copy mismatch"
     achieved = touched / (ms * 1e-3) / 1e9
     res = dict(
         metric="LoD decode queries/s (batch 4 x 64 heads at 128K context, one layer)",
@@ -305,8 +330,11 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
                       traffic=profiled_traffic("lod_decode", w.name), algorithmic_bytes_per_launch=touched,
                       peak_source=peaks["source"], nominal_peak_gbs=8000.0),
         e2e=dict(value=world * w.B / (e2e_ms * 1e-3), unit="queries/s",
-                 h2d_bytes_per_step=qh.numel() * qh.element_size() + newkv.numel() * newkv.element_size(),
-                 d2h_bytes_per_step=outh.numel() * outh.element_size(), ms_per_step=e2e_ms),
+                 h2d_bytes_per_step=hin.numel() * hin.element_size(),
+                 d2h_bytes_per_step=hout.numel() * hout.element_size(), ms_per_step=e2e_ms,
+                 step="one CUDA graph per step: pinned input copy, cache-row writes, lod_decode, "
+                      "output copy" if graphs else "eager: pinned input copy, cache-row writes, "
+                      "lod_decode, output copy"),
         gpu_launches=2 * args.steps,
         clocks=cs.summary(),
         l2=("inputs larger than L2: %d device replicas of cache, index, queries and workspace "
@@ -437,6 +465,7 @@ def main():
     ap.add_argument("--workload", default="decode_gqa_128k_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the prefill/build/oracle legs")
+    ap.add_argument("--graphs", type=int, default=1, help="e2e: one CUDA graph per step (0 = eager)")
     ap.add_argument("--replicas", type=int, default=4,
                     help="decode: device replicas of the inputs used in rotation (1 = flush L2 instead)")
     args = ap.parse_args()

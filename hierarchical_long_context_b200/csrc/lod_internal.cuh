@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 
+#include <atomic>
 #include <utility>
 
 #include "lod_common.cuh"
@@ -36,6 +37,21 @@ struct BuildArgs {
   int32_t* gMeta;      // size | first page << 16 | end page << 24 per group
   uint32_t* status;    // device status word (workspace header)
 };
+
+// Opt `kern` in to `smem` bytes of dynamic shared memory, once per device
+// (later calls make no CUDA call, so launches stay capturable in a graph).
+template <typename... KArgs>
+cudaError_t set_smem_once(void (*kern)(KArgs...), size_t smem) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launch `kern` as a programmatic dependent of the preceding work in `stream`
 // (it may start before that work completes and must call pdl_wait before
