@@ -1100,7 +1100,7 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
     } else if constexpr (NQ <= 8) {
       auto sk = scan_kernel<T, D, NQ>;
       const size_t smem = ScanSmem<T, D, NQ>::bytes;
-      e = set_smem_once(sk, smem);
+      e = set_smem_once<scan_kernel<T, D, NQ>>(smem);
       if (e != cudaSuccess) return e;
       e = launch_pdl(sk, dim3((unsigned)a.units, (unsigned)nsplit), dim3(kThreads), smem, stream, a);
     } else {
@@ -1111,7 +1111,7 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
   if (rows > 0) {
     auto rk = refine_kernel<T, D, NQ>;
     const size_t smem = RefineSmem<T, D>::bytes;
-    e = set_smem_once(rk, smem);
+    e = set_smem_once<refine_kernel<T, D, NQ>>(smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows);

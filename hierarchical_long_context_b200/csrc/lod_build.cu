@@ -420,7 +420,7 @@ template <typename T, int D, int KMAX>
 cudaError_t launch_kmeans_t(const BuildArgs& a, int64_t nchunks, int B, cudaStream_t stream) {
   const size_t smem = BuildSmem<T, D, KMAX>::bytes;
   auto kern = kmeans_kernel<T, D, KMAX>;
-  cudaError_t e = set_smem_once(kern, smem);
+  cudaError_t e = set_smem_once<kmeans_kernel<T, D, KMAX>>(smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nchunks, (unsigned)a.Hkv, (unsigned)B);
   kern<<<grid, kBuildThreads, smem, stream>>>(a);

@@ -38,17 +38,18 @@ struct BuildArgs {
   uint32_t* status;    // device status word (workspace header)
 };
 
-// Opt `kern` in to `smem` bytes of dynamic shared memory, once per device
-// (later calls make no CUDA call, so launches stay capturable in a graph).
-template <typename... KArgs>
-cudaError_t set_smem_once(void (*kern)(KArgs...), size_t smem) {
+// Opt kernel `Kern` in to `smem` bytes of dynamic shared memory, once per
+// device (later calls make no CUDA call, so launches stay capturable in a
+// graph).  The flag is per kernel: Kern is a template argument.
+template <auto Kern>
+cudaError_t set_smem_once(size_t smem) {
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
   if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
   return e;
 }

@@ -458,7 +458,7 @@ template <int NQ>
 cudaError_t launch_nq(const AttendArgs& a, const TcMaps& maps, cudaStream_t stream) {
   auto kern = scan_tc_kernel<NQ>;
   const size_t smem = TcSmem::bytes;
-  cudaError_t e = set_smem_once(kern, smem);
+  cudaError_t e = set_smem_once<scan_tc_kernel<NQ>>(smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)a.units, (unsigned)a.nsplit), dim3(kThreads), smem, stream, maps, a);
 }

@@ -125,6 +125,27 @@ def test_decode_on_gpu_index_matches_oracle(name, T, seq_lens):
     print(name, st)
 
 
+@pytest.mark.parametrize("kw", [
+    dict(d=64, Hq=2, Hkv=2),                                                  # bf16 d=64 (CUDA-core scan), MHA
+    dict(Hq=4, Hkv=2, clusters=(16,), top_groups=16, top_pages=4),            # g=2, k=16, widest selection
+    dict(dtype="f32", Hq=8, Hkv=2, clusters=(1,), top_groups=1, top_pages=1),  # fp32 d=128, k=1, one page
+    dict(Hq=16, Hkv=2, window=256, sinks=0),                                   # g=8, short window, no sinks
+])
+def test_decode_parameter_sweep(kw):
+    """Head ratios, head sizes, dtypes, cluster counts and selection widths at
+    the edges of what lod_params accepts, each against the oracle."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, T=4096, **kw)
+    T = 4096
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 777], draws=2)
+    cfg = lt.oracle_cfg(w)
+    st = _check_decode(w, p, Kc, Vc, ix, rows, cfg,
+                       lambda b, h, K, V, n: lt.unit_from_gpu(ix, b, h, T // 256, p))
+    print(kw, st)
+
+
 def test_decode_on_oracle_index_matches_oracle():
     """The attention kernels alone: the index is the oracle's, imported."""
     w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, Hkv=2, Hq=16)
@@ -164,6 +185,7 @@ def test_zero_variance_decode_equals_dense():
     ("prefill_128k_bf16", 2048 + 100, None),      # ragged tail, one call
     ("prefill_128k_bf16", 2048 + 100, 1024),      # two calls: the second continues the first
     ("decode_tiny_f32", 1536 + 37, None),
+    ("decode_gqa_32k_bf16", 1024 + 300, None),    # g = 8: one position per scan unit
 ])
 def test_prefill_matches_oracle(name, T, split):
     w = synth.WORKLOADS[name]
