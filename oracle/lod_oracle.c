@@ -47,6 +47,9 @@
  *             the lower global group id (chunk * k + slot); pages by
  *             scale * q.k_page_mean, ties to the lower page slot; a group with
  *             no more pages than `top_pages` is opened entirely.
+ *   R-twotier top_pages = 0 is the pages' two-tier LoD ("Level of Detail
+ *             Attention", the quality tables' "Two-tier LoD" rows): an opened
+ *             group is opened whole, with no page tier and no page remainder.
  *   R-coarse  every unopened page of an opened group is its own coarse entry
  *             (mean key logit + ln(count), mean value); ln(count) is added
  *             after the 1/sqrt(d) scale, since n copies of exp(x) are
@@ -72,7 +75,8 @@ typedef struct {
   int32_t clusters;   /* k: groups per chunk */
   int32_t iters;      /* Lloyd rounds */
   int32_t top_groups; /* groups opened per query (8 on the page) */
-  int32_t top_pages;  /* pages opened per opened group (2 on the page) */
+  int32_t top_pages;  /* pages opened per opened group (2 on the page); 0:
+                         every page (two-tier LoD, opened groups go whole) */
   int32_t window;     /* sliding window in tokens, a multiple of chunk */
   int32_t sinks;      /* number of sink tokens at the start */
   int32_t store_bf16; /* 1: summaries rounded to bfloat16, 0: to float32 */
@@ -399,7 +403,7 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
   const int G = p->top_groups, TP = p->top_pages;
   const double sc = scale_of(p);
   const float sc32 = (float)sc;
-  if (t < 0 || p->window <= 0 || p->window % C || G < 1 || G > 64 || TP < 1 || TP > 64)
+  if (t < 0 || p->window <= 0 || p->window % C || G < 1 || G > 64 || TP < 0 || TP > 64)
     return ORC_EINVAL;
 
   /* R-window */
@@ -491,7 +495,9 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
     }
     int nopen_p = 0;
     int32_t op[64];
-    if (forced_pages) {
+    if (TP == 0) {  /* two-tier LoD: an opened group is opened whole */
+      for (int r = 0; r < np; ++r) op[nopen_p++] = pr[r].pos;
+    } else if (forced_pages) {
       for (int r = 0; r < TP; ++r) {
         int32_t f = forced_pages[i * TP + r];
         if (f >= 0) op[nopen_p++] = (int32_t)(f - c * P);
@@ -501,7 +507,7 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
       nopen_p = np < TP ? np : TP;
       for (int r = 0; r < nopen_p; ++r) op[r] = pr[r].pos;
     }
-    for (int r = 0; r < nopen_p; ++r) sel_pages[i * TP + r] = (int32_t)(c * P + op[r]);
+    for (int r = 0; r < nopen_p && r < TP; ++r) sel_pages[i * TP + r] = (int32_t)(c * P + op[r]);
     for (int r = 0; r < np; ++r) {
       int sl = pr[r].pos, is_open = 0;
       for (int u = 0; u < nopen_p; ++u) is_open |= (op[u] == sl);

@@ -202,6 +202,47 @@ def test_everything_opened_gives_dense_attention(tiny):
             np.testing.assert_allclose(out, dout, rtol=0, atol=1e-12)
 
 
+def test_two_tier_is_whole_group_attention_written_out(tiny):
+    """Two-tier LoD (top_pages = 0): the opened groups' members are exact and
+    no page tier exists.  Checked against the entry list written out here in
+    numpy from the index arrays (window, sinks, whole opened groups exact,
+    every other visible group as mean-key logit + ln n with its mean value)."""
+    w, _, K, V, _ = tiny
+    T = 2048
+    cfg = _cfg(w, top_groups=3, top_pages=0)
+    idx = oracle.build_sequence(cfg, 0, K[:T], V[:T], T // 256)
+    k, C, sc = cfg.clusters, cfg.chunk, 1.0 / np.sqrt(cfg.d)
+    Kd, Vd = K.astype(np.float64), V.astype(np.float64)
+    for q in _rows(w, 6):
+        for t in (T - 1, 1700, 1100):
+            out, lse, sg, sp, st = oracle.attend_row(cfg, q, t, K, V, idx)
+            assert sp.size == 0 and st["n_coarse_pages"] == 0
+            ws = 256 * max(0, t // 256 - cfg.window // 256 + 1)
+            qd = q.astype(np.float64)
+            ids = [g for g in range((ws // C) * k) if idx["gCnt"][g] > 0]
+            s32 = {g: float(np.float32(np.dot(q.astype(np.float32), idx["gK"][g].astype(np.float32)))
+                            * np.float32(sc)) for g in ids}
+            opened = sorted(ids, key=lambda g: (-s32[g], g))[:cfg.top_groups]
+            assert list(sg[:len(opened)]) == opened
+            lg, vals = [], []
+            for pos in list(range(min(cfg.sinks, ws))) + list(range(ws, t + 1)):
+                lg.append(sc * qd @ Kd[pos]); vals.append(Vd[pos])
+            for g in ids:
+                c, j = divmod(g, k)
+                if g in opened:
+                    off = int(np.sum(idx["gCnt"][c * k:c * k + j]))
+                    for m in range(int(idx["gCnt"][g])):
+                        pos = c * C + idx["perm"][c * C + off + m]
+                        lg.append(sc * qd @ Kd[pos]); vals.append(Vd[pos])
+                else:
+                    lg.append(sc * qd @ idx["gK"][g] + np.log(idx["gCnt"][g])); vals.append(idx["gV"][g])
+            lg = np.array(lg)
+            wgt = np.exp(lg - lg.max())
+            want = (wgt[:, None] * np.array(vals)).sum(0) / wgt.sum()
+            np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+            assert abs(lse - (lg.max() + np.log(wgt.sum()))) < 1e-12
+
+
 def test_window_covering_everything_is_dense(tiny):
     w, cfg, K, V, idx = tiny
     for q in _rows(w, 4):
