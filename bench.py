@@ -361,6 +361,51 @@ def synth_q(w):
     return synth.decode_queries(w)
 
 
+def run_decode_variant(w, dev, stream, peaks, steps, replicas, label):
+    """A decode leg on workload `w` (device time of `steps` back-to-back steps
+    over rotating input replicas, as the headline leg) with the roofline over
+    the bytes its own selections touch."""
+    from hierarchical_long_context_b200 import api, metrics
+    p = params_for(w)
+    K, V = synth_kv(w)
+    Kd, Vd = K.to(dev), V.to(dev)
+    ix = api.Index(p, dev)
+    api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix, stream=stream)
+    q = synth_q(w).to(dev)
+    sl = torch.full((w.B,), w.T, dtype=torch.int64, device=dev)
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE, dev)
+    sg = torch.empty(w.B, w.Hq, p.top_groups, dtype=torch.int32, device=dev)
+    spg = torch.empty(w.B, w.Hq, p.top_groups, max(p.top_pages, 1), dtype=torch.int32, device=dev)
+    out = api.lod_decode(p, q, Kd, Vd, sl, ix, sel_groups=sg, sel_pages=spg if p.top_pages else None, ws=ws,
+                         stream=stream)
+    torch.cuda.synchronize()
+    touched = metrics.decode_touched_bytes(p, ix, sl, sg, spg)
+    reps = [(q, Kd, Vd, ix, ws, out)]
+    for _ in range(max(1, replicas) - 1):
+        ixr = api.Index(p, dev)
+        for f in api._lib.INDEX_FIELDS:
+            getattr(ixr, f).copy_(getattr(ix, f))
+        reps.append((q.clone(), Kd.clone(), Vd.clone(), ixr, torch.zeros_like(ws), torch.empty_like(out)))
+    R = len(reps)
+
+    def step(i):
+        qr, Kr, Vr, ixr, wsr, outr = reps[i % R]
+        api.lod_decode(p, qr, Kr, Vr, sl, ixr, out=outr, ws=wsr, stream=stream)
+
+    ms = time_region(step, steps, 10, stream) / steps
+    status = 0
+    for r in reps:
+        status |= api.lod_get_status(r[4], stream)
+    gbs = touched / (ms * 1e-3) / 1e9
+    del reps
+    return dict(workload=label, value=w.B / (ms * 1e-3), unit="queries/s", ms_per_step=ms,
+                seq_len=w.T, B=w.B, top_groups=p.top_groups, top_pages=p.top_pages,
+                l2="%d rotating input replicas" % R,
+                roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                              frac=gbs / peaks["hbm_gbs"], algorithmic_bytes_per_launch=touched),
+                status_word=status)
+
+
 def run_prefill(w, dev, stream, steps, peaks):
     from hierarchical_long_context_b200 import api, metrics, synth
     p = params_for(w)
@@ -488,6 +533,10 @@ def main():
     res.pop("_touch")
     extras = {}
     if not args.no_extras:
+        extras["decode_two_tier"] = run_decode_variant(
+            w.with_(top_pages=0), dev, stream, peaks, 1000, 4,
+            "%s, two-tier LoD (top_pages = 0: opened groups read whole)" % w.name)
+        torch.cuda.empty_cache()
         wp = synth.WORKLOADS["prefill_128k_bf16"]
         extras["prefill"] = run_prefill(wp, dev, stream, 2, peaks)
         wb = synth.WORKLOADS["build_128k_bf16"]

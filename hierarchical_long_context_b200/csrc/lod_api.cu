@@ -57,8 +57,8 @@ int32_t validate(const lod_params* p) {
     return fail(LOD_EUNSUPPORTED, "kmeans_iters must be in [1, 64]");
   if (p->top_groups < 1 || p->top_groups > lod::kMaxTopGroups)
     return fail(LOD_EUNSUPPORTED, "top_groups must be in [1, %d]", lod::kMaxTopGroups);
-  if (p->top_pages < 1 || p->top_pages > lod::kMaxTopPages)
-    return fail(LOD_EUNSUPPORTED, "top_pages must be in [1, %d]", lod::kMaxTopPages);
+  if (p->top_pages < 0 || p->top_pages > lod::kMaxTopPages)
+    return fail(LOD_EUNSUPPORTED, "top_pages must be in [0, %d] (0: two-tier LoD)", lod::kMaxTopPages);
   if (p->window < p->chunk || p->window % p->chunk)
     return fail(LOD_EINVAL, "window (%d) must be a positive multiple of chunk", p->window);
   if (p->sinks < 0 || p->sinks >= p->chunk) return fail(LOD_EINVAL, "sinks must be in [0, chunk)");

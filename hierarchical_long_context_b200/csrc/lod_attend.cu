@@ -959,7 +959,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const bool prange_ok = !(p1 < p0 || p1 > a.P || p1 - p0 > 32);
     const int np = prange_ok ? p1 - p0 : 0;
     const T* pKc = pK + (c * a.P + (prange_ok ? p0 : 0)) * D;
-    rows_dot_coalesced<T, D, 8>(np, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
+    // (two-tier LoD opens the group whole: no page scores)
+    rows_dot_coalesced<T, D, 8>(a.TP > 0 ? np : 0, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
     mycnt[lane] = pcl;
     mybeg[lane] = pbl;
     int open_slot[kMaxTopPages];
@@ -1004,12 +1005,19 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 #pragma unroll
       for (int x = 0; x < kMaxTopPages; ++x) is_open |= (open_slot[x] == p0 + lane);
       // coarse entries: the unopened pages of this group (lane p), staged with the first batch
-      const bool cv = lane < np && !is_open && cntp > 0 && cntp <= kPage;
-      if (lane < np && !is_open && (cntp <= 0 || cntp > kPage)) set_status(a.status, LOD_ST_BAD_COUNT);
+      // (two-tier LoD has no page tier: no coarse pages)
+      const bool cv = a.TP > 0 && lane < np && !is_open && cntp > 0 && cntp <= kPage;
+      if (a.TP > 0 && lane < np && !is_open && (cntp <= 0 || cntp > kPage)) set_status(a.status, LOD_ST_BAD_COUNT);
       const unsigned cm = __ballot_sync(0xffffffffu, cv);
       const float lgc = cv ? sc + __logf((float)cntp) : -INFINITY;
-      // exact members of the opened pages, 32 per batch: lane e -> (page e/16, member e%16)
-      const int nbatch = (nopen * kPage + 31) / 32;
+      // exact members, 32 per batch.  Paged: lane e -> (opened page e/16,
+      // member e%16).  Two-tier LoD (top_pages = 0): the whole group, one
+      // contiguous run of the member-ordered copies from its first page.
+      const int b0 = __shfl_sync(0xffffffffu, begp, 0);
+      const bool whole = a.TP == 0;
+      const bool okrun = gcnt > 0 && gcnt <= kChunk && b0 >= 0 && b0 + gcnt <= kChunk;
+      if (whole && !okrun && lane == 0) set_status(a.status, LOD_ST_BAD_MEMBER);
+      const int nbatch = whole ? (okrun ? (gcnt + 31) / 32 : 0) : (nopen * kPage + 31) / 32;
       for (int bt = 0; bt < (nbatch > 0 ? nbatch : 1); ++bt) {
         const int e = bt * 32 + lane;
         const int x = e / kPage, mi = e % kPage;
@@ -1018,19 +1026,27 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         for (int y = 0; y < kMaxTopPages; ++y)
           if (y == x) slot = open_slot[y];
         const int sl_lane = slot >= 0 ? slot - p0 : 0;
-        const int n_of = __shfl_sync(0xffffffffu, cntp, sl_lane & 31);
-        const int b_of = __shfl_sync(0xffffffffu, begp, sl_lane & 31);
+        int n_of = __shfl_sync(0xffffffffu, cntp, sl_lane & 31);
+        int b_of = __shfl_sync(0xffffffffu, begp, sl_lane & 31);
         bool ev = x < nopen && slot >= 0 && mi < n_of;
-        if (ev && n_of > kPage) {
+        if (whole) {
+          ev = okrun && e < gcnt;
+          n_of = 1;
+          b_of = b0 + e;
+        }
+        if (ev && !whole && n_of > kPage) {
           set_status(a.status, LOD_ST_BAD_PAGE);
           ev = false;
         }
-        if (ev && (b_of < 0 || b_of + n_of > kChunk)) {
+        if (ev && !whole && (b_of < 0 || b_of + n_of > kChunk)) {
           set_status(a.status, LOD_ST_BAD_MEMBER);
           ev = false;
         }
+        if (whole) {
+          n_of = 0;
+        }
         // the page's members are consecutive rows of the member-ordered copies
-        const int64_t row = c * kChunk + (ev ? b_of + mi : 0);
+        const int64_t row = c * kChunk + (ev ? b_of + (whole ? 0 : mi) : 0);
         batch(ev, mK + row * D, mV + row * D, bt == 0 && cv, lgc, pV + (c * a.P + p0 + lane) * D);
       }
     }

@@ -45,6 +45,10 @@ def decode_touched_bytes(p, index, seq_lens, sel_groups, sel_pages) -> int:
             total += ((t - ws + 1) + ns) * 2 * row
             heads = range(h * p.g, (h + 1) * p.g)
             groups = set(int(x) for hq in heads for x in sg[b, hq] if x >= 0)
+            if p.top_pages == 0:  # two-tier: every opened group read whole, no page tier
+                for gid in groups:
+                    total += 2 * 2 + 2 + int(gCnt[b, h, gid]) * 2 * row  # page range, first offset, K and V
+                continue
             opened = set(int(x) for hq in heads for x in sp[b, hq].ravel() if x >= 0)
             for gid in groups:
                 c, j = divmod(gid, k)

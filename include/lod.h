@@ -67,7 +67,8 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
  * Parameters.  Supported: dtype F32 or BF16 (cache, summaries, q and out all
  * in this dtype); d in {64, 128}; chunk = 256 and page = 16 (the page's
  * values); 1 <= clusters <= 16; 1 <= kmeans_iters <= 64; 1 <= top_groups
- * <= 16; 1 <= top_pages <= 4; window a positive multiple of chunk (the
+ * <= 16; 0 <= top_pages <= 4 (0: two-tier LoD, an opened group is opened
+ * whole with no page tier); window a positive multiple of chunk (the
  * page says 256-512); 0 <= sinks < chunk; Hq a multiple of Hkv with
  * Hq/Hkv a power of two no larger than 8; Tmax a positive multiple of chunk.
  * scale <= 0 selects 1/sqrt(d).
@@ -83,7 +84,7 @@ typedef struct lod_params {
   int32_t clusters;     /* k-means groups per chunk */
   int32_t kmeans_iters; /* Lloyd rounds */
   int32_t top_groups;   /* groups opened per query: 8 */
-  int32_t top_pages;    /* pages opened per opened group: 2 */
+  int32_t top_pages;    /* pages opened per opened group: 2; 0 = every page (two-tier LoD) */
   int32_t window;       /* sliding window in tokens (block granular) */
   int32_t sinks;        /* sink tokens at positions [0, sinks) */
   int32_t reserved0;    /* must be 0 */
