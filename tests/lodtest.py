@@ -181,7 +181,10 @@ def compare_builds(gu: dict, ou: dict, cfg: oracle.Config, bf16: bool) -> dict:
             np.testing.assert_array_equal(gu["pCnt"][c * P:(c + 1) * P], ou["pCnt"][c * P:(c + 1) * P])
             for key, n in (("gK", k), ("gV", k), ("pK", P), ("pV", P)):
                 g_, o_ = gu[key][c * n:(c + 1) * n], ou[key][c * n:(c + 1) * n]
-                tol = (2.0 ** -8 * np.abs(o_) + 1e-6) if bf16 else (2e-6 * np.abs(o_) + 1e-6)
+                # both sides round an fp32 sum (taken in different orders) to
+                # bf16: the results may straddle a rounding boundary and differ
+                # by one bf16 ulp, at most 2^-7 of the value
+                tol = (2.0 ** -7 * np.abs(o_) + 1e-6) if bf16 else (2e-6 * np.abs(o_) + 1e-6)
                 assert np.all(np.abs(g_ - o_) <= tol), (c, key)
     return stats
 
