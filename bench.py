@@ -361,14 +361,18 @@ def synth_q(w):
     return synth.decode_queries(w)
 
 
-def run_decode_variant(w, dev, stream, peaks, steps, replicas, label):
+def run_decode_variant(w, dev, stream, peaks, steps, replicas, label, device_gen=False):
     """A decode leg on workload `w` (device time of `steps` back-to-back steps
     over rotating input replicas, as the headline leg) with the roofline over
     the bytes its own selections touch."""
     from hierarchical_long_context_b200 import api, metrics
+    from hierarchical_long_context_b200 import synth
     p = params_for(w)
-    K, V = synth_kv(w)
-    Kd, Vd = K.to(dev), V.to(dev)
+    if device_gen:
+        Kd, Vd = synth.kv_cache_device(w, dev)
+    else:
+        K, V = synth_kv(w)
+        Kd, Vd = K.to(dev), V.to(dev)
     ix = api.Index(p, dev)
     api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix, stream=stream)
     q = synth_q(w).to(dev)
@@ -536,6 +540,10 @@ def main():
         extras["decode_two_tier"] = run_decode_variant(
             w.with_(top_pages=0), dev, stream, peaks, 1000, 4,
             "%s, two-tier LoD (top_pages = 0: opened groups read whole)" % w.name)
+        torch.cuda.empty_cache()
+        extras["decode_1m"] = run_decode_variant(
+            synth.WORKLOADS["decode_gqa_1m_bf16"], dev, stream, peaks, 500, 4,
+            "decode_gqa_1m_bf16: one sequence at 1M context (device-generated inputs)", device_gen=True)
         torch.cuda.empty_cache()
         wp = synth.WORKLOADS["prefill_128k_bf16"]
         extras["prefill"] = run_prefill(wp, dev, stream, 2, peaks)

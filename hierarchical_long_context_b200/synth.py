@@ -87,6 +87,10 @@ WORKLOADS = {
         "prefill_128k_bf16", B=1, Hq=32, Hkv=8, d=128, T=131072, dtype="bf16",
         n_centers=512, rope_theta=1e6, window=512, sinks=4, mode="prefill",
         note="chunked causal prefill at 128K"),
+    "decode_gqa_1m_bf16": Workload(
+        "decode_gqa_1m_bf16", B=1, Hq=64, Hkv=8, d=128, T=1048576, dtype="bf16",
+        n_centers=512, rope_theta=1e6, n_outliers=4, window=512, sinks=4,
+        note="long-context GQA decode at 1M (one sequence); device-generated (kv_cache_device)"),
     "build_128k_bf16": Workload(
         "build_128k_bf16", B=1, Hq=8, Hkv=8, d=128, T=131072, dtype="bf16",
         n_centers=2048, rope_theta=1e6, clusters=(4, 8), window=512, sinks=4, mode="build",
@@ -177,6 +181,41 @@ def kv_cache(w: Workload, T: int | None = None, threads: int = 8):
 
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(fill, range(w.B * w.Hkv)))
+    return K, V
+
+
+def kv_cache_device(w: Workload, device, T: int | None = None):
+    """The KV cache [B, Hkv, T, d] (cache dtype) generated on `device` with
+    the same recipe as unit_kv (unit-norm Gaussian centres, key = centre +
+    sigma N(0, I), seeded outlier channels before RoPE, N(0, 1) values) from
+    seeded torch generators instead of numpy: for contexts whose host
+    generation would take minutes.  Deterministic for (w, device type)."""
+    T = w.T if T is None else T
+    K = torch.empty((w.B, w.Hkv, T, w.d), dtype=w.torch_dtype, device=device)
+    V = torch.empty_like(K)
+    h2 = w.d // 2
+    inv = w.rope_theta ** (-2.0 * torch.arange(h2, dtype=torch.float64, device=device) / w.d)
+    step = 65536
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            tag = zlib.crc32(("%s/%d/%d" % (w.name, b, h)).encode())
+            g = torch.Generator(device=device).manual_seed((w.seed << 32) ^ tag)
+            cen = torch.randn((w.n_centers, w.d), generator=g, device=device)
+            cen /= cen.norm(dim=1, keepdim=True)
+            ch = torch.randperm(w.d, generator=g, device=device)[:w.n_outliers]
+            sg = torch.randint(0, 2, (w.n_outliers,), generator=g, device=device).float() * 2 - 1
+            for t0 in range(0, T, step):
+                n = min(step, T - t0)
+                z = torch.randint(0, w.n_centers, (n,), generator=g, device=device)
+                k = cen[z] + w.sigma * torch.randn((n, w.d), generator=g, device=device)
+                if w.n_outliers:
+                    k[:, ch] += w.outlier_mag * sg
+                if w.rope_theta:
+                    ang = torch.arange(t0, t0 + n, dtype=torch.float64, device=device)[:, None] * inv[None, :]
+                    c, s = torch.cos(ang).float(), torch.sin(ang).float()
+                    k = torch.cat([k[:, :h2] * c - k[:, h2:] * s, k[:, h2:] * c + k[:, :h2] * s], dim=1)
+                K[b, h, t0:t0 + n] = k.to(w.torch_dtype)
+                V[b, h, t0:t0 + n] = torch.randn((n, w.d), generator=g, device=device).to(w.torch_dtype)
     return K, V
 
 

@@ -11,6 +11,7 @@ times, on outputs the oracle can compute one by one.
     are checked against the oracle.
   * Index build at 128K with k = 4 and k = 8: whole build, sampled KV heads
     compared chunk by chunk.
+  * One sequence at a 1M-token context (inputs generated on the device).
 """
 import numpy as np
 import pytest
@@ -65,6 +66,38 @@ def test_decode_full_size(name, units):
         rows = [(_np(q[b, hq]), w.T - 1, _np(out[b, hq]).astype(np.float64), float(lse[b, hq]),
                  sg[b, hq].cpu().numpy(), sp[b, hq].cpu().numpy()) for hq in range(h * w.g, (h + 1) * w.g)]
         print(name, (b, h), st, lt.check_rows(cfg, w.dtype, Kn, Vn, gu, rows))
+
+
+def test_decode_1m_full_size():
+    """One sequence at a 1M-token context (32760 visible groups per KV head):
+    the GPU builds the whole index and decodes; one KV head is rebuilt by the
+    oracle (build under the margin rule) and its 8 query heads checked."""
+    dev = _dev()
+    w = synth.WORKLOADS["decode_gqa_1m_bf16"]
+    Kd, Vd = synth.kv_cache_device(w, dev)
+    p = lt.params_of(w)
+    ix = api.Index(p, dev)
+    nch = w.T // 256
+    api.lod_build_index(p, Kd, Vd, 0, nch, ix)
+    q = synth.decode_queries(w).to(dev)
+    sl = torch.full((w.B,), w.T, dtype=torch.int64, device=dev)
+    lse = torch.empty(w.B, w.Hq, dtype=torch.float32, device=dev)
+    sg = torch.empty(w.B, w.Hq, p.top_groups, dtype=torch.int32, device=dev)
+    sp = torch.empty(w.B, w.Hq, p.top_groups, p.top_pages, dtype=torch.int32, device=dev)
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE, dev)
+    out = api.lod_decode(p, q, Kd, Vd, sl, ix, lse=lse, sel_groups=sg, sel_pages=sp, ws=ws)
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws) == 0
+    cfg = lt.oracle_cfg(w)
+    h = 5
+    Kn, Vn = _np(Kd[0, h]), _np(Vd[0, h])
+    gu = lt.unit_from_gpu(ix, 0, h, nch, p)
+    ou = oracle.build_sequence(cfg, h, Kn, Vn, nch)
+    st = lt.compare_builds(gu, ou, cfg, True)
+    assert st["diverged"] <= max(2, nch // 20), st
+    rows = [(_np(q[0, hq]), w.T - 1, _np(out[0, hq]).astype(np.float64), float(lse[0, hq]),
+             sg[0, hq].cpu().numpy(), sp[0, hq].cpu().numpy()) for hq in range(h * w.g, (h + 1) * w.g)]
+    print("1M", st, lt.check_rows(cfg, w.dtype, Kn, Vn, gu, rows))
 
 
 def test_prefill_full_size():
