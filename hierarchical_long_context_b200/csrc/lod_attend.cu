@@ -56,6 +56,32 @@ __device__ __forceinline__ void unpack16(const uint4& raw, float* f) {
   }
 }
 
+// N consecutive elements from shared memory as floats (one vector load).
+template <typename T, int N>
+__device__ __forceinline__ void lds_f(const T* p, float (&v)[N]) {
+  if constexpr (sizeof(T) == 4) {
+    if constexpr (N == 4) {
+      const float4 a = *reinterpret_cast<const float4*>(p);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else {
+      static_assert(N == 2, "unsupported f32 vector width");
+      const float2 a = *reinterpret_cast<const float2*>(p);
+      v[0] = a.x; v[1] = a.y;
+    }
+  } else if constexpr (N == 4) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(a.x << 16);
+    v[1] = __uint_as_float(a.x & 0xffff0000u);
+    v[2] = __uint_as_float(a.y << 16);
+    v[3] = __uint_as_float(a.y & 0xffff0000u);
+  } else {
+    static_assert(N == 2, "unsupported bf16 vector width");
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(p);
+    v[0] = __uint_as_float(a << 16);
+    v[1] = __uint_as_float(a & 0xffff0000u);
+  }
+}
+
 // Dot product of a whole d-row (owned by one lane) with q held in shared memory.
 template <typename T, int D>
 __device__ __forceinline__ float row_dot(const T* __restrict__ row, const float* __restrict__ qs) {
@@ -662,6 +688,18 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   if (tid == 0) fence_mbar_init();
   pdl_wait();  // the scan's partial states and group scores are visible from here on
   pdl_launch_dependents();
+  // the sink tokens [0, min(sinks, window start)) are exact entries (last
+  // warp); their rows go to L2 now, while the groups are selected
+  const int64_t wsq = (t / kChunk - a.window / kChunk + 1) > 0 ? (t / kChunk - a.window / kChunk + 1) * kChunk : 0;
+  const int64_t nsk = a.sinks < wsq ? a.sinks : wsq;
+  const T* Kb = static_cast<const T*>(a.K) + b * a.sb + kvh * a.sh;
+  const T* Vb = static_cast<const T*>(a.V) + b * a.sb + kvh * a.sh;
+  if (warp == kWarps - 1)
+    for (int64_t e = lane; e < nsk; e += 32)
+      for (int o = 0; o < ROWB; o += 128) {
+        prefetch_l2(reinterpret_cast<const char*>(Kb + e * a.st) + o);
+        prefetch_l2(reinterpret_cast<const char*>(Vb + e * a.st) + o);
+      }
 
   const int nsplit = a.nsplit;
   // the split states this thread merges (component c = tid of each), loaded
@@ -690,6 +728,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const float2* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
     constexpr int kSel = 16;  // scores per thread kept in registers (up to 4096 groups)
     const bool in_regs = Gq <= kSel * kThreads;
+    const int ns = (Gq + kThreads - 1) / kThreads;  // register slots in use (uniform)
     float sv[kSel];
     float bs = -INFINITY;
     int bi = 0x7fffffff;
@@ -697,11 +736,12 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 #pragma unroll
       for (int e = 0; e < kSel; ++e) {
         const int i = tid + e * kThreads;
-        sv[e] = i < Gq ? srow[i].x : -INFINITY;
+        sv[e] = -INFINITY;
+        if (e < ns && i < Gq) sv[e] = srow[i].x;
       }
 #pragma unroll
       for (int e = 0; e < kSel; ++e)
-        if (sv[e] > bs) {  // first occurrence: the smaller id wins a tie
+        if (e < ns && sv[e] > bs) {  // first occurrence: the smaller id wins a tie
           bs = sv[e];
           bi = tid + e * kThreads;
         }
@@ -745,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       int wcount = 0;
 #pragma unroll
       for (int e = 0; e < kSel; ++e) {
-        msk[e] = __ballot_sync(0xffffffffu, okey32(sv[e]) >= lo);
+        msk[e] = e < ns ? __ballot_sync(0xffffffffu, okey32(sv[e]) >= lo) : 0u;
         wcount += __popc(msk[e]);
       }
       if (lane == 0) wtot[warp] = wcount;
@@ -759,6 +799,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       }
 #pragma unroll
       for (int e = 0; e < kSel; ++e) {
+        if (e >= ns) break;
         if ((msk[e] >> lane) & 1u) {
           const int pos = base + __popc(msk[e] & lt);
           if (pos < SM::kSurvCap) surv[pos] = group_key(sv[e], tid + e * kThreads);
@@ -863,16 +904,16 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   const int16_t* pB = a.pBeg + unit_kv * a.Cmax * a.P;
   const T* mK = static_cast<const T*>(a.mK) + unit_kv * a.Cmax * kChunk * D;
   const T* mV = static_cast<const T*>(a.mV) + unit_kv * a.Cmax * kChunk * D;
-  const T* Kb = static_cast<const T*>(a.K) + b * a.sb + kvh * a.sh;
-  const T* Vb = static_cast<const T*>(a.V) + b * a.sb + kvh * a.sh;
   T* myV = Vst + warp * SM::kRows * D;
   float* mysc = sc_s + warp * 64;
   const T** mykp = reinterpret_cast<const T**>(posm_s) + warp * 32;
   int* mycnt = reinterpret_cast<int*>(smem + SM::off_pc) + warp * 32;
   int* mybeg = mycnt + kWarps * 32;
   uint32_t phase = 0;
-  // member key rows scored per round: all 32 of a batch for bf16 rows
+  // member key rows scored per round of coalesced loads; rows past the first
+  // round are brought into L2 while that round is in flight
   constexpr int kMemberSteps = 8;
+  constexpr int kFirstRound = kMemberSteps * (32 / LPR);
   // One batch of up to 32 exact tokens (lane e: `ev`, key and value rows
   // `krow`, `vrow`) and up to 32 coarse entries (lane p: `cvb`, logit `lgc`,
   // value row `crow`): the value rows are staged in shared memory by TMA
@@ -882,14 +923,19 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const unsigned vm = __ballot_sync(0xffffffffu, ev);
     const unsigned cmb = __ballot_sync(0xffffffffu, cvb);
     if (!(vm | cmb)) return;
-    if (lane == 0) mbar_arrive_expect(&bar[warp], (uint32_t)(__popc(vm) + __popc(cmb)) * ROWB);
-    __syncwarp();
-    if (ev) bulk_g2s(myV + lane * D, vrow, ROWB, &bar[warp]);
-    if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
-    // members are packed: lanes 0..nvalid-1 hold the valid ones in order
+    // exact tokens are packed: the valid ones take ranks 0..nvalid-1 in lane
+    // order, for their key pointers, scores, weights and staged value rows
     const int nvalid = __popc(vm);
     const int my_rank = __popc(vm & ((1u << lane) - 1u));
-    if (ev) mykp[my_rank] = krow;
+    if (lane == 0) mbar_arrive_expect(&bar[warp], (uint32_t)(nvalid + __popc(cmb)) * ROWB);
+    __syncwarp();
+    if (ev) bulk_g2s(myV + my_rank * D, vrow, ROWB, &bar[warp]);
+    if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
+    if (ev) {
+      mykp[my_rank] = krow;
+      if (my_rank >= kFirstRound)
+        for (int o = 0; o < ROWB; o += 128) prefetch_l2(reinterpret_cast<const char*>(krow) + o);
+    }
     __syncwarp();
     rows_dot_coalesced<T, D, kMemberSteps>(nvalid, [&](int i) { return mykp[i]; }, qv, mysc + 32);
     __syncwarp();
@@ -904,6 +950,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] *= corr;
     m = mn;
+    if (ev) mysc[my_rank] = pe;  // the exact tokens' weights in rank order
     const bool okw = mbar_wait(&bar[warp], phase, a.status);
     phase ^= 1u;
     if (!okw) {
@@ -911,31 +958,49 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       __syncwarp();
       return;
     }
-    unsigned long long rest = (unsigned long long)vm | ((unsigned long long)cmb << 32);
-    while (rest) {
-      const int j = __ffsll((long long)rest) - 1;
-      rest &= rest - 1;
-      const float pj = __shfl_sync(0xffffffffu, j < 32 ? pe : pc, j & 31);
-      float v[DPL];
-      if constexpr (sizeof(T) == 2 && DPL == 4) {
-        const uint2 rw = *reinterpret_cast<const uint2*>(myV + j * D + lane * DPL);
-        v[0] = __uint_as_float(rw.x << 16);
-        v[1] = __uint_as_float(rw.x & 0xffff0000u);
-        v[2] = __uint_as_float(rw.y << 16);
-        v[3] = __uint_as_float(rw.y & 0xffff0000u);
-      } else {
+    __syncwarp();
+    // exact tokens: the packed rows in rank order, four per step
+    int j = 0;
+    for (; j + 4 <= nvalid; j += 4) {
+      const float4 p4 = *reinterpret_cast<const float4*>(mysc + j);
+      float v0[DPL], v1[DPL], v2[DPL], v3[DPL];
+      lds_f<T, DPL>(myV + (j + 0) * D + lane * DPL, v0);
+      lds_f<T, DPL>(myV + (j + 1) * D + lane * DPL, v1);
+      lds_f<T, DPL>(myV + (j + 2) * D + lane * DPL, v2);
+      lds_f<T, DPL>(myV + (j + 3) * D + lane * DPL, v3);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) v[i] = Elem<T>::to_f(myV[j * D + lane * DPL + i]);
+      for (int i = 0; i < DPL; i += 2) {
+        float2 a2 = make_float2(acc[i], acc[i + 1]);
+        a2 = ffma2(make_float2(p4.x, p4.x), make_float2(v0[i], v0[i + 1]), a2);
+        a2 = ffma2(make_float2(p4.y, p4.y), make_float2(v1[i], v1[i + 1]), a2);
+        a2 = ffma2(make_float2(p4.z, p4.z), make_float2(v2[i], v2[i + 1]), a2);
+        a2 = ffma2(make_float2(p4.w, p4.w), make_float2(v3[i], v3[i + 1]), a2);
+        acc[i] = a2.x;
+        acc[i + 1] = a2.y;
       }
+    }
+    for (; j < nvalid; ++j) {
+      const float pj = mysc[j];
+      float v[DPL];
+      lds_f<T, DPL>(myV + j * D + lane * DPL, v);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, v[i], acc[i]);
+    }
+    // coarse entries, in lane order
+    unsigned rest = cmb;
+    while (rest) {
+      const int jc = __ffs((int)rest) - 1;
+      rest &= rest - 1;
+      const float pj = __shfl_sync(0xffffffffu, pc, jc);
+      float v[DPL];
+      lds_f<T, DPL>(myV + (32 + jc) * D + lane * DPL, v);
 #pragma unroll
       for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, v[i], acc[i]);
     }
     __syncwarp();
   };
-  // the sink tokens [0, min(sinks, window start)) are exact entries (last warp)
+  // the sink tokens (last warp)
   if (warp == kWarps - 1) {
-    const int64_t wsq = (t / kChunk - a.window / kChunk + 1) > 0 ? (t / kChunk - a.window / kChunk + 1) * kChunk : 0;
-    const int64_t nsk = a.sinks < wsq ? a.sinks : wsq;
     for (int64_t e0 = 0; e0 < nsk; e0 += 32)
       batch(e0 + lane < nsk, Kb + (e0 + lane) * a.st, Vb + (e0 + lane) * a.st, false, 0.f, pV);
   }

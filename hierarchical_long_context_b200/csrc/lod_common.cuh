@@ -181,6 +181,11 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Bring the 128-byte line holding `p` into L2 (no register result, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // One-dimensional TMA bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0),
 // completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
