@@ -545,8 +545,8 @@ struct RefineSmem {
 // Scores of up to 32 d-rows against q, loaded with coalesced 16-byte loads:
 // each half (or quarter) of the warp reads one whole row per step and the
 // row's score is reduced over its lanes.  rowptr(i) gives row i (valid for
-// i < n).  Writes score i to out[i].
-template <typename T, int D, int STEPS, typename RowPtr>
+// i < n).  Writes score i to out[i].  EVICT_FIRST: rows read once (L2 policy).
+template <typename T, int D, int STEPS, bool EVICT_FIRST = false, typename RowPtr>
 __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const float (&qv)[16 / sizeof(T)],
                                                    float* out) {
   constexpr int EPL = 16 / sizeof(T);
@@ -554,12 +554,16 @@ __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const f
   constexpr int RPI = 32 / LPR;  // STEPS: loads in flight per lane per round
   const int lane = threadIdx.x & 31;
   const int li = lane % LPR, sub = lane / LPR;
+  const uint64_t pol = EVICT_FIRST ? l2_policy_evict_first() : 0;
   for (int base = 0; base < n; base += STEPS * RPI) {
   uint4 raw[STEPS];
 #pragma unroll
   for (int it = 0; it < STEPS; ++it) {
     const int i = base + it * RPI + sub;
-    if (i < n) raw[it] = __ldg(reinterpret_cast<const uint4*>(rowptr(i) + li * EPL));
+    if (i < n) {
+      const uint4* src = reinterpret_cast<const uint4*>(rowptr(i) + li * EPL);
+      raw[it] = EVICT_FIRST ? ldg_hint(src, pol) : __ldg(src);
+    }
   }
 #pragma unroll
   for (int it = 0; it < STEPS; ++it) {
@@ -914,6 +918,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   // round are brought into L2 while that round is in flight
   constexpr int kMemberSteps = 8;
   constexpr int kFirstRound = kMemberSteps * (32 / LPR);
+  const uint64_t l2once = l2_policy_evict_first();  // member rows are read once
   // One batch of up to 32 exact tokens (lane e: `ev`, key and value rows
   // `krow`, `vrow`) and up to 32 coarse entries (lane p: `cvb`, logit `lgc`,
   // value row `crow`): the value rows are staged in shared memory by TMA
@@ -929,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const int my_rank = __popc(vm & ((1u << lane) - 1u));
     if (lane == 0) mbar_arrive_expect(&bar[warp], (uint32_t)(nvalid + __popc(cmb)) * ROWB);
     __syncwarp();
-    if (ev) bulk_g2s(myV + my_rank * D, vrow, ROWB, &bar[warp]);
+    if (ev) bulk_g2s_hint(myV + my_rank * D, vrow, ROWB, &bar[warp], l2once);
     if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
     if (ev) {
       mykp[my_rank] = krow;
@@ -937,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
         for (int o = 0; o < ROWB; o += 128) prefetch_l2(reinterpret_cast<const char*>(krow) + o);
     }
     __syncwarp();
-    rows_dot_coalesced<T, D, kMemberSteps>(nvalid, [&](int i) { return mykp[i]; }, qv, mysc + 32);
+    rows_dot_coalesced<T, D, kMemberSteps, true>(nvalid, [&](int i) { return mykp[i]; }, qv, mysc + 32);
     __syncwarp();
     const float lge = ev ? mysc[32 + my_rank] : -INFINITY;
     const float lgcb = cvb ? lgc : -INFINITY;

@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t grow0 = unit_kv * a.Cmax * a.k;  // this unit's first summary row
   const int32_t* gM = a.gMeta + grow0;  // size | page range per group
 
-  // producer (warp 0, all lanes): tile t0 + i into ring slot i % kStages
+  // producer (warp 0, all lanes): tile t0 + i into ring slot i % kStages;
+  // the tiles are read once per call (evict-first in L2)
+  const uint64_t l2pol = l2_policy_evict_first();
   auto issue_tile = [&](int i) {
     const int st = i % kStages;
     const int64_t tile = t0 + i;
@@ -159,16 +161,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect(&full[st], 2u * kTileBytes);
       if (tile < gt) {
         const int row = (int)(grow0 + tile * TROWS);
-        tc::tma_load_2d(kd, &maps.gK, 0, row, &full[st]);
-        tc::tma_load_2d(kd + kTileBytes / 2, &maps.gK, 64, row, &full[st]);
-        tc::tma_load_2d(vd, &maps.gV, 0, row, &full[st]);
-        tc::tma_load_2d(vd + kTileBytes / 2, &maps.gV, 64, row, &full[st]);
+        tc::tma_load_2d(kd, &maps.gK, 0, row, &full[st], l2pol);
+        tc::tma_load_2d(kd + kTileBytes / 2, &maps.gK, 64, row, &full[st], l2pol);
+        tc::tma_load_2d(vd, &maps.gV, 0, row, &full[st], l2pol);
+        tc::tma_load_2d(vd + kTileBytes / 2, &maps.gV, 64, row, &full[st], l2pol);
       } else {
         const int pos = (int)(ws + (tile - gt) * TROWS);
-        tc::tma_load_4d(kd, &maps.K, 0, pos, kvh, b, &full[st]);
-        tc::tma_load_4d(kd + kTileBytes / 2, &maps.K, 64, pos, kvh, b, &full[st]);
-        tc::tma_load_4d(vd, &maps.V, 0, pos, kvh, b, &full[st]);
-        tc::tma_load_4d(vd + kTileBytes / 2, &maps.V, 64, pos, kvh, b, &full[st]);
+        tc::tma_load_4d(kd, &maps.K, 0, pos, kvh, b, &full[st], l2pol);
+        tc::tma_load_4d(kd + kTileBytes / 2, &maps.K, 64, pos, kvh, b, &full[st], l2pol);
+        tc::tma_load_4d(vd, &maps.V, 0, pos, kvh, b, &full[st], l2pol);
+        tc::tma_load_4d(vd + kTileBytes / 2, &maps.V, 64, pos, kvh, b, &full[st], l2pol);
       }
     }
     if (tile < gt) {  // the tile's groups' size and page range (zero past the visible ones)
