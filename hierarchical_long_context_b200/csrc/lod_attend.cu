@@ -82,6 +82,60 @@ __device__ __forceinline__ void lds_f(const T* p, float (&v)[N]) {
   }
 }
 
+// Read-only global loads as volatile asm: they keep their place in program
+// order (the compiler neither sinks them to their first use nor merges them),
+// so that loads meant to overlap are in flight together.
+__device__ __forceinline__ uint4 ldv_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ int ldv_s32(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ int ldv_s16(const int16_t* p) {
+  short v;
+  asm volatile("ld.global.nc.s16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+template <typename T, int N>
+__device__ __forceinline__ void ldv_f(const T* p, float (&v)[N]) {
+  if constexpr (N * sizeof(T) == 16) {
+    const uint4 a = ldv_u4(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    if constexpr (sizeof(T) == 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(w[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+  } else if constexpr (N * sizeof(T) == 8) {
+    uint32_t x, y;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "l"(p));
+    if constexpr (sizeof(T) == 4) {
+      v[0] = __uint_as_float(x);
+      v[1] = __uint_as_float(y);
+    } else {
+      v[0] = __uint_as_float(x << 16);
+      v[1] = __uint_as_float(x & 0xffff0000u);
+      v[2] = __uint_as_float(y << 16);
+      v[3] = __uint_as_float(y & 0xffff0000u);
+    }
+  } else {
+    static_assert(N * sizeof(T) == 4 && sizeof(T) == 2, "unsupported vector width");
+    uint32_t x;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(x) : "l"(p));
+    v[0] = __uint_as_float(x << 16);
+    v[1] = __uint_as_float(x & 0xffff0000u);
+  }
+}
+
 // Dot product of a whole d-row (owned by one lane) with q held in shared memory.
 template <typename T, int D>
 __device__ __forceinline__ float row_dot(const T* __restrict__ row, const float* __restrict__ qs) {
@@ -534,8 +588,7 @@ struct RefineSmem {
   static constexpr size_t off_c = off_pos + sizeof(int64_t) * kWarps * 32;    // Cand [kMaxTopGroups]
   static constexpr size_t off_key = off_c + sizeof(Cand) * kMaxTopGroups + 16;  // uint64 [kWarps][32]
   static constexpr size_t off_wb = off_key + 8 * kWarps * 32;                  // uint64 [kWarps]
-  static constexpr size_t off_pc = off_wb + 8 * kWarps;                      // int [2][kWarps][32]
-  static constexpr size_t off_bar = off_pc + 4 * 2 * kWarps * 32 + 16;
+  static constexpr size_t off_bar = off_wb + 8 * kWarps + 16;
   static constexpr size_t bytes = off_bar + 8 * kWarps + 16;
   // group selection: the survivors of the bound reuse the value buffers
   static constexpr int kSurvCap = (int)(off_q / 8);
@@ -562,7 +615,7 @@ __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const f
     const int i = base + it * RPI + sub;
     if (i < n) {
       const uint4* src = reinterpret_cast<const uint4*>(rowptr(i) + li * EPL);
-      raw[it] = EVICT_FIRST ? ldg_hint(src, pol) : __ldg(src);
+      raw[it] = EVICT_FIRST ? ldg_hint(src, pol) : ldv_u4(src);
     }
   }
 #pragma unroll
@@ -911,8 +964,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   T* myV = Vst + warp * SM::kRows * D;
   float* mysc = sc_s + warp * 64;
   const T** mykp = reinterpret_cast<const T**>(posm_s) + warp * 32;
-  int* mycnt = reinterpret_cast<int*>(smem + SM::off_pc) + warp * 32;
-  int* mybeg = mycnt + kWarps * 32;
   uint32_t phase = 0;
   // member key rows scored per round of coalesced loads; rows past the first
   // round are brought into L2 while that round is in flight
@@ -1017,22 +1068,21 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const int meta = __float_as_int(a.gsc[(u * NQ + r) * (a.Cmax * a.k) + gid].y);
     const int gcnt = meta & 0xffff;
     const int p0 = (meta >> 16) & 0xff, p1 = (meta >> 24) & 0xff;
-    // one round trip: the chunk's page counts and member runs, the group's
-    // mean value and its pages' summary scores
-    float gv[DPL];
-    load_f<T, DPL>(gV + (int64_t)gid * D + lane * DPL, gv);
-    int pcl = 0, pbl = 0;  // the chunk's page counts and member offsets (slot = lane)
-    if (lane < a.P) {
-      pcl = pC[c * a.P + lane];
-      pbl = pB[c * a.P + lane];
-    }
+    // one round trip: the group's mean value, its pages' member counts and
+    // offsets (lane l: page p0 + l) and their summary scores (volatile loads
+    // keep this order; the counts are first needed after the page choice)
     const bool prange_ok = !(p1 < p0 || p1 > a.P || p1 - p0 > 32);
     const int np = prange_ok ? p1 - p0 : 0;
+    float gv[DPL];
+    ldv_f<T, DPL>(gV + (int64_t)gid * D + lane * DPL, gv);
+    int cntp = 0, begp = 0;
+    if (lane < np) {
+      cntp = ldv_s32(pC + c * a.P + p0 + lane);
+      begp = ldv_s16(pB + c * a.P + p0 + lane);
+    }
     const T* pKc = pK + (c * a.P + (prange_ok ? p0 : 0)) * D;
     // (two-tier LoD opens the group whole: no page scores)
     rows_dot_coalesced<T, D, 8>(a.TP > 0 ? np : 0, [&](int i) { return pKc + (int64_t)i * D; }, qv, mysc);
-    mycnt[lane] = pcl;
-    mybeg[lane] = pbl;
     int open_slot[kMaxTopPages];
 #pragma unroll
     for (int x = 0; x < kMaxTopPages; ++x) open_slot[x] = -1;
@@ -1048,13 +1098,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     if (!prange_ok) {
       if (lane == 0) set_status(a.status, LOD_ST_BAD_PAGE);
     } else {
-      // page counts/offsets and the page summary scores
+      // the page summary scores
       __syncwarp();
-      int cntp = 0, begp = 0;
-      if (lane < np) {
-        cntp = mycnt[p0 + lane];
-        begp = mybeg[p0 + lane];
-      }
       const float sc = lane < np ? mysc[lane] : -INFINITY;
       // top-TP pages by (score desc, slot asc)
       float s2 = sc;

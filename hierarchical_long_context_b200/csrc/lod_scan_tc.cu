@@ -73,11 +73,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t u = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // launched as a programmatic dependent: inputs are read only after the
-  // preceding kernel has completed; the refine kernel may launch right away
-  // (it waits for this grid's completion before reading what it writes)
-  pdl_wait();
-  pdl_launch_dependents();
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -110,6 +105,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     kvh = (int)((u / nblk) % a.Hkv);
     blk = u % nblk;
   }
+
+  // ---- set-up that reads no input, done while the preceding kernel drains:
+  // barriers and tensor maps (warp 0), TMEM (warp 1), zeroed weights and the
+  // query rows brought into L2 (softmax warps)
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1 + 32);  // the producer's expect_tx + 32 cp.async arrivals
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(fin, 1);
+    *abort_s = 0;
+    fence_mbar_init();
+    tc::prefetch_tensormap(&maps.gK);
+    tc::prefetch_tensormap(&maps.gV);
+    tc::prefetch_tensormap(&maps.K);
+    tc::prefetch_tensormap(&maps.V);
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp >= 2) {
+    const int t = tid - 64;
+    for (int c2 = t; c2 < 4 * N * 128 / 16; c2 += kSoftThreads)
+      reinterpret_cast<uint4*>(Ps)[c2] = make_uint4(0, 0, 0, 0);
+    // (an L2 prefetch has no effect on what a later load returns)
+    const int r = t >> 1;
+    const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
+    if (r < NQ && (a.seq_lens ? r < a.g : (r < a.g * a.NP && pi < a.pos_hi))) {
+      const int hq = kvh * a.g + (r % a.g);
+      prefetch_l2(static_cast<const __nv_bfloat16*>(a.q) + (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D + (t & 1) * 64);
+    }
+  }
+  // launched as a programmatic dependent: inputs are read only after the
+  // preceding kernel has completed; the refine kernel may launch right away
+  // (it waits for this grid's completion before reading what it writes)
+  pdl_wait();
+  pdl_launch_dependents();
+
   int64_t t_row[NQ];
   bool ok[NQ];
   int64_t t_max = -1;
@@ -185,32 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_mbar_arrive_noinc(&full[st]);
   };
 
-  // ---- set-up: barriers and the first ring stages (warp 0), TMEM (warp 1),
-  // the query operand and zeroed weights (softmax warps)
+  // ---- the first ring stages (warp 0) and the query operand (softmax warps)
   if (warp == 0) {
-    if (lane == 0) {
-      for (int i = 0; i < kStages; ++i) {
-        mbar_init(&full[i], 1 + 32);  // the producer's expect_tx + 32 cp.async arrivals
-        mbar_init(&empty[i], 1);
-      }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&s_full[i], 1);
-        mbar_init(&s_free[i], 4);
-        mbar_init(&p_full[i], 4);
-        mbar_init(&o_done[i], 1);
-      }
-      mbar_init(fin, 1);
-      *abort_s = 0;
-      fence_mbar_init();
-      tc::prefetch_tensormap(&maps.gK);
-      tc::prefetch_tensormap(&maps.gV);
-      tc::prefetch_tensormap(&maps.K);
-      tc::prefetch_tensormap(&maps.V);
-    }
     __syncwarp();
     for (int i = 0; i < kStages && i < ntile; ++i) issue_tile(i);
   }
-  if (warp == 1) tc::tmem_alloc(tmem_slot, kTmemCols);
   if (warp >= 2) {
     const int t = tid - 64;
     for (int c2 = t; c2 < N * (D / 8); c2 += kSoftThreads) {
@@ -229,8 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t off = (uint32_t)((c >> 3) * (N * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
       *reinterpret_cast<uint4*>(Qs + off) = v;
     }
-    for (int c2 = t; c2 < 4 * N * 128 / 16; c2 += kSoftThreads)
-      reinterpret_cast<uint4*>(Ps)[c2] = make_uint4(0, 0, 0, 0);
   }
   tc::fence_proxy_async();
   tc::fence_before_sync();
