@@ -60,6 +60,7 @@ class RowStats(ctypes.Structure):
 _f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
 
 
 def _load():
@@ -83,6 +84,16 @@ def _load():
         lib.orc_attend_row.argtypes = [
             ctypes.POINTER(Params), _f32p, ctypes.c_int64, _f32p, _f32p, ctypes.c_int64,
             _f64p, _f64p, _i32p, _f64p, _f64p, _i32p, _i32p, _i32p, _i32p,
+            ctypes.c_void_p, ctypes.c_void_p, _f64p, ctypes.POINTER(ctypes.c_double),
+            _i32p, _i32p, ctypes.POINTER(RowStats)]
+        lib.orc_quantize_pages.restype = ctypes.c_int
+        lib.orc_quantize_pages.argtypes = [
+            ctypes.POINTER(Params), _f32p, ctypes.c_int64, _i32p, _i32p, _i32p, _u8p, _f32p, _f32p]
+        lib.orc_attend_row_q.restype = ctypes.c_int
+        lib.orc_attend_row_q.argtypes = [
+            ctypes.POINTER(Params), _f32p, ctypes.c_int64, _f32p, _f32p, ctypes.c_int64,
+            _f64p, _f64p, _i32p, _f64p, _f64p, _i32p, _i32p, _i32p, _i32p,
+            _u8p, _f32p, _f32p, _u8p, _f32p, _f32p,
             ctypes.c_void_p, ctypes.c_void_p, _f64p, ctypes.POINTER(ctypes.c_double),
             _i32p, _i32p, ctypes.POINTER(RowStats)]
         lib.orc_dense_row.restype = ctypes.c_int
@@ -162,9 +173,31 @@ def build_sequence(cfg: Config, unit: int, K, V, nchunks: int, want_objective: b
     return out
 
 
-def attend_row(cfg: Config, q, t: int, K, V, index: dict, forced_groups=None, forced_pages=None):
+def quantize_pages(cfg: Config, X, index: dict) -> dict:
+    """Three-tier INT4 page quantiser (keys or values X, [T, d]) over the pages
+    of `index`: code [nchunks*chunk, d] uint8 in member order, scale and low
+    [nchunks*P, d] float32 per page slot and channel."""
+    lib = _load()
+    X = _f32(X)
+    n, C, P, d = index["nchunks"], cfg.chunk, cfg.page_slots, cfg.d
+    code = np.empty((n * C, d), np.uint8)
+    scale = np.empty((n * P, d), np.float32)
+    low = np.empty((n * P, d), np.float32)
+    rc = lib.orc_quantize_pages(
+        ctypes.byref(cfg.c()), X, n, np.ascontiguousarray(index["pCnt"], np.int32),
+        np.ascontiguousarray(index["pBeg"], np.int32), np.ascontiguousarray(index["perm"], np.int32),
+        code, scale, low)
+    if rc != 0:
+        raise ValueError("orc_quantize_pages failed: %d" % rc)
+    return dict(code=code, scale=scale, low=low)
+
+
+def attend_row(cfg: Config, q, t: int, K, V, index: dict, forced_groups=None, forced_pages=None,
+               kq: dict = None, vq: dict = None):
     """LoD attention of one query at position t against one sequence's index.
-    Returns (out[d] fp64, lse, sel_groups, sel_pages, stats dict)."""
+    kq / vq (quantize_pages of K and V): the opened pages' members are read
+    decompressed (three-tier INT4).  Returns (out[d] fp64, lse, sel_groups,
+    sel_pages, stats dict)."""
     lib = _load()
     q = _f32(q); K = _f32(K); V = _f32(V)
     G, TP = cfg.top_groups, cfg.top_pages
@@ -179,13 +212,18 @@ def attend_row(cfg: Config, q, t: int, K, V, index: dict, forced_groups=None, fo
         assert fg.size == G
         fp = np.ascontiguousarray(forced_pages, np.int32)
         assert fp.size == G * TP
-    rc = lib.orc_attend_row(
+    qargs = []
+    if kq is not None:
+        qargs = [np.ascontiguousarray(kq["code"], np.uint8), _f32(kq["scale"]), _f32(kq["low"]),
+                 np.ascontiguousarray(vq["code"], np.uint8), _f32(vq["scale"]), _f32(vq["low"])]
+    fn = lib.orc_attend_row_q if kq is not None else lib.orc_attend_row
+    rc = fn(
         ctypes.byref(cfg.c()), q, t, K, V, index["nchunks"],
         np.ascontiguousarray(index["gK"], np.float64), np.ascontiguousarray(index["gV"], np.float64),
         np.ascontiguousarray(index["gCnt"], np.int32), np.ascontiguousarray(index["pK"], np.float64),
         np.ascontiguousarray(index["pV"], np.float64), np.ascontiguousarray(index["pCnt"], np.int32),
         np.ascontiguousarray(index["pBeg"], np.int32), np.ascontiguousarray(index["gPage"], np.int32),
-        np.ascontiguousarray(index["perm"], np.int32),
+        np.ascontiguousarray(index["perm"], np.int32), *qargs,
         fg.ctypes.data_as(ctypes.c_void_p) if fg is not None else None,
         fp.ctypes.data_as(ctypes.c_void_p) if fp is not None else None,
         out, ctypes.byref(lse), sg, sp, ctypes.byref(st))

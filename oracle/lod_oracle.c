@@ -54,6 +54,18 @@
  *             (mean key logit + ln(count), mean value); ln(count) is added
  *             after the 1/sqrt(d) scale, since n copies of exp(x) are
  *             exp(x + ln n).
+ *   R-int4    three-tier INT4 ("Level of Detail Attention", the paragraph
+ *             after the quality tables: the centroids keep similar keys
+ *             together, so the cache can be stored at INT4, and in the
+ *             three-tier mode only the selected pages are decompressed): the
+ *             member keys and values of every page are stored as 4-bit codes
+ *             of a per-page, per-channel asymmetric quantiser.  For page p and
+ *             channel j over the page's members: low = min x, scale =
+ *             (max x - low) / 15 in fp32, code = clamp(rint((x - low) /
+ *             scale), 0, 15) (0 when scale = 0), and the decompressed value is
+ *             fmaf(code, scale, low) in fp32.  Opened pages' exact entries use
+ *             the decompressed keys and values; the summaries, the sinks and
+ *             the window keep the cache values.
  *   R-prec    decisions that turn floating point into an integer (the k-means
  *             argmin and argmax, the top-k rankings) are taken in fp32, the
  *             precision of the GPU kernels; every softmax, mean and output is
@@ -333,6 +345,53 @@ int orc_build_sequence(const orc_params* p, uint64_t unit, const float* K, const
   return ORC_OK;
 }
 
+/*
+ * Page quantiser of R-int4 for one sequence.  X: [nchunks*chunk][d] cache
+ * values (keys or values); pCnt/pBeg/perm: the index of orc_build_sequence.
+ * Outputs, member-ordered like perm (row m of chunk c is the token at offset
+ * perm[c*chunk + m]):
+ *   code  [nchunks*chunk][d]  one 4-bit code per byte (0 past the members)
+ *   scale [nchunks*P][d]      per page slot and channel (0 for unused slots)
+ *   low   [nchunks*P][d]
+ */
+int orc_quantize_pages(const orc_params* p, const float* X, int64_t nchunks, const int32_t* pCnt,
+                       const int32_t* pBeg, const int32_t* perm, uint8_t* code, float* scale,
+                       float* low) {
+  const int d = p->d, C = p->chunk, P = orc_page_slots(p);
+  if (d <= 0 || C <= 0) return ORC_EINVAL;
+  memset(code, 0, (size_t)nchunks * C * d);
+  for (int64_t c = 0; c < nchunks; ++c)
+    for (int q = 0; q < P; ++q) {
+      const int64_t pid = c * P + q;
+      const int m = pCnt[pid], b0 = pBeg[pid];
+      for (int j = 0; j < d; ++j) {
+        scale[pid * d + j] = 0.0f;
+        low[pid * d + j] = 0.0f;
+      }
+      if (m <= 0) continue;
+      if (b0 < 0 || b0 + m > C) return ORC_EINVAL;
+      for (int j = 0; j < d; ++j) {
+        float lo = INFINITY, hi = -INFINITY;
+        for (int r = 0; r < m; ++r) {
+          const float x = X[(c * C + perm[c * C + b0 + r]) * (int64_t)d + j];
+          if (x < lo) lo = x;
+          if (x > hi) hi = x;
+        }
+        const float sc = (hi - lo) / 15.0f;
+        scale[pid * d + j] = sc;
+        low[pid * d + j] = lo;
+        for (int r = 0; r < m; ++r) {
+          const float x = X[(c * C + perm[c * C + b0 + r]) * (int64_t)d + j];
+          float v = sc > 0.0f ? rintf((x - lo) / sc) : 0.0f;
+          if (v < 0.0f) v = 0.0f;
+          if (v > 15.0f) v = 15.0f;
+          code[(c * C + b0 + r) * (int64_t)d + j] = (uint8_t)v;
+        }
+      }
+    }
+  return ORC_OK;
+}
+
 /* Per-row bookkeeping returned by orc_attend_row, for the invariant tests. */
 typedef struct {
   int64_t n_exact;         /* exact (position) entries */
@@ -393,12 +452,14 @@ static void take_top(ranked* r, int n, int m) {
  * ids c*k+j, best first, -1 padded), sel_pages[top_groups*top_pages]
  * (chunk-global page slots c*P+slot), stats.
  */
-int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* K, const float* V,
-                   int64_t nchunks_built, const double* gK, const double* gV, const int32_t* gCnt,
-                   const double* pK, const double* pV, const int32_t* pCnt, const int32_t* pBeg,
-                   const int32_t* gPage, const int32_t* perm, const int32_t* forced_groups,
-                   const int32_t* forced_pages, double* out, double* lse, int32_t* sel_groups,
-                   int32_t* sel_pages, orc_row_stats* st) {
+int orc_attend_row_q(const orc_params* p, const float* q, int64_t t, const float* K, const float* V,
+                     int64_t nchunks_built, const double* gK, const double* gV, const int32_t* gCnt,
+                     const double* pK, const double* pV, const int32_t* pCnt, const int32_t* pBeg,
+                     const int32_t* gPage, const int32_t* perm, const uint8_t* kcode,
+                     const float* kscale, const float* klow, const uint8_t* vcode,
+                     const float* vscale, const float* vlow, const int32_t* forced_groups,
+                     const int32_t* forced_pages, double* out, double* lse, int32_t* sel_groups,
+                     int32_t* sel_pages, orc_row_stats* st) {
   const int d = p->d, C = p->chunk, k = p->clusters, P = orc_page_slots(p);
   const int G = p->top_groups, TP = p->top_pages;
   const double sc = scale_of(p);
@@ -423,10 +484,14 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
   ranked* gr = (ranked*)malloc(sizeof(ranked) * (nvis * k + 1));
   ranked* pr = (ranked*)malloc(sizeof(ranked) * (P + 1));
   char* opened = (char*)calloc((size_t)(nvis * k + 1), 1);
-  if (!lg || !vf || !vd || !mult || !gr || !pr || !opened) {
-    free(lg); free(vf); free(vd); free(mult); free(gr); free(pr); free(opened);
+  /* R-int4: decompressed member rows of the opened pages (keys, then values) */
+  const int quant = kcode && kscale && klow && vcode && vscale && vlow;
+  float* deq = quant ? (float*)malloc(sizeof(float) * 2 * (size_t)(G * C + 1) * d) : NULL;
+  if (!lg || !vf || !vd || !mult || !gr || !pr || !opened || (quant && !deq)) {
+    free(lg); free(vf); free(vd); free(mult); free(gr); free(pr); free(opened); free(deq);
     return ORC_ENOMEM;
   }
+  int64_t ndeq = 0;
   int64_t ne = 0;
   orc_row_stats s = {0};
   s.window_start = (double)ws;
@@ -515,7 +580,19 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
       if (is_open) {
         for (int m = 0; m < pCnt[pid]; ++m) {
           int64_t pos = c * C + perm[c * C + pBeg[pid] + m];
-          lg[ne] = sc * dot64f(q, K + pos * d, d); vf[ne] = V + pos * d; vd[ne] = 0; mult[ne] = 1; ++ne;
+          if (quant) {
+            float* kh = deq + (size_t)(2 * ndeq) * d;
+            float* vh = kh + d;
+            const int64_t row = (c * C + pBeg[pid] + m) * (int64_t)d;
+            for (int j = 0; j < d; ++j) {
+              kh[j] = fmaf((float)kcode[row + j], kscale[pid * d + j], klow[pid * d + j]);
+              vh[j] = fmaf((float)vcode[row + j], vscale[pid * d + j], vlow[pid * d + j]);
+            }
+            ++ndeq;
+            lg[ne] = sc * dot64f(q, kh, d); vf[ne] = vh; vd[ne] = 0; mult[ne] = 1; ++ne;
+          } else {
+            lg[ne] = sc * dot64f(q, K + pos * d, d); vf[ne] = V + pos * d; vd[ne] = 0; mult[ne] = 1; ++ne;
+          }
           s.n_exact++;
         }
       } else {
@@ -543,8 +620,20 @@ int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* 
   for (int64_t e = 0; e < ne; ++e) ws_ += exp(lg[e] - m) / L;
   s.weight_sum = ws_;
   if (st) *st = s;
-  free(lg); free(vf); free(vd); free(mult); free(gr); free(pr); free(opened);
+  free(lg); free(vf); free(vd); free(mult); free(gr); free(pr); free(opened); free(deq);
   return ORC_OK;
+}
+
+/* orc_attend_row_q with the opened pages read in the cache values. */
+int orc_attend_row(const orc_params* p, const float* q, int64_t t, const float* K, const float* V,
+                   int64_t nchunks_built, const double* gK, const double* gV, const int32_t* gCnt,
+                   const double* pK, const double* pV, const int32_t* pCnt, const int32_t* pBeg,
+                   const int32_t* gPage, const int32_t* perm, const int32_t* forced_groups,
+                   const int32_t* forced_pages, double* out, double* lse, int32_t* sel_groups,
+                   int32_t* sel_pages, orc_row_stats* st) {
+  return orc_attend_row_q(p, q, t, K, V, nchunks_built, gK, gV, gCnt, pK, pV, pCnt, pBeg, gPage, perm,
+                          NULL, NULL, NULL, NULL, NULL, NULL, forced_groups, forced_pages, out, lse,
+                          sel_groups, sel_pages, st);
 }
 
 /* Full softmax attention of one query at position t over keys [0, t], fp64. */

@@ -330,3 +330,102 @@ def test_forced_selection_reproduces_free_selection(tiny_bf16):
         out2, lse2, sg2, sp2, _ = oracle.attend_row(cfg, q, t, K, V, idx, sg, sp)
         np.testing.assert_allclose(out, out2, rtol=0, atol=1e-13)   # entry order differs
         np.testing.assert_array_equal(sg, sg2)
+
+
+# ---------------------------------------------------------------- three-tier INT4
+
+def _page_members(idx, cfg, pid):
+    """(chunk, member-order rows, token offsets) of page slot `pid`."""
+    C, P = cfg.chunk, cfg.page_slots
+    c, b0, m = pid // P, idx["pBeg"][pid], idx["pCnt"][pid]
+    rows = c * C + b0 + np.arange(m)
+    return c, rows, c * C + idx["perm"][c * C + b0 + np.arange(m)]
+
+
+def _fused(qz, rows, pid):
+    """code * scale + low with one rounding to fp32 (the product of a 4-bit
+    code and an fp32 scale, plus an fp32 low, is exact in fp64)."""
+    return (qz["code"][rows].astype(np.float64) * qz["scale"][pid].astype(np.float64)
+            + qz["low"][pid].astype(np.float64)).astype(np.float32)
+
+
+@pytest.mark.parametrize("which", ["tiny", "tiny_bf16"])
+def test_int4_codes_are_nearest_grid_points(which, request):
+    """Three-tier INT4 reading: per page and channel the grid is low + c *
+    scale, c = 0..15, low = min and low + 15 scale = max over the page's
+    members; every member gets a nearest grid point.  Checked by enumerating
+    all 16 grid points in fp64, independently of the oracle's rounding."""
+    w, cfg, K, V, idx = request.getfixturevalue(which)
+    for X in (K, V):
+        X = np.asarray(X, np.float32)
+        qz = oracle.quantize_pages(cfg, X, idx)
+        assert qz["code"].max() <= 15
+        used = np.nonzero(idx["pCnt"] > 0)[0]
+        for pid in used[:: max(1, len(used) // 40)]:
+            _, rows, toks = _page_members(idx, cfg, pid)
+            x = X[toks].astype(np.float64)                       # [m, d]
+            lo = qz["low"][pid].astype(np.float64)
+            sc = qz["scale"][pid].astype(np.float64)
+            np.testing.assert_array_equal(lo, x.min(0))
+            np.testing.assert_allclose(lo + 15 * sc, x.max(0), rtol=1e-6, atol=1e-6)
+            grid = lo[None, :] + np.arange(16)[:, None] * sc[None, :]    # [16, d]
+            dist = np.abs(x[:, None, :] - grid[None, :, :])              # [m, 16, d]
+            best = dist.min(1)
+            got = np.take_along_axis(dist, qz["code"][rows].astype(np.int64)[:, None, :], 1)[:, 0]
+            # the fp32 quotient may round a near-tie either way
+            assert np.all(got <= best + 1e-6 * (np.abs(x) + 15 * sc[None, :]) + 1e-12)
+            # round trip within half a step
+            xh = (qz["code"][rows].astype(np.float32) * qz["scale"][pid] + qz["low"][pid]).astype(np.float64)
+            assert np.all(np.abs(xh - x) <= sc[None, :] / 2 * (1 + 1e-5) + 1e-7 * np.abs(x) + 1e-12)
+
+
+def test_int4_constant_pages_decompress_exactly():
+    """A page whose members are equal in a channel has scale 0, code 0 and
+    decompresses to the value itself: on the zero-variance cache every page
+    is constant, so three-tier INT4 equals the cache-value path and dense
+    attention (How It Works, zero-variance paragraph)."""
+    w = synth.WORKLOADS["decode_tiny_f32_zero_variance"]
+    K, V = synth.unit_kv(w, 0, 0)
+    cfg = _cfg(w)
+    idx = oracle.build_sequence(cfg, 0, K, V, w.T // 256)
+    kq, vq = oracle.quantize_pages(cfg, K, idx), oracle.quantize_pages(cfg, V, idx)
+    used = idx["pCnt"] > 0
+    assert np.all(kq["scale"][used] == 0) and np.all(vq["scale"][used] == 0)
+    assert np.all(kq["code"] == 0) and np.all(vq["code"] == 0)
+    for q in _rows(w, 6):
+        for t in (w.T - 1, 3000):
+            o4, l4, sg4, sp4, _ = oracle.attend_row(cfg, q, t, K, V, idx, kq=kq, vq=vq)
+            o, l, sg, sp, _ = oracle.attend_row(cfg, q, t, K, V, idx)
+            np.testing.assert_array_equal(o4, o)
+            assert l4 == l and np.array_equal(sg4, sg) and np.array_equal(sp4, sp)
+            dout, dlse = oracle.dense_row(cfg, q, t, K, V)
+            np.testing.assert_allclose(o4, dout, rtol=0, atol=1e-10)
+
+
+def test_int4_everything_opened_is_dense_over_the_decompressed_cache(tiny_bf16):
+    """With every group and page opened, three-tier INT4 attention is full
+    attention over the cache in which each indexed position holds its
+    decompressed key and value (sinks and window keep the cache values):
+    the decompression is applied to exactly the opened members."""
+    w, _, K, V, _ = tiny_bf16
+    K = np.asarray(K, np.float32); V = np.asarray(V, np.float32)
+    cfg = _cfg(w, top_groups=64, top_pages=64)
+    T = 1536
+    idx = oracle.build_sequence(cfg, 0, K[:T], V[:T], T // 256)
+    kq, vq = oracle.quantize_pages(cfg, K[:T], idx), oracle.quantize_pages(cfg, V[:T], idx)
+    P = cfg.page_slots
+    for q in _rows(w, 4):
+        for t in (T - 1, 1300):
+            nvis = t // 256 - cfg.window // 256 + 1
+            Kh, Vh = K[:t + 1].copy(), V[:t + 1].copy()
+            for pid in range(nvis * P):
+                if idx["pCnt"][pid] <= 0:
+                    continue
+                _, rows, toks = _page_members(idx, cfg, pid)
+                Kh[toks] = _fused(kq, rows, pid)
+                Vh[toks] = _fused(vq, rows, pid)
+            out, lse, _, _, st = oracle.attend_row(cfg, q, t, K, V, idx, kq=kq, vq=vq)
+            assert st["n_coarse_groups"] == 0 and st["n_coarse_pages"] == 0
+            dout, dlse = oracle.dense_row(cfg, q, t, Kh, Vh)
+            np.testing.assert_allclose(out, dout, rtol=0, atol=1e-9)
+            assert abs(lse - dlse) < 1e-9
