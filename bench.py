@@ -215,12 +215,12 @@ def barrier(world):
 
 # ---------------------------------------------------------------- workloads
 
-def params_for(w, k=None):
+def params_for(w, k=None, kv_bits=0):
     from hierarchical_long_context_b200 import api
     return api.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, Tmax=((w.T + 255) // 256) * 256,
                       dtype=w.torch_dtype, clusters=k or w.clusters[0], kmeans_iters=w.iters,
                       top_groups=w.top_groups, top_pages=w.top_pages, window=w.window, sinks=w.sinks,
-                      seed=w.seed)
+                      seed=w.seed, kv_bits=kv_bits)
 
 
 def run_decode(w, args, dev, stream, world, rank, peaks):
@@ -361,13 +361,13 @@ def synth_q(w):
     return synth.decode_queries(w)
 
 
-def run_decode_variant(w, dev, stream, peaks, steps, replicas, label, device_gen=False):
+def run_decode_variant(w, dev, stream, peaks, steps, replicas, label, device_gen=False, kv_bits=0):
     """A decode leg on workload `w` (device time of `steps` back-to-back steps
     over rotating input replicas, as the headline leg) with the roofline over
     the bytes its own selections touch."""
     from hierarchical_long_context_b200 import api, metrics
     from hierarchical_long_context_b200 import synth
-    p = params_for(w)
+    p = params_for(w, kv_bits=kv_bits)
     if device_gen:
         Kd, Vd = synth.kv_cache_device(w, dev)
     else:
@@ -403,7 +403,7 @@ def run_decode_variant(w, dev, stream, peaks, steps, replicas, label, device_gen
     gbs = touched / (ms * 1e-3) / 1e9
     del reps
     return dict(workload=label, value=w.B / (ms * 1e-3), unit="queries/s", ms_per_step=ms,
-                seq_len=w.T, B=w.B, top_groups=p.top_groups, top_pages=p.top_pages,
+                seq_len=w.T, B=w.B, top_groups=p.top_groups, top_pages=p.top_pages, kv_bits=p.kv_bits,
                 l2="%d rotating input replicas" % R,
                 roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
                               frac=gbs / peaks["hbm_gbs"], algorithmic_bytes_per_launch=touched),
@@ -537,6 +537,10 @@ def main():
     res.pop("_touch")
     extras = {}
     if not args.no_extras:
+        extras["decode_int4"] = run_decode_variant(
+            w, dev, stream, peaks, 1000, 4,
+            "%s, three-tier INT4 (opened pages read from 4-bit codes)" % w.name, kv_bits=4)
+        torch.cuda.empty_cache()
         extras["decode_two_tier"] = run_decode_variant(
             w.with_(top_pages=0), dev, stream, peaks, 1000, 4,
             "%s, two-tier LoD (top_pages = 0: opened groups read whole)" % w.name)

@@ -29,14 +29,15 @@ class lod_params(ctypes.Structure):
         ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("chunk", ctypes.c_int32),
         ("page", ctypes.c_int32), ("clusters", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
         ("top_groups", ctypes.c_int32), ("top_pages", ctypes.c_int32), ("window", ctypes.c_int32),
-        ("sinks", ctypes.c_int32), ("reserved0", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("sinks", ctypes.c_int32), ("kv_bits", ctypes.c_int32), ("seed", ctypes.c_uint64),
         ("scale", ctypes.c_float), ("reserved1", ctypes.c_int32), ("Tmax", ctypes.c_int64),
     ]
 
 
 class lod_index(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("gK", "gV", "gCnt", "pK", "pV", "pCnt", "pBeg", "gPage", "perm", "mK", "mV", "gMeta")]
+                ("gK", "gV", "gCnt", "pK", "pV", "pCnt", "pBeg", "gPage", "perm", "mK", "mV", "gMeta",
+                 "qK", "qV", "qKs", "qVs")]
 
 
 INDEX_FIELDS = [f for f, _ in lod_index._fields_]

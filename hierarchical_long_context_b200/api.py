@@ -36,12 +36,13 @@ class Params:
     scale: float = 0.0
     chunk: int = 256
     page: int = 16
+    kv_bits: int = 0   # 4: three-tier INT4 (opened pages read from 4-bit codes)
 
     def c(self) -> _lib.lod_params:
         return _lib.lod_params(
             _DT[self.dtype], self.B, self.Hq, self.Hkv, self.d, self.chunk, self.page,
             self.clusters, self.kmeans_iters, self.top_groups, self.top_pages, self.window,
-            self.sinks, 0, self.seed & (2**64 - 1), self.scale, 0, self.Tmax)
+            self.sinks, self.kv_bits, self.seed & (2**64 - 1), self.scale, 0, self.Tmax)
 
     @property
     def page_slots(self) -> int:
@@ -53,7 +54,8 @@ class Params:
 
 
 class Index:
-    """The twelve device arrays of lod_index, as torch tensors."""
+    """The sixteen device arrays of lod_index, as torch tensors (the arrays
+    the parameters do not use are empty)."""
 
     def __init__(self, params: Params, device="cuda"):
         lib = load()
@@ -71,9 +73,14 @@ class Index:
         self.pBeg = torch.zeros(*u, Cmax * P, dtype=torch.int16, device=device)
         self.gPage = torch.zeros(*u, Cmax * (k + 1), dtype=torch.int16, device=device)
         self.perm = torch.full((*u, Cmax * p.chunk), -1, dtype=torch.int16, device=device)
-        self.mK = torch.zeros(*u, Cmax * p.chunk, d, dtype=p.dtype, device=device)
+        int4 = p.kv_bits == 4
+        self.mK = torch.zeros(*u, 0 if int4 else Cmax * p.chunk, d, dtype=p.dtype, device=device)
         self.mV = torch.zeros_like(self.mK)
         self.gMeta = torch.zeros(*u, Cmax * k, dtype=torch.int32, device=device)
+        self.qK = torch.zeros(*u, Cmax * p.chunk if int4 else 0, d // 2, dtype=torch.uint8, device=device)
+        self.qV = torch.zeros_like(self.qK)
+        self.qKs = torch.zeros(*u, Cmax * P if int4 else 0, d, 2, dtype=torch.float32, device=device)
+        self.qVs = torch.zeros_like(self.qKs)
         for i, f in enumerate(_lib.INDEX_FIELDS):
             t = getattr(self, f)
             assert t.numel() * t.element_size() == sizes[i], (f, t.numel() * t.element_size(), sizes[i])

@@ -34,13 +34,16 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t elem_bytes(const lod_params* p) { return p->dtype == LOD_DTYPE_F32 ? 4 : 2; }
 int32_t page_slots(const lod_params* p) { return p->chunk / p->page + p->clusters; }
 int32_t g_of(const lod_params* p) { return p->Hq / p->Hkv; }
-int kg_of(const lod_params* p) { return p->top_groups <= 8 ? 8 : 16; }
 // query rows per scan unit (registers: NQ x 8 fp32 accumulators per lane)
 int nq_max(const lod_params*) { return 8; }
 
 int32_t validate(const lod_params* p) {
   if (!p) return fail(LOD_EINVAL, "params is NULL");
-  if (p->reserved0 != 0 || p->reserved1 != 0) return fail(LOD_EINVAL, "reserved fields must be 0");
+  if (p->reserved1 != 0) return fail(LOD_EINVAL, "reserved fields must be 0");
+  if (p->kv_bits != 0 && p->kv_bits != 4)
+    return fail(LOD_EUNSUPPORTED, "kv_bits = %d unsupported (0 or 4)", p->kv_bits);
+  if (p->kv_bits == 4 && p->top_pages == 0)
+    return fail(LOD_EUNSUPPORTED, "three-tier INT4 (kv_bits = 4) needs top_pages >= 1");
   if (p->dtype != LOD_DTYPE_F32 && p->dtype != LOD_DTYPE_BF16)
     return fail(LOD_EUNSUPPORTED, "dtype %d unsupported (0=f32, 1=bf16)", p->dtype);
   if (p->B < 1 || p->Hq < 1 || p->Hkv < 1) return fail(LOD_EINVAL, "B, Hq, Hkv must be >= 1");
@@ -79,13 +82,17 @@ int32_t validate_kv(const lod_params* p, const void* K, const void* V, const int
   return LOD_OK;
 }
 
-int32_t validate_index(const lod_index* ix) {
+int32_t validate_index(const lod_params* p, const lod_index* ix) {
   if (!ix) return fail(LOD_EINVAL, "index is NULL");
-  const void* ptrs[LOD_INDEX_ARRAYS] = {ix->gK,   ix->gV,    ix->gCnt, ix->pK, ix->pV, ix->pCnt,
-                                        ix->pBeg, ix->gPage, ix->perm, ix->mK, ix->mV, ix->gMeta};
+  const void* ptrs[LOD_INDEX_ARRAYS] = {ix->gK,   ix->gV,    ix->gCnt, ix->pK, ix->pV,    ix->pCnt,
+                                        ix->pBeg, ix->gPage, ix->perm, ix->mK, ix->mV,    ix->gMeta,
+                                        ix->qK,   ix->qV,    ix->qKs,  ix->qVs};
+  const bool int4 = p->kv_bits == 4;
   for (int i = 0; i < LOD_INDEX_ARRAYS; ++i) {
+    const bool used = (i == 9 || i == 10) ? !int4 : (i >= 12 ? int4 : true);
+    if (!used) continue;
     if (!ptrs[i]) return fail(LOD_EINVAL, "index field %d is NULL", i);
-    if (i == 0 || i == 1 || i == 3 || i == 4 || i == 9 || i == 10) {
+    if (i == 0 || i == 1 || i == 3 || i == 4 || i == 9 || i == 10 || i >= 12) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index summary %d must be 16-byte aligned", i);
     } else if (i == 8) {
       if (!aligned16(ptrs[i])) return fail(LOD_EINVAL, "index member list (perm) must be 16-byte aligned");
@@ -216,6 +223,11 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   a.mK = ix->mK;
   a.mV = ix->mV;
   a.gMeta = ix->gMeta;
+  a.kv_bits = p->kv_bits;
+  a.qK = ix->qK;
+  a.qV = ix->qV;
+  a.qKs = reinterpret_cast<const float2*>(ix->qKs);
+  a.qVs = reinterpret_cast<const float2*>(ix->qVs);
   a.B = p->B;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
@@ -269,6 +281,11 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.mK = ix->mK;
   a.mV = ix->mV;
   a.gMeta = ix->gMeta;
+  a.kv_bits = p->kv_bits;
+  a.qK = ix->qK;
+  a.qV = ix->qV;
+  a.qKs = reinterpret_cast<float2*>(ix->qKs);
+  a.qVs = reinterpret_cast<float2*>(ix->qVs);
   a.status = static_cast<uint32_t*>(ws);
   cudaError_t e = lod::launch_build(a, p->dtype, p->d, c1 - c0, p->B, stream);
   if (e != cudaSuccess) return cuda_fail(e, "index build launch");
@@ -296,8 +313,11 @@ int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]) {
   bytes[6] = units * Cmax * P * sizeof(int16_t);
   bytes[7] = units * Cmax * (k + 1) * sizeof(int16_t);
   bytes[8] = units * Cmax * p->chunk * sizeof(int16_t);
-  bytes[9] = bytes[10] = units * Cmax * p->chunk * d * e;
+  const bool int4 = p->kv_bits == 4;
+  bytes[9] = bytes[10] = int4 ? 0 : units * Cmax * p->chunk * d * e;
   bytes[11] = units * Cmax * k * sizeof(int32_t);
+  bytes[12] = bytes[13] = int4 ? units * Cmax * p->chunk * d / 2 : 0;
+  bytes[14] = bytes[15] = int4 ? units * Cmax * P * d * 2 * sizeof(float) : 0;
   g_err[0] = 0;
   return LOD_OK;
 }
@@ -321,7 +341,7 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V, const
                         size_t ws_bytes, lod_stream_t stream) {
   int32_t rc = validate(p);
   if (!rc) rc = validate_kv(p, K, V, kv_strides);
-  if (!rc) rc = validate_index(index);
+  if (!rc) rc = validate_index(p, index);
   if (rc) return rc;
   if (chunk_begin < 0 || chunk_end <= chunk_begin || chunk_end * p->chunk > p->Tmax)
     return fail(LOD_EINVAL, "chunk range [%lld, %lld) invalid for Tmax %lld", (long long)chunk_begin,
@@ -340,7 +360,7 @@ int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void
                    size_t ws_bytes, lod_stream_t stream) {
   int32_t rc = validate(p);
   if (!rc) rc = validate_kv(p, K, V, kv_strides);
-  if (!rc) rc = validate_index(index);
+  if (!rc) rc = validate_index(p, index);
   if (rc) return rc;
   if (!q || !out || !seq_lens) return fail(LOD_EINVAL, "q, out and seq_lens must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
@@ -376,7 +396,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
                     lod_stream_t stream) {
   int32_t rc = validate(p);
   if (!rc) rc = validate_kv(p, K, V, kv_strides);
-  if (!rc) rc = validate_index(index);
+  if (!rc) rc = validate_index(p, index);
   if (rc) return rc;
   if (!q || !out) return fail(LOD_EINVAL, "q and out must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
@@ -493,7 +513,7 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
                                       int32_t* sel_pages, uint32_t* status, lod_stream_t stream) {
   int32_t rc = validate(p);
   if (!rc) rc = validate_kv(p, K, V, kv_strides);
-  if (!rc) rc = validate_index(index);
+  if (!rc) rc = validate_index(p, index);
   if (rc) return rc;
   if (!q || !out || !seq_lens) return fail(LOD_EINVAL, "q, out and seq_lens must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");

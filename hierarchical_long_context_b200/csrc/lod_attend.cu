@@ -136,6 +136,38 @@ __device__ __forceinline__ void ldv_f(const T* p, float (&v)[N]) {
   }
 }
 
+// 4-bit code i of the packed word w as a float (2^23 + code, minus 2^23: exact).
+__device__ __forceinline__ float nibble_f(uint32_t w, int i) {
+  return __int_as_float(0x4B000000u | ((w >> (4 * i)) & 15u)) - 8388608.0f;
+}
+
+// Sum over the warp of 16 per-lane values: lane l receives the total of value
+// l >> 1 (each step halves the values a lane keeps and exchanges the other half).
+__device__ __forceinline__ float transpose_sum16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int h = 8, b = 16; h >= 1; h >>= 1, b >>= 1) {
+    const bool up = (lane & b) != 0;
+#pragma unroll
+    for (int j = 0; j < h; ++j) {
+      const float send = up ? v[j] : v[j + h];
+      const float keep = up ? v[j + h] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, b);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// The 4-bit codes of `lane`'s DPL channels in one member-ordered row.
+template <int D, int DPL>
+__device__ __forceinline__ uint32_t lane_codes(const uint8_t* row, int lane) {
+  if constexpr (DPL == 4) {
+    return *reinterpret_cast<const uint16_t*>(row + lane * 2);
+  } else {
+    static_assert(DPL == 2, "channels per lane");
+    return row[lane];
+  }
+}
+
 // Dot product of a whole d-row (owned by one lane) with q held in shared memory.
 template <typename T, int D>
 __device__ __forceinline__ float row_dot(const T* __restrict__ row, const float* __restrict__ qs) {
@@ -679,7 +711,8 @@ __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* red) {
   return r;
 }
 
-template <typename T, int D, int NQ>
+// Q4: three-tier INT4 (opened pages read from 4-bit codes; a.kv_bits == 4).
+template <typename T, int D, int NQ, bool Q4>
 __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   constexpr int DPL = D / 32;
   constexpr int EPL = 16 / sizeof(T);
@@ -1055,6 +1088,138 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     }
     __syncwarp();
   };
+  // Three-tier INT4 ("Level of Detail Attention", the paragraph after the
+  // quality tables: only the selected pages are decompressed): up to two
+  // opened pages (rows ra/rb of the member-ordered codes, na/nb members, page
+  // slots sa/sb, all relative to the unit) per batch, with the coarse entries
+  // of `batch`.  The pages' codes and (scale, low) quantisers are staged by
+  // TMA; a member's logit is q.low + sum_j (q_j scale_j) code_j and the values
+  // enter as scale_j sum_r p_r code_rj + low_j sum_r p_r per page.  Lane e is
+  // member e % 16 of page e / 16.
+  auto batch_q = [&](int npg, int64_t ra, int na, int64_t sa, int64_t rb, int nb, int64_t sb, bool cvb, float lgc,
+                     const T* crow) {
+    const unsigned cmb = __ballot_sync(0xffffffffu, cvb);
+    if (npg == 0 && !cmb) return;
+    unsigned char* stg = reinterpret_cast<unsigned char*>(myV);
+    constexpr int PB = 8 * D;  // one staged piece: 16 rows of d/2 codes, or d (scale, low) pairs
+    const uint8_t* qKu = a.qK + unit_kv * a.Cmax * kChunk * (D / 2);
+    const uint8_t* qVu = a.qV + unit_kv * a.Cmax * kChunk * (D / 2);
+    const float2* qKsu = a.qKs + unit_kv * a.Cmax * a.P * D;
+    const float2* qVsu = a.qVs + unit_kv * a.Cmax * a.P * D;
+    if (lane == 0) {
+      uint32_t bytes = (uint32_t)__popc(cmb) * ROWB;
+      if (npg > 0) bytes += (uint32_t)(na * D + 2 * PB);
+      if (npg > 1) bytes += (uint32_t)(nb * D + 2 * PB);
+      mbar_arrive_expect(&bar[warp], bytes);
+      if (npg > 0) {
+        bulk_g2s_hint(stg + 0 * PB, qKu + ra * (D / 2), (uint32_t)(na * (D / 2)), &bar[warp], l2once);
+        bulk_g2s_hint(stg + 2 * PB, qVu + ra * (D / 2), (uint32_t)(na * (D / 2)), &bar[warp], l2once);
+        bulk_g2s(stg + 4 * PB, qKsu + sa * D, PB, &bar[warp]);
+        bulk_g2s(stg + 6 * PB, qVsu + sa * D, PB, &bar[warp]);
+      }
+      if (npg > 1) {
+        bulk_g2s_hint(stg + 1 * PB, qKu + rb * (D / 2), (uint32_t)(nb * (D / 2)), &bar[warp], l2once);
+        bulk_g2s_hint(stg + 3 * PB, qVu + rb * (D / 2), (uint32_t)(nb * (D / 2)), &bar[warp], l2once);
+        bulk_g2s(stg + 5 * PB, qKsu + sb * D, PB, &bar[warp]);
+        bulk_g2s(stg + 7 * PB, qVsu + sb * D, PB, &bar[warp]);
+      }
+    }
+    __syncwarp();
+    if (cvb) bulk_g2s(myV + (32 + lane) * D, crow, ROWB, &bar[warp]);
+    float qd[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) qd[i] = qs[lane * DPL + i];
+    const bool okw = mbar_wait(&bar[warp], phase, a.status);
+    phase ^= 1u;
+    if (!okw) {
+      (void)mbar_wait(&bar[warp], phase ^ 1u, a.status);  // drain before the buffer is reused
+      __syncwarp();
+      return;
+    }
+    // logits of the pair's members
+    float lge = -INFINITY;
+    bool ev = false;
+#pragma unroll 1
+    for (int x = 0; x < npg; ++x) {
+      const int n = x == 0 ? na : nb;
+      const float2* kq = reinterpret_cast<const float2*>(stg + (4 + x) * PB);
+      const uint8_t* kc = stg + x * PB;
+      float qsc[DPL], qlo = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const float2 z = kq[lane * DPL + i];
+        qsc[i] = qd[i] * z.x;
+        qlo = fmaf(qd[i], z.y, qlo);
+      }
+      qlo = warp_sum(qlo);
+      float part[kPage];
+#pragma unroll
+      for (int r = 0; r < kPage; ++r) {
+        part[r] = 0.f;
+        if (r < n) {
+          const uint32_t w = lane_codes<D, DPL>(kc + r * (D / 2), lane);
+          float sdot = 0.f;
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) sdot = fmaf(qsc[i], nibble_f(w, i), sdot);
+          part[r] = sdot;
+        }
+      }
+      const float tot = transpose_sum16(part, lane) + qlo;  // member lane >> 1
+      const float v = __shfl_sync(0xffffffffu, tot, (2 * (lane & 15)) & 31);
+      if ((lane >> 4) == x && (lane & 15) < n) {
+        lge = v;
+        ev = true;
+      }
+    }
+    const float lgcb = cvb ? lgc : -INFINITY;
+    const float bm = warp_max(fmaxf(lge, lgcb));
+    const float mn = fmaxf(m, bm);
+    const float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    const float pe = ev ? __expf(lge - mn) : 0.f;
+    const float pc = cvb ? __expf(lgcb - mn) : 0.f;
+    l = l * corr + warp_sum(pe + pc);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] *= corr;
+    m = mn;
+    mysc[lane] = pe;  // member r of page x at 16 x + r
+    __syncwarp();
+#pragma unroll 1
+    for (int x = 0; x < npg; ++x) {
+      const int n = x == 0 ? na : nb;
+      const float2* vq = reinterpret_cast<const float2*>(stg + (6 + x) * PB);
+      const uint8_t* vc = stg + (2 + x) * PB;
+      float ac[DPL], ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) ac[i] = 0.f;
+#pragma unroll
+      for (int r = 0; r < kPage; ++r) {
+        if (r < n) {
+          const float pr = mysc[16 * x + r];
+          const uint32_t w = lane_codes<D, DPL>(vc + r * (D / 2), lane);
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) ac[i] = fmaf(pr, nibble_f(w, i), ac[i]);
+          ps += pr;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const float2 z = vq[lane * DPL + i];
+        acc[i] = fmaf(z.x, ac[i], fmaf(z.y, ps, acc[i]));
+      }
+    }
+    // coarse entries, in lane order
+    unsigned rest = cmb;
+    while (rest) {
+      const int jc = __ffs((int)rest) - 1;
+      rest &= rest - 1;
+      const float pj = __shfl_sync(0xffffffffu, pc, jc);
+      float v[DPL];
+      lds_f<T, DPL>(myV + (32 + jc) * D + lane * DPL, v);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, v[i], acc[i]);
+    }
+    __syncwarp();
+  };
   // the sink tokens (last warp)
   if (warp == kWarps - 1) {
     for (int64_t e0 = 0; e0 < nsk; e0 += 32)
@@ -1133,6 +1298,42 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       const bool okrun = gcnt > 0 && gcnt <= kChunk && b0 >= 0 && b0 + gcnt <= kChunk;
       if (whole && !okrun && lane == 0) set_status(a.status, LOD_ST_BAD_MEMBER);
       const int nbatch = whole ? (okrun ? (gcnt + 31) / 32 : 0) : (nopen * kPage + 31) / 32;
+      if constexpr (Q4) {  // three-tier INT4: the opened pages two per batch
+        const int npair = (nopen + 1) / 2;
+        for (int bt = 0; bt < (npair > 0 ? npair : 1); ++bt) {
+          int sa = -1, sb = -1;
+#pragma unroll
+          for (int y = 0; y < kMaxTopPages; ++y) {
+            if (y == 2 * bt) sa = open_slot[y];
+            if (y == 2 * bt + 1) sb = open_slot[y];
+          }
+          int na = __shfl_sync(0xffffffffu, cntp, (sa - p0) & 31);
+          int ba = __shfl_sync(0xffffffffu, begp, (sa - p0) & 31);
+          int nb = __shfl_sync(0xffffffffu, cntp, (sb - p0) & 31);
+          int bb = __shfl_sync(0xffffffffu, begp, (sb - p0) & 31);
+          if (sa < 0) na = 0;
+          if (sb < 0) nb = 0;
+          if (na > kPage || nb > kPage) {
+            if (lane == 0) set_status(a.status, LOD_ST_BAD_PAGE);
+            if (na > kPage) na = 0;
+            if (nb > kPage) nb = 0;
+          }
+          if ((na > 0 && (ba < 0 || ba + na > kChunk)) || (nb > 0 && (bb < 0 || bb + nb > kChunk))) {
+            if (lane == 0) set_status(a.status, LOD_ST_BAD_MEMBER);
+            if (na > 0 && (ba < 0 || ba + na > kChunk)) na = 0;
+            if (nb > 0 && (bb < 0 || bb + nb > kChunk)) nb = 0;
+          }
+          if (na <= 0) {  // pack a lone page into the first place
+            na = nb;
+            ba = bb;
+            sa = sb;
+            nb = 0;
+          }
+          const int npg = (na > 0 ? 1 : 0) + (nb > 0 ? 1 : 0);
+          batch_q(npg, c * kChunk + ba, na, c * a.P + sa, c * kChunk + bb, nb, c * a.P + sb, bt == 0 && cv, lgc,
+                  pV + (c * a.P + p0 + lane) * D);
+        }
+      } else
       for (int bt = 0; bt < (nbatch > 0 ? nbatch : 1); ++bt) {
         const int e = bt * 32 + lane;
         const int x = e / kPage, mi = e % kPage;
@@ -1240,9 +1441,10 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
     if (e != cudaSuccess) return e;
   }
   if (rows > 0) {
-    auto rk = refine_kernel<T, D, NQ>;
+    const bool q4 = a.kv_bits == 4;
+    auto rk = q4 ? refine_kernel<T, D, NQ, true> : refine_kernel<T, D, NQ, false>;
     const size_t smem = RefineSmem<T, D>::bytes;
-    e = set_smem_once<refine_kernel<T, D, NQ>>(smem);
+    e = q4 ? set_smem_once<refine_kernel<T, D, NQ, true>>(smem) : set_smem_once<refine_kernel<T, D, NQ, false>>(smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows);

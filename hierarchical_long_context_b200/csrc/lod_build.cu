@@ -81,6 +81,53 @@ __device__ __forceinline__ float2 pair_of(const uint32_t* w, int p) {
   }
 }
 
+// Three-tier INT4 ("Level of Detail Attention", the paragraph after the
+// quality tables: INT4 KV storage, only the selected pages decompressed):
+// one page's members as 4-bit codes of a per-channel asymmetric quantiser.
+// Lane `lane` owns channels [lane * DPL, lane * DPL + DPL); get(r, i) is
+// member r's value in the lane's channel i.  Per channel: low = min, scale =
+// (max - low) / 15, code = clamp(rint((x - low) / scale), 0, 15) (0 when
+// scale = 0), all in IEEE fp32.  codes: the page's first member-ordered row
+// (d/2 bytes per row, channel 2i in the low nibble); qs: (scale, low) per
+// channel of the page slot.
+template <int D, int DPL, typename Get>
+__device__ __forceinline__ void quantize_page(int pc, Get get, uint8_t* codes, float2* qs, int lane) {
+  float lo[DPL], sc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kPage; ++r) {
+      if (r < pc) {
+        const float x = get(r, i);
+        if (x < mn) mn = x;
+        if (x > mx) mx = x;
+      }
+    }
+    lo[i] = mn;
+    sc[i] = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    qs[lane * DPL + i] = make_float2(sc[i], lo[i]);
+  }
+#pragma unroll
+  for (int r = 0; r < kPage; ++r) {
+    if (r >= pc) break;
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      float v = sc[i] > 0.0f ? rintf(__fdiv_rn(__fsub_rn(get(r, i), lo[i]), sc[i])) : 0.0f;
+      v = fminf(fmaxf(v, 0.0f), 15.0f);
+      w |= (uint32_t)v << (4 * i);
+    }
+    uint8_t* dst = codes + (int64_t)r * (D / 2) + lane * (DPL / 2);
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
+    } else {
+      static_assert(DPL == 2, "channels per lane");
+      *dst = (uint8_t)w;
+    }
+  }
+}
+
 template <typename T, int D, int KMAX>
 struct BuildSmem {
   static constexpr int PMAX = kChunk / kPage + KMAX;  // page slots per chunk
@@ -376,11 +423,20 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
       pV[pg * D + lane * DPL + i] = Elem<T>::from_f(sv[i] / (float)pc);
       psum[pg * D + lane * DPL + i] = sv[i];
     }
+    if (a.kv_bits == 4) {  // three-tier INT4: the page's members as 4-bit codes
+      const int64_t mrow = (unit * a.Cmax + c) * kChunk + m0;  // member-ordered row of the first member
+      const int64_t prow = (unit * a.Cmax + c) * P + pg;       // page slot
+      quantize_page<D, DPL>(
+          pc, [&](int r, int i) { return xval(first + perm_s[m0 + r], lane * DPL + i); },
+          a.qK + mrow * (D / 2), a.qKs + prow * D, lane);
+      quantize_page<D, DPL>(pc, [&](int r, int i) { return vv[r][i]; }, a.qV + mrow * (D / 2),
+                            a.qVs + prow * D, lane);
+    }
   }
   // member-ordered copies: row m = the token at chunk offset perm[m], so each
   // page's members are consecutive rows (keys from shared memory, values
-  // from the rows the page sums just read)
-  {
+  // from the rows the page sums just read); three-tier INT4 keeps codes instead
+  if (a.kv_bits != 4) {
     constexpr int C16 = ROWB / 16;  // 16-byte pieces per row
     uint4* mKc = reinterpret_cast<uint4*>(static_cast<T*>(a.mK) + ((unit * a.Cmax + c) * kChunk) * D);
     uint4* mVc = reinterpret_cast<uint4*>(static_cast<T*>(a.mV) + ((unit * a.Cmax + c) * kChunk) * D);
@@ -396,6 +452,11 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
     const int slot = used + item / D, i = item % D;
     pK[slot * D + i] = Elem<T>::from_f(0.f);
     pV[slot * D + i] = Elem<T>::from_f(0.f);
+    if (a.kv_bits == 4) {
+      const int64_t q = ((unit * a.Cmax + c) * P + slot) * D + i;
+      a.qKs[q] = make_float2(0.f, 0.f);
+      a.qVs[q] = make_float2(0.f, 0.f);
+    }
   }
   __syncthreads();
   // group means: key = the final centroid; value = its pages' sums in page order

@@ -35,6 +35,11 @@ struct BuildArgs {
   void* mK;            // member-ordered key / value copies
   void* mV;
   int32_t* gMeta;      // size | first page << 16 | end page << 24 per group
+  int kv_bits;         // 4: three-tier INT4 (qK/qV codes + qKs/qVs quantisers instead of mK/mV)
+  uint8_t* qK;         // [..][Cmax * chunk][d / 2] member-ordered 4-bit codes
+  uint8_t* qV;
+  float2* qKs;         // [..][Cmax * P][d] (scale, low) per page slot and channel
+  float2* qVs;
   uint32_t* status;    // device status word (workspace header)
 };
 
@@ -106,6 +111,11 @@ struct AttendArgs {
   const void* mK;           // member-ordered key / value copies [..][Cmax * chunk][d]
   const void* mV;
   const int32_t* gMeta;     // size | first page << 16 | end page << 24 per group
+  int kv_bits;              // 4: opened pages read from the INT4 codes below
+  const uint8_t* qK;        // [..][Cmax * chunk][d / 2] member-ordered 4-bit codes
+  const uint8_t* qV;
+  const float2* qKs;        // [..][Cmax * P][d] (scale, low) per page slot and channel
+  const float2* qVs;
   int B, Hq, Hkv, g;
   int64_t Tmax, Cmax;
   int k, P, G, TP, window, sinks;

@@ -65,7 +65,10 @@ def decode_touched_bytes(p, index, seq_lens, sel_groups, sel_pages) -> int:
                         total += row
             for pid in opened:
                 n = int(pCnt[b, h, pid])
-                total += n * 2 * row  # K and V rows (one contiguous run per page)
+                if p.kv_bits == 4:  # three-tier INT4: K and V codes + (scale, low) quantisers
+                    total += n * 2 * (d // 2) + 2 * d * 8
+                else:
+                    total += n * 2 * row  # K and V rows (one contiguous run per page)
     return total
 
 

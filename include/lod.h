@@ -71,7 +71,13 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
  * whole with no page tier); window a positive multiple of chunk (the
  * page says 256-512); 0 <= sinks < chunk; Hq a multiple of Hkv with
  * Hq/Hkv a power of two no larger than 8; Tmax a positive multiple of chunk.
- * scale <= 0 selects 1/sqrt(d).
+ * scale <= 0 selects 1/sqrt(d).  kv_bits 0 or 4: 4 is the pages' three-tier
+ * INT4 mode ("Level of Detail Attention", the paragraph after the quality
+ * tables: INT4 KV storage, only the selected pages decompressed), where the
+ * members of every indexed page are kept as 4-bit codes of a per-page,
+ * per-channel quantiser (see lod_index) and an opened page is read from
+ * them; it needs top_pages >= 1.  The summaries, the sinks and the window
+ * always use the cache dtype.
  */
 typedef struct lod_params {
   int32_t dtype;        /* lod_dtype */
@@ -87,7 +93,7 @@ typedef struct lod_params {
   int32_t top_pages;    /* pages opened per opened group: 2; 0 = every page (two-tier LoD) */
   int32_t window;       /* sliding window in tokens (block granular) */
   int32_t sinks;        /* sink tokens at positions [0, sinks) */
-  int32_t reserved0;    /* must be 0 */
+  int32_t kv_bits;      /* 0: opened pages read in the cache dtype; 4: three-tier INT4 */
   uint64_t seed;        /* k-means initialisation seed */
   float scale;          /* softmax scale on q.k; <= 0 means 1/sqrt(d) */
   int32_t reserved1;    /* must be 0 */
@@ -114,6 +120,16 @@ typedef struct lod_params {
  *                         last member are not written)
  *   gMeta   [Cmax*k]      int32 gCnt and gPage of a group in one word:
  *                         size | first page slot << 16 | end page slot << 24
+ *   qK, qV  [Cmax*chunk][d/2] uint8, kv_bits = 4 only: the member-ordered
+ *                         keys / values as 4-bit codes, two per byte
+ *                         (channel 2i in the low nibble, 2i+1 in the high)
+ *   qKs, qVs [Cmax*P][d][2] float, kv_bits = 4 only: per page slot and
+ *                         channel the quantiser (scale, low) over the page's
+ *                         members: low = min, scale = (max - low) / 15,
+ *                         code = clamp(rint((x - low) / scale), 0, 15) (0 when
+ *                         scale = 0); a member reads fmaf(code, scale, low)
+ * With kv_bits = 4 the member copies mK, mV are unused (size 0, may be NULL);
+ * with kv_bits = 0 the four INT4 arrays are unused (size 0, may be NULL).
  * Every array is laid out [B][Hkv][...] in that order.  gK, gV, pK, pV, perm,
  * mK and mV must be 16-byte aligned, gCnt, pCnt and gMeta 4-byte aligned.
  */
@@ -130,6 +146,10 @@ typedef struct lod_index {
   void* mK;
   void* mV;
   int32_t* gMeta;
+  uint8_t* qK;
+  uint8_t* qV;
+  float* qKs;
+  float* qVs;
 } lod_index;
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -139,11 +159,12 @@ int32_t lod_version(void);
 const char* lod_last_error(void);
 
 /*
- * Byte sizes of the twelve lod_index arrays, in field order (gK, gV, gCnt,
- * pK, pV, pCnt, pBeg, gPage, perm, mK, mV, gMeta), written to bytes[0..11]
- * (host).  Validates `p` like every other entry point.
+ * Byte sizes of the sixteen lod_index arrays, in field order (gK, gV, gCnt,
+ * pK, pV, pCnt, pBeg, gPage, perm, mK, mV, gMeta, qK, qV, qKs, qVs), written
+ * to bytes[0..15] (host); an array the parameters do not use has size 0.
+ * Validates `p` like every other entry point.
  */
-#define LOD_INDEX_ARRAYS 12
+#define LOD_INDEX_ARRAYS 16
 int32_t lod_index_sizes(const lod_params* p, size_t bytes[LOD_INDEX_ARRAYS]);
 
 /*

@@ -64,10 +64,49 @@ def pack_meta(u: dict, k: int) -> np.ndarray:
     return (cnt | (gp[:, :k] << 16) | (gp[:, 1:] << 24)).reshape(-1).astype(np.int32)
 
 
+def pack_codes(code: np.ndarray) -> np.ndarray:
+    """[rows, d] 4-bit codes -> [rows, d/2] bytes (channel 2i in the low nibble)."""
+    code = np.asarray(code, np.uint8)
+    return (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_codes."""
+    packed = np.asarray(packed, np.uint8)
+    out = np.empty((packed.shape[0], packed.shape[1] * 2), np.uint8)
+    out[:, 0::2] = packed & 15
+    out[:, 1::2] = packed >> 4
+    return out
+
+
+def quantized(u: dict, K: np.ndarray, V: np.ndarray, cfg: oracle.Config) -> dict:
+    """u with the oracle's three-tier INT4 pages of K and V added (kq, vq)."""
+    return dict(u, kq=oracle.quantize_pages(cfg, K, u), vq=oracle.quantize_pages(cfg, V, u))
+
+
+def check_int4_pages(ix: api.Index, b: int, h: int, u: dict, K: np.ndarray, V: np.ndarray,
+                     cfg: oracle.Config) -> int:
+    """The GPU's INT4 codes and (scale, low) quantisers equal the oracle's
+    quantiser applied to the GPU-built index, bit for bit (every member row,
+    every used page slot).  Returns the number of member rows compared."""
+    n, C, P = u["nchunks"], cfg.chunk, cfg.page_slots
+    used = u["pCnt"][:n * P] > 0
+    members = u["perm"][:n * C] >= 0
+    for X, codes, qs in ((K, ix.qK, ix.qKs), (V, ix.qV, ix.qVs)):
+        oq = oracle.quantize_pages(cfg, X, u)
+        gq = qs[b, h, :n * P].cpu().numpy()
+        np.testing.assert_array_equal(gq[used][..., 0], oq["scale"][used])
+        np.testing.assert_array_equal(gq[used][..., 1], oq["low"][used])
+        gc = unpack_codes(codes[b, h, :n * C].cpu().numpy())
+        np.testing.assert_array_equal(gc[members], oq["code"][members])
+    return int(members.sum())
+
+
 def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params, K=None, V=None) -> None:
     """Write an oracle-built index of one sequence into a GPU index.  K, V
     (that sequence's cache rows, [T][d] tensors) fill the member-ordered
-    copies: row m of chunk c is the token at offset perm[m]."""
+    copies: row m of chunk c is the token at offset perm[m]; with
+    p.kv_bits = 4, u's INT4 pages (kq, vq of `quantized`) fill the codes."""
     n = u["nchunks"]
     k, P, C = p.clusters, p.page_slots, p.chunk
     dev = ix.gK.device
@@ -82,7 +121,13 @@ def unit_to_gpu(ix: api.Index, b: int, h: int, u: dict, p: api.Params, K=None, V
     put(ix.gPage, u["gPage"], n * (k + 1))
     put(ix.perm, u["perm"], n * C)
     put(ix.gMeta, pack_meta(u, k), n * k)
-    if K is not None:
+    if p.kv_bits == 4:
+        for key, codes, qs in (("kq", ix.qK, ix.qKs), ("vq", ix.qV, ix.qVs)):
+            q = u[key]
+            codes[b, h, :n * C].copy_(torch.from_numpy(pack_codes(q["code"][:n * C])).to(dev))
+            sl = np.stack([q["scale"][:n * P], q["low"][:n * P]], -1).astype(np.float32)
+            qs[b, h, :n * P].copy_(torch.from_numpy(np.ascontiguousarray(sl)).to(dev))
+    elif K is not None:
         perm = torch.from_numpy(np.asarray(u["perm"][:n * C], dtype=np.int64))
         rows = torch.arange(n * C) // C * C + perm
         ok = perm >= 0
@@ -192,13 +237,16 @@ def compare_builds(gu: dict, ou: dict, cfg: oracle.Config, bf16: bool) -> dict:
 def check_rows(cfg: oracle.Config, dtype: str, K: np.ndarray, V: np.ndarray, u: dict, rows,
                threads: int = 8) -> dict:
     """rows: list of (q[d] float32, t, gpu_out[d], gpu_lse, gpu_sel_groups, gpu_sel_pages).
-    Checks selection (tie rule) and output against the oracle on index u."""
+    Checks selection (tie rule) and output against the oracle on index u
+    (three-tier INT4 when u carries the pages' codes, see `quantized`)."""
     tol = TOL[dtype]
     sc = np.float32(cfg.scale if cfg.scale > 0 else 1.0 / np.sqrt(cfg.d))
 
+    qk = dict(kq=u["kq"], vq=u["vq"]) if "kq" in u else {}
+
     def one(row):
         q, t, gout, glse, gsg, gsp = row
-        out, lse, sg, sp, st = oracle.attend_row(cfg, q, t, K, V, u)
+        out, lse, sg, sp, st = oracle.attend_row(cfg, q, t, K, V, u, **qk)
         forced = False
         if not (np.array_equal(np.sort(sg), np.sort(gsg))):
             # differing opened groups must be score ties within TIE
@@ -220,7 +268,7 @@ def check_rows(cfg: oracle.Config, dtype: str, K: np.ndarray, V: np.ndarray, u: 
                     assert max(abs(s(x) - s(y)) for x in a - b for y in b - a) <= TIE
                     forced = True
         if forced:
-            out, lse, *_ = oracle.attend_row(cfg, q, t, K, V, u, gsg, gsp)
+            out, lse, *_ = oracle.attend_row(cfg, q, t, K, V, u, gsg, gsp, **qk)
         err = float(np.max(np.abs(out - gout)))
         assert err <= tol, "t=%d max-abs %.3g > %g" % (t, err, tol)
         lerr = abs(lse - glse)

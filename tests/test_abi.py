@@ -53,7 +53,23 @@ def test_index_sizes_match_the_documented_layout():
     u = 2 * 2
     assert s == [u * Cmax * k * 128 * 2] * 2 + [u * Cmax * k * 4] + [u * Cmax * Pp * 128 * 2] * 2 + \
         [u * Cmax * Pp * 4, u * Cmax * Pp * 2, u * Cmax * (k + 1) * 2, u * Cmax * 256 * 2] + \
-        [u * Cmax * 256 * 128 * 2] * 2 + [u * Cmax * k * 4]
+        [u * Cmax * 256 * 128 * 2] * 2 + [u * Cmax * k * 4] + [0] * 4
+
+
+def test_int4_index_sizes_replace_the_member_copies():
+    p = P(kv_bits=4)
+    rc, s = _sizes(p)
+    assert rc == 0
+    Cmax, Pp, u = 4096 // 256, 256 // 16 + 4, 2 * 2
+    assert s[9] == s[10] == 0
+    assert s[12] == s[13] == u * Cmax * 256 * 128 // 2
+    assert s[14] == s[15] == u * Cmax * Pp * 128 * 2 * 4
+
+
+@pytest.mark.parametrize("kw", [dict(kv_bits=8), dict(kv_bits=4, top_pages=0)])
+def test_unsupported_int4_settings(kw):
+    rc, _ = _sizes(P(**kw))
+    assert rc == _lib.LOD_EUNSUPPORTED
 
 
 @pytest.mark.parametrize("kw, code", [
@@ -127,7 +143,7 @@ def test_null_and_misaligned_pointers_fail_before_any_launch():
 
 def test_reserved_fields_must_be_zero():
     p = P().c()
-    p.reserved0 = 1
+    p.reserved1 = 1
     sizes = (ctypes.c_size_t * len(_lib.INDEX_FIELDS))()
     assert _lib.load().lod_index_sizes(ctypes.byref(p), sizes) == _lib.LOD_EINVAL
 
@@ -138,4 +154,5 @@ def test_struct_layout_matches_the_header():
     assert _lib.lod_params.scale.offset == 64
     assert _lib.lod_params.Tmax.offset == 72
     assert ctypes.sizeof(_lib.lod_params) == 80
-    assert ctypes.sizeof(_lib.lod_index) == 8 * 12
+    assert _lib.lod_params.kv_bits.offset == 52
+    assert ctypes.sizeof(_lib.lod_index) == 8 * 16

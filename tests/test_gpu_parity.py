@@ -21,11 +21,11 @@ def _cuda():
     return torch.device("cuda")
 
 
-def _setup(w, k=None, T=None):
+def _setup(w, k=None, T=None, **pkw):
     dev = _cuda()
     T = T or w.T
     Kc, Vc = synth.kv_cache(w, T)
-    p = lt.params_of(w, k, Tmax=((T + 255) // 256) * 256)
+    p = lt.params_of(w, k, Tmax=((T + 255) // 256) * 256, **pkw)
     Kd = torch.zeros((w.B, w.Hkv, p.Tmax, w.d), dtype=w.torch_dtype, device=dev)
     Vd = torch.zeros_like(Kd)
     Kd[:, :, :T] = Kc.to(dev)
@@ -160,6 +160,82 @@ def test_decode_on_oracle_index_matches_oracle():
         for h in range(w.Hkv):
             ous[(b, h)] = oracle.build_sequence(cfg, b * w.Hkv + h, _np(Kc[b, h]), _np(Vc[b, h]), T // 256)
             lt.unit_to_gpu(ix, b, h, ous[(b, h)], p, Kd[b, h], Vd[b, h])
+    rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 300], draws=4)
+    st = _check_decode(w, p, Kc, Vc, ix, rows, cfg, lambda b, h, K, V, n: ous[(b, h)])
+    print(st)
+
+
+# ------------------------------------------------------------------ three-tier INT4
+
+@pytest.mark.parametrize("name, k, T, kw", [
+    ("decode_gqa_32k_bf16", 4, 4096, {}),
+    ("decode_gqa_32k_bf16", 8, 2048, dict(d=64)),
+    ("decode_tiny_f32", 4, 4096, {}),
+])
+def test_int4_build_matches_oracle(name, k, T, kw):
+    """Three-tier INT4 build: the codes and per-page quantisers equal the
+    oracle's quantiser on the GPU-built index bit for bit; the summaries
+    follow the same rules as the cache-dtype build."""
+    w = synth.WORKLOADS[name].with_(**kw)
+    w = w.with_(B=min(w.B, 2), Hkv=min(w.Hkv, 2), Hq=min(w.Hkv, 2) * w.g)
+    p, Kc, Vc, Kd, Vd = _setup(w, k, T, kv_bits=4)
+    ix = api.Index(p)
+    assert ix.mK.numel() == 0 and ix.qK.numel() > 0
+    nch = T // 256
+    api.lod_build_index(p, Kd, Vd, 0, nch, ix)
+    torch.cuda.synchronize()
+    cfg = lt.oracle_cfg(w, k)
+    rows = 0
+    tot = dict(chunks=0, fragile=0, diverged=0, keys_checked=0)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            K, V = _np(Kc[b, h]), _np(Vc[b, h])
+            gu = lt.unit_from_gpu(ix, b, h, nch, p)
+            lt.check_index_consistency(gu, K, V, cfg, w.dtype == "bf16")
+            rows += lt.check_int4_pages(ix, b, h, gu, K, V, cfg)
+            ou = oracle.build_sequence(cfg, b * w.Hkv + h, K, V, nch)
+            st = lt.compare_builds(gu, ou, cfg, w.dtype == "bf16")
+            for key in tot:
+                tot[key] += st[key]
+    print(name, k, kw, rows, tot)
+    assert rows > 0.9 * w.B * w.Hkv * nch * 256
+    assert tot["diverged"] <= max(1, tot["chunks"] // 20)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),                                        # bf16 d=128, g=8 (tensor-core scan), two pages a group
+    dict(Hq=4, Hkv=2, top_pages=4, top_groups=16),  # two page pairs a group, g=2
+    dict(d=64, Hq=2, Hkv=2, top_pages=1),           # one page a group, CUDA-core scan, MHA
+    dict(dtype="f32", Hq=8, Hkv=2),                 # fp32 cache
+])
+def test_int4_decode_matches_oracle(kw):
+    """Three-tier INT4 decode on the GPU-built index against the oracle
+    reading the same pages decompressed."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, T=4096, Hq=16, Hkv=2).with_(**kw)
+    T = 4096
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T, kv_bits=4)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 777], draws=2)
+    cfg = lt.oracle_cfg(w)
+    st = _check_decode(w, p, Kc, Vc, ix, rows, cfg,
+                       lambda b, h, K, V, n: lt.quantized(lt.unit_from_gpu(ix, b, h, T // 256, p), K, V, cfg))
+    print(kw, st)
+
+
+def test_int4_decode_on_oracle_index_matches_oracle():
+    """The INT4 attention kernels alone: index and codes are the oracle's."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, Hkv=2, Hq=16)
+    T = 6144
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T, kv_bits=4)
+    cfg = lt.oracle_cfg(w)
+    ix = api.Index(p)
+    ous = {}
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            K, V = _np(Kc[b, h]), _np(Vc[b, h])
+            ous[(b, h)] = lt.quantized(oracle.build_sequence(cfg, b * w.Hkv + h, K, V, T // 256), K, V, cfg)
+            lt.unit_to_gpu(ix, b, h, ous[(b, h)], p)
     rows = _decode_rows(p, w, Kd, Vd, ix, [T, T - 300], draws=4)
     st = _check_decode(w, p, Kc, Vc, ix, rows, cfg, lambda b, h, K, V, n: ous[(b, h)])
     print(st)
