@@ -517,11 +517,15 @@ def main():
     ap.add_argument("--graphs", type=int, default=1, help="e2e: one CUDA graph per step (0 = eager)")
     ap.add_argument("--replicas", type=int, default=4,
                     help="decode: device replicas of the inputs used in rotation (1 = flush L2 instead)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per step (0 = the workload's own; smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     from hierarchical_long_context_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.batch > 0:
+        w = w.with_(B=args.batch)
     world, rank, local = dist_setup(args) if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     if args.impl == "reference":
