@@ -137,6 +137,22 @@ def lod_build_index(params: Params, K, V, chunk_begin: int, chunk_end: int, inde
         ctypes.byref(index.c()), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def lod_build_ready(params: Params, K, V, seq_lens, index: Index, ws=None, stream=None) -> None:
+    """Online build: for every sequence whose length (seq_lens, device int64
+    [B]) is a positive multiple of the chunk, build the chunk it just
+    completed; the decision is taken on the device, so this can be issued
+    every decode step, e.g. on a second stream."""
+    lib = load()
+    st = _kv_strides(params, K, V)
+    if seq_lens.shape != (params.B,) or seq_lens.dtype != torch.int64 or seq_lens.device != K.device:
+        raise ValueError("seq_lens must be int64 [B] on the cache's device")
+    if ws is None:
+        ws = workspace(params, _lib.LOD_OP_BUILD, K.device)
+    check("lod_build_ready", lib.lod_build_ready(
+        ctypes.byref(params.c()), _ptr(K), _ptr(V), st, _ptr(seq_lens), ctypes.byref(index.c()),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def lod_decode(params: Params, q, K, V, seq_lens, index: Index, out=None, lse=None, sel_groups=None,
                sel_pages=None, ws=None, stream=None):
     """One decode step: q [B, Hq, d] at positions seq_lens - 1.  Returns out."""

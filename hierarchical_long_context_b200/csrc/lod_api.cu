@@ -253,7 +253,8 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
-                 int64_t c1, const lod_index* ix, void* ws, cudaStream_t stream) {
+                 int64_t c1, const lod_index* ix, void* ws, cudaStream_t stream,
+                 const int64_t* seq_lens = nullptr) {
   lod::BuildArgs a;
   memset(&a, 0, sizeof(a));
   a.K = K;
@@ -268,6 +269,7 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.sinks = p->sinks;
   a.P = page_slots(p);
   a.chunk_begin = c0;
+  a.seq_lens = seq_lens;
   a.seed = p->seed;
   a.gK = ix->gK;
   a.gV = ix->gV;
@@ -350,6 +352,21 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V, const
   if (!ws || !aligned16(ws) || ws_bytes < lod::kWsHeader)
     return fail(LOD_EINVAL, "workspace too small or misaligned");
   rc = do_build(p, K, V, kv_strides, chunk_begin, chunk_end, index, ws, (cudaStream_t)stream);
+  if (!rc) g_err[0] = 0;
+  return rc;
+}
+
+int32_t lod_build_ready(const lod_params* p, const void* K, const void* V, const int64_t kv_strides[3],
+                        const int64_t* seq_lens, const lod_index* index, void* ws, size_t ws_bytes,
+                        lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (!rc) rc = validate_index(p, index);
+  if (rc) return rc;
+  if (!seq_lens) return fail(LOD_EINVAL, "seq_lens must be non-NULL");
+  if (!ws || !aligned16(ws) || ws_bytes < lod::kWsHeader)
+    return fail(LOD_EINVAL, "workspace too small or misaligned");
+  rc = do_build(p, K, V, kv_strides, 0, 1, index, ws, (cudaStream_t)stream, seq_lens);
   if (!rc) g_err[0] = 0;
   return rc;
 }

@@ -154,8 +154,14 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
   constexpr int NP = D / 2;                      // dimension pairs
   using SM = BuildSmem<T, D, KMAX>;
   constexpr int PMAX = SM::PMAX;
-  const int64_t c = a.chunk_begin + blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
+  int64_t cc = a.chunk_begin + blockIdx.x;
+  if (a.seq_lens) {  // online build: the chunk sequence b's length has just completed, if any
+    const int64_t L = a.seq_lens[b];
+    if (L < kChunk || L % kChunk != 0 || L / kChunk > a.Cmax) return;
+    cc = L / kChunk - 1;
+  }
+  const int64_t c = cc;
   const int64_t unit = (int64_t)b * a.Hkv + h;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int first = (c == 0) ? a.sinks : 0;  // sink positions are never clustered

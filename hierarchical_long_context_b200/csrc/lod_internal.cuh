@@ -22,6 +22,7 @@ struct BuildArgs {
   int sinks;
   int P;               // page slots per chunk
   int64_t chunk_begin;
+  const int64_t* seq_lens;  // non-null: per sequence, the chunk its length just completed (else nothing)
   uint64_t seed;
   void* gK;
   void* gV;

@@ -198,6 +198,24 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V,
                         const lod_index* index, void* ws, size_t ws_bytes, lod_stream_t stream);
 
 /*
+ * Online index build for decode ("How It Works", paragraph 1: the index is
+ * built as inference proceeds, after every chunk of 256 tokens): for every
+ * sequence b whose length seq_lens[b] (device [B] int64) is a positive
+ * multiple of chunk, builds the chunk that length has just completed,
+ * [seq_lens[b] - chunk, seq_lens[b]), for all KV heads, exactly as
+ * lod_build_index would; other sequences are left alone.  The decision is
+ * taken on the device, so the call can be issued every decode step (or every
+ * step of a captured graph) on a second stream, concurrently with
+ * lod_decode: a chunk completed at length L is first visible to a query at
+ * position >= L - chunk + window (the block window), i.e. window - chunk
+ * steps later, and the build must be ordered before that decode.  ws as for
+ * lod_build_index.  Same errors as lod_build_index.
+ */
+int32_t lod_build_ready(const lod_params* p, const void* K, const void* V,
+                        const int64_t kv_strides[3], const int64_t* seq_lens, const lod_index* index,
+                        void* ws, size_t ws_bytes, lod_stream_t stream);
+
+/*
  * LoD decode ("How It Works", paragraphs 2-3): one query per sequence b at
  * position t = seq_lens[b] - 1 (the current token's K/V is already in the
  * cache).  The exact window is [chunk * max(0, t/chunk - window/chunk + 1), t],

@@ -241,6 +241,53 @@ def test_int4_decode_on_oracle_index_matches_oracle():
     print(st)
 
 
+# ------------------------------------------------------------------ online build
+
+def test_online_build_during_decode_matches_bulk_build():
+    """The index built online -- lod_build_ready issued every decode step on a
+    second stream, concurrently with lod_decode -- equals the bulk build bit
+    for bit, and the decodes of those steps equal decodes on the bulk-built
+    index (the chunk being built is not yet visible to them)."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=4, Hkv=2, Hq=16)
+    T = 4096
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    dev = Kd.device
+    L0 = [2045, 2041, 2047, 1900]   # three sequences complete chunk 7 at different steps
+    steps = 12
+    ix_on, ix_bulk = api.Index(p), api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, 7, ix_on)
+    api.lod_build_index(p, Kd, Vd, 0, 8, ix_bulk)
+    ws_b = api.workspace(p, api._lib.LOD_OP_BUILD)
+    ws_d = api.workspace(p, api._lib.LOD_OP_DECODE)
+    ws_r = api.workspace(p, api._lib.LOD_OP_DECODE)
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    outs_on, outs_ref = [], []
+    for s in range(steps):
+        sl = torch.tensor([x + s + 1 for x in L0], dtype=torch.int64, device=dev)
+        q = synth.decode_queries(w, stream="queries%d" % s).to(dev)
+        side.wait_stream(main)             # the step's inputs (lengths) are ready
+        api.lod_build_ready(p, Kd, Vd, sl, ix_on, ws=ws_b, stream=side)
+        outs_on.append(api.lod_decode(p, q, Kd, Vd, sl, ix_on, ws=ws_d))
+        outs_ref.append(api.lod_decode(p, q, Kd, Vd, sl, ix_bulk, ws=ws_r))
+        sl.record_stream(side)
+    main.wait_stream(side)
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws_d) == 0 and api.lod_get_status(ws_b) == 0
+    for a, b in zip(outs_on, outs_ref):
+        assert torch.equal(a, b)
+    k, P, C = p.clusters, p.page_slots, p.chunk
+    fresh = api.Index(p)
+    per = {"gK": k, "gV": k, "gCnt": k, "pK": P, "pV": P, "pCnt": P, "pBeg": P, "gPage": k + 1,
+           "perm": C, "mK": C, "mV": C, "gMeta": k}
+    for f, n in per.items():
+        on, bulk = getattr(ix_on, f), getattr(ix_bulk, f)
+        for b in range(w.B):
+            built = 8 if b < 3 else 7        # sequence 3 never reaches 2048 tokens
+            assert torch.equal(on[b, :, :built * n], bulk[b, :, :built * n]), (f, b)
+            if b == 3:                        # its chunk 7 is untouched
+                assert torch.equal(on[b, :, 7 * n:8 * n], getattr(fresh, f)[b, :, 7 * n:8 * n]), f
+
+
 def test_zero_variance_decode_equals_dense():
     """Level of Detail Attention, How It Works: zero-variance groups give full
     attention -- checked on the GPU path directly against dense softmax."""
