@@ -199,10 +199,11 @@ def dist_setup(args):
     return world, rank, local
 
 
-def dist_max(x: float, world: int) -> float:
+def dist_max(x: float, world: int, device: str = "cuda") -> float:
+    """Max of x over the ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -220,11 +221,13 @@ def params_for(w, k=None, kv_bits=0):
     return api.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, Tmax=((w.T + 255) // 256) * 256,
                       dtype=w.torch_dtype, clusters=k or w.clusters[0], kmeans_iters=w.iters,
                       top_groups=w.top_groups, top_pages=w.top_pages, window=w.window, sinks=w.sinks,
-                      seed=w.seed, kv_bits=kv_bits)
+                      seed=w.seed, kv_bits=kv_bits,
+                      head_shard=(w.hkv_model << 16) | w.kvh0 if w.hkv_model else 0)
 
 
 def run_decode(w, args, dev, stream, world, rank, peaks):
     from hierarchical_long_context_b200 import api, metrics
+    qf = world if args.shard == "batch" else 1  # sequences decoded per step, over all ranks, / w.B
     p = params_for(w)
     K, V = synth_kv(w)
     Kd, Vd = K.to(dev), V.to(dev)
@@ -321,7 +324,7 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
     achieved = touched / (ms * 1e-3) / 1e9
     res = dict(
         metric="LoD decode queries/s (batch 4 x 64 heads at 128K context, one layer)",
-        value=world * w.B / (ms_max * 1e-3), unit="queries/s", ms_per_step=ms_max,
+        value=qf * w.B / (ms_max * 1e-3), unit="queries/s", ms_per_step=ms_max,
         ms_p10=float(np.percentile(ts, 10)), ms_p90=float(np.percentile(ts, 90)),
         head_rows_per_s=world * w.B * w.Hq / (ms_max * 1e-3), wall_s_timed=wall,
         status_word=status,
@@ -329,7 +332,7 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
                       peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved / peaks["hbm_gbs"],
                       traffic=profiled_traffic("lod_decode", w.name), algorithmic_bytes_per_launch=touched,
                       peak_source=peaks["source"], nominal_peak_gbs=8000.0),
-        e2e=dict(value=world * w.B / (e2e_ms * 1e-3), unit="queries/s",
+        e2e=dict(value=qf * w.B / (e2e_ms * 1e-3), unit="queries/s",
                  h2d_bytes_per_step=hin.numel() * hin.element_size(),
                  d2h_bytes_per_step=hout.numel() * hout.element_size(), ms_per_step=e2e_ms,
                  step="one CUDA graph per step: pinned input copy, cache-row writes, lod_decode, "
@@ -517,6 +520,8 @@ def main():
     ap.add_argument("--graphs", type=int, default=1, help="e2e: one CUDA graph per step (0 = eager)")
     ap.add_argument("--replicas", type=int, default=4,
                     help="decode: device replicas of the inputs used in rotation (1 = flush L2 instead)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="N > 1: every rank its own batch (weak scaling) or the KV heads split over ranks (strong)")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per step (0 = the workload's own; smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -532,8 +537,8 @@ def main():
         if rank == 0:
             run_reference(args, w)
         return
-    if world > 1:
-        w = w.with_(seed=w.seed + rank)  # every rank its own replica of the batch
+    wg = w
+    w = synth.shard(w, args.shard, rank, world)
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
@@ -564,11 +569,13 @@ def main():
     if rank == 0:
         line = dict(metric=res["metric"], value=res["value"], unit=res["unit"], n_gpus=world,
                     steps=args.steps, warmup=args.warmup, ms_per_step=res["ms_per_step"],
-                    higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+                    higher_is_better=True, scaling="strong" if args.shard == "heads" and world > 1 else "weak",
+                    vs_baseline=None, dtype="bf16",
                     data="synthetic (seeded Gaussian-mixture keys + RoPE + outlier channels, N(0,1) values)",
-                    config=dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, seq_len=w.T,
+                    config=dict(workload=w.name, B=wg.B, Hq=wg.Hq, Hkv=wg.Hkv, d=w.d, seq_len=w.T,
                                 clusters=w.clusters[0], top_groups=w.top_groups, top_pages=w.top_pages,
-                                window=w.window, sinks=w.sinks, parallelism="replicas x%d" % world,
+                                window=w.window, sinks=w.sinks,
+                                parallelism=("heads x%d" if args.shard == "heads" else "replicas x%d") % world,
                                 l2=res["l2"]),
                     roofline=res["roofline"], cpu_baseline=extras.pop("cpu_baseline", None),
                     e2e=res["e2e"], gpu_launches=res["gpu_launches"], clocks=res["clocks"],

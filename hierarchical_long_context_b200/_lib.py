@@ -31,7 +31,7 @@ class lod_params(ctypes.Structure):
         ("page", ctypes.c_int32), ("clusters", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
         ("top_groups", ctypes.c_int32), ("top_pages", ctypes.c_int32), ("window", ctypes.c_int32),
         ("sinks", ctypes.c_int32), ("kv_bits", ctypes.c_int32), ("seed", ctypes.c_uint64),
-        ("scale", ctypes.c_float), ("reserved1", ctypes.c_int32), ("Tmax", ctypes.c_int64),
+        ("scale", ctypes.c_float), ("head_shard", ctypes.c_int32), ("Tmax", ctypes.c_int64),
     ]
 
 

@@ -37,12 +37,13 @@ class Params:
     chunk: int = 256
     page: int = 16
     kv_bits: int = 0   # 4: three-tier INT4 (opened pages read from 4-bit codes)
+    head_shard: int = 0  # (model KV heads << 16) | first KV head, for a head-sharded process
 
     def c(self) -> _lib.lod_params:
         return _lib.lod_params(
             _DT[self.dtype], self.B, self.Hq, self.Hkv, self.d, self.chunk, self.page,
             self.clusters, self.kmeans_iters, self.top_groups, self.top_pages, self.window,
-            self.sinks, self.kv_bits, self.seed & (2**64 - 1), self.scale, 0, self.Tmax)
+            self.sinks, self.kv_bits, self.seed & (2**64 - 1), self.scale, self.head_shard, self.Tmax)
 
     @property
     def page_slots(self) -> int:

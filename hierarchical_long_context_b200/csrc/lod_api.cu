@@ -39,7 +39,11 @@ int nq_max(const lod_params*) { return 8; }
 
 int32_t validate(const lod_params* p) {
   if (!p) return fail(LOD_EINVAL, "params is NULL");
-  if (p->reserved1 != 0) return fail(LOD_EINVAL, "reserved fields must be 0");
+  if (p->head_shard != 0) {
+    const int tot = p->head_shard >> 16, first = p->head_shard & 0xffff;
+    if (tot < p->Hkv || first + p->Hkv > tot)
+      return fail(LOD_EINVAL, "head_shard: KV heads [%d, %d) outside the model's %d", first, first + p->Hkv, tot);
+  }
   if (p->kv_bits != 0 && p->kv_bits != 4)
     return fail(LOD_EUNSUPPORTED, "kv_bits = %d unsupported (0 or 4)", p->kv_bits);
   if (p->kv_bits == 4 && p->top_pages == 0)
@@ -267,6 +271,7 @@ int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_
   a.k = p->clusters;
   a.iters = p->kmeans_iters;
   a.sinks = p->sinks;
+  a.head_shard = p->head_shard;
   a.P = page_slots(p);
   a.chunk_begin = c0;
   a.seq_lens = seq_lens;

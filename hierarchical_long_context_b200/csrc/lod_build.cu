@@ -224,7 +224,9 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
   for (int j = 0; j < k; ++j) {
     int pick;
     if (j == 0) {
-      const uint64_t hsh = splitmix64(a.seed ^ ((uint64_t(unit) << 32) + uint64_t(c)));
+      // the initialisation's sequence-head index is model-wide under head sharding
+      const int64_t sunit = a.head_shard ? (int64_t)b * (a.head_shard >> 16) + (a.head_shard & 0xffff) + h : unit;
+      const uint64_t hsh = splitmix64(a.seed ^ ((uint64_t(sunit) << 32) + uint64_t(c)));
       pick = (int)(hsh % uint64_t(n));
     } else {
       float bv;

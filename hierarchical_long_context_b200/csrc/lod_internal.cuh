@@ -20,6 +20,7 @@ struct BuildArgs {
   int k;               // clusters
   int iters;           // Lloyd rounds
   int sinks;
+  int head_shard;      // 0, or (model KV heads << 16) | this shard's first KV head
   int P;               // page slots per chunk
   int64_t chunk_begin;
   const int64_t* seq_lens;  // non-null: per sequence, the chunk its length just completed (else nothing)

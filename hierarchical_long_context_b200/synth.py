@@ -53,6 +53,8 @@ class Workload:
     chunk: int = 256
     page: int = 16
     note: str = ""
+    kvh0: int = 0              # global index of the first KV head (a head shard's slice)
+    hkv_model: int = 0         # a head shard's model-wide KV head count (0: not sharded)
 
     @property
     def g(self) -> int:
@@ -101,7 +103,25 @@ WORKLOADS = {
 def _unit_rng(w: Workload, b: int, kvh: int, stream: str) -> np.random.Generator:
     tag = zlib.crc32(w.name.replace("_zero_variance", "").encode())
     s2 = zlib.crc32(stream.encode())
-    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, tag, b, kvh, s2])))
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, tag, b, kvh + w.kvh0, s2])))
+
+
+def shard(w: Workload, mode: str, rank: int, world: int) -> Workload:
+    """Rank `rank`'s part of workload `w` on `world` GPUs.  "batch": every
+    rank decodes its own batch (a replica with its own seed; weak scaling).
+    "heads": the ranks split the KV heads (with their query heads) of the one
+    batch, as tensor-parallel attention does; rank r generates exactly its
+    slice of the global inputs (strong scaling).  No data crosses ranks."""
+    if world == 1:
+        return w
+    if mode == "batch":
+        return w.with_(seed=w.seed + rank)
+    if mode == "heads":
+        if w.Hkv % world:
+            raise ValueError("%d KV heads do not split over %d ranks" % (w.Hkv, world))
+        h = w.Hkv // world
+        return w.with_(Hkv=h, Hq=h * w.g, kvh0=w.kvh0 + rank * h, hkv_model=w.hkv_model or w.Hkv)
+    raise ValueError("shard mode %r" % mode)
 
 
 def _rope(x: np.ndarray, theta: float, pos0: int = 0) -> np.ndarray:
@@ -198,7 +218,7 @@ def kv_cache_device(w: Workload, device, T: int | None = None):
     step = 65536
     for b in range(w.B):
         for h in range(w.Hkv):
-            tag = zlib.crc32(("%s/%d/%d" % (w.name, b, h)).encode())
+            tag = zlib.crc32(("%s/%d/%d" % (w.name, b, h + w.kvh0)).encode())
             g = torch.Generator(device=device).manual_seed((w.seed << 32) ^ tag)
             cen = torch.randn((w.n_centers, w.d), generator=g, device=device)
             cen /= cen.norm(dim=1, keepdim=True)

@@ -77,7 +77,12 @@ typedef enum { LOD_OP_BUILD = 0, LOD_OP_DECODE = 1, LOD_OP_PREFILL = 2 } lod_op;
  * members of every indexed page are kept as 4-bit codes of a per-page,
  * per-channel quantiser (see lod_index) and an opened page is read from
  * them; it needs top_pages >= 1.  The summaries, the sinks and the window
- * always use the cache dtype.
+ * always use the cache dtype.  head_shard: a process that holds KV heads
+ * [first, first + Hkv) of a model with more KV heads (tensor-parallel
+ * attention) passes (model KV heads << 16) | first, so that the k-means
+ * initialisation of sequence b, head h uses the model-wide index
+ * b * (model KV heads) + first + h and the shard's index equals the one an
+ * unsharded process builds; 0 for an unsharded model.
  */
 typedef struct lod_params {
   int32_t dtype;        /* lod_dtype */
@@ -96,7 +101,7 @@ typedef struct lod_params {
   int32_t kv_bits;      /* 0: opened pages read in the cache dtype; 4: three-tier INT4 */
   uint64_t seed;        /* k-means initialisation seed */
   float scale;          /* softmax scale on q.k; <= 0 means 1/sqrt(d) */
-  int32_t reserved1;    /* must be 0 */
+  int32_t head_shard;   /* 0, or (model KV heads << 16) | first KV head of this shard */
   int64_t Tmax;         /* capacity of the KV cache and of the index, in tokens */
 } lod_params;
 

@@ -141,11 +141,11 @@ def test_null_and_misaligned_pointers_fail_before_any_launch():
     assert rc == _lib.LOD_EINVAL and b"query range" in L.lod_last_error()
 
 
-def test_reserved_fields_must_be_zero():
-    p = P().c()
-    p.reserved1 = 1
+def test_head_shard_must_lie_inside_the_model():
     sizes = (ctypes.c_size_t * len(_lib.INDEX_FIELDS))()
-    assert _lib.load().lod_index_sizes(ctypes.byref(p), sizes) == _lib.LOD_EINVAL
+    for hs, rc in (((4 << 16) | 2, 0), ((4 << 16) | 3, _lib.LOD_EINVAL), ((1 << 16) | 0, _lib.LOD_EINVAL)):
+        p = P(head_shard=hs).c()
+        assert _lib.load().lod_index_sizes(ctypes.byref(p), sizes) == rc, hs
 
 
 def test_struct_layout_matches_the_header():

@@ -288,6 +288,30 @@ def test_online_build_during_decode_matches_bulk_build():
                 assert torch.equal(on[b, :, 7 * n:8 * n], getattr(fresh, f)[b, :, 7 * n:8 * n]), f
 
 
+def test_head_shard_builds_the_unsharded_index_slice():
+    """A process holding KV heads [2, 4) of a 4-head model (head_shard) builds
+    exactly those heads' slice of the unsharded index, and decodes them alike."""
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, Hkv=4, Hq=16)
+    T = 2048
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    ws_ = synth.shard(w, "heads", 1, 2)
+    ps = lt.params_of(ws_, Tmax=p.Tmax, head_shard=(ws_.hkv_model << 16) | ws_.kvh0)
+    Ks, Vs = Kd[:, 2:4].contiguous(), Vd[:, 2:4].contiguous()
+    ixs = api.Index(ps)
+    api.lod_build_index(ps, Ks, Vs, 0, T // 256, ixs)
+    for f in api._lib.INDEX_FIELDS:
+        a, b = getattr(ix, f), getattr(ixs, f)
+        if a.numel():
+            assert torch.equal(a[:, 2:4], b), f
+    sl = torch.full((w.B,), T, dtype=torch.int64, device=Kd.device)
+    q = synth.decode_queries(w).to(Kd.device)
+    out = api.lod_decode(p, q, Kd, Vd, sl, ix)
+    outs = api.lod_decode(ps, q[:, 8:16].contiguous(), Ks, Vs, sl, ixs)
+    assert torch.equal(out[:, 8:16], outs)
+
+
 def test_zero_variance_decode_equals_dense():
     """Level of Detail Attention, How It Works: zero-variance groups give full
     attention -- checked on the GPU path directly against dense softmax."""
