@@ -136,9 +136,17 @@ __device__ __forceinline__ void ldv_f(const T* p, float (&v)[N]) {
   }
 }
 
-// 4-bit code i of the packed word w as a float (2^23 + code, minus 2^23: exact).
-__device__ __forceinline__ float nibble_f(uint32_t w, int i) {
-  return __int_as_float(0x4B000000u | ((w >> (4 * i)) & 15u)) - 8388608.0f;
+// The 4-bit codes of a lane's channels (nibbles 0..DPL-1 of w) as float
+// pairs.  Nibble i is placed into the mantissa of 2^23 in place (2^23 +
+// 2^(4i) code, exact) and one packed fma scales it back: x * 2^-4i -
+// 2^(23-4i) = code, exactly.
+template <int DPL>
+__device__ __forceinline__ void lane_nibbles(uint32_t w, float2 (&c)[DPL / 2]) {
+  c[0] = ffma2(make_float2(__uint_as_float(0x4B000000u | (w & 0xFu)), __uint_as_float(0x4B000000u | (w & 0xF0u))),
+               make_float2(1.0f, 0.0625f), make_float2(-8388608.0f, -524288.0f));
+  if constexpr (DPL == 4)
+    c[1] = ffma2(make_float2(__uint_as_float(0x4B000000u | (w & 0xF00u)), __uint_as_float(0x4B000000u | (w & 0xF000u))),
+                 make_float2(1.0f / 256.0f, 1.0f / 4096.0f), make_float2(-32768.0f, -2048.0f));
 }
 
 // Sum over the warp of 16 per-lane values: lane l receives the total of value
@@ -816,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const int64_t wbq = t / kChunk - a.window / kChunk + 1;
     const int Gq = wbq > 0 ? (int)(wbq * a.k) : 0;  // visible groups of this row
     const float2* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
-    constexpr int kSel = 16;  // scores per thread kept in registers (up to 4096 groups)
+    constexpr int kSel = 8;  // scores per thread kept in registers (up to 2048 groups)
     const bool in_regs = Gq <= kSel * kThreads;
     const int ns = (Gq + kThreads - 1) / kThreads;  // register slots in use (uniform)
     float sv[kSel];
@@ -1144,12 +1152,14 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       const int n = x == 0 ? na : nb;
       const float2* kq = reinterpret_cast<const float2*>(stg + (4 + x) * PB);
       const uint8_t* kc = stg + x * PB;
-      float qsc[DPL], qlo = 0.f;
+      float2 qsc[DPL / 2];
+      float qlo = 0.f;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        const float2 z = kq[lane * DPL + i];
-        qsc[i] = qd[i] * z.x;
-        qlo = fmaf(qd[i], z.y, qlo);
+      for (int i = 0; i < DPL; i += 2) {
+        const float2 z0 = kq[lane * DPL + i], z1 = kq[lane * DPL + i + 1];
+        qsc[i / 2] = make_float2(qd[i] * z0.x, qd[i + 1] * z1.x);
+        qlo = fmaf(qd[i], z0.y, qlo);
+        qlo = fmaf(qd[i + 1], z1.y, qlo);
       }
       qlo = warp_sum(qlo);
       float part[kPage];
@@ -1157,11 +1167,12 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       for (int r = 0; r < kPage; ++r) {
         part[r] = 0.f;
         if (r < n) {
-          const uint32_t w = lane_codes<D, DPL>(kc + r * (D / 2), lane);
-          float sdot = 0.f;
+          float2 cw[DPL / 2];
+          lane_nibbles<DPL>(lane_codes<D, DPL>(kc + r * (D / 2), lane), cw);
+          float2 sd = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) sdot = fmaf(qsc[i], nibble_f(w, i), sdot);
-          part[r] = sdot;
+          for (int i = 0; i < DPL / 2; ++i) sd = ffma2(qsc[i], cw[i], sd);
+          part[r] = sd.x + sd.y;
         }
       }
       const float tot = transpose_sum16(part, lane) + qlo;  // member lane >> 1
@@ -1188,23 +1199,26 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       const int n = x == 0 ? na : nb;
       const float2* vq = reinterpret_cast<const float2*>(stg + (6 + x) * PB);
       const uint8_t* vc = stg + (2 + x) * PB;
-      float ac[DPL], ps = 0.f;
+      float2 ac[DPL / 2];
+      float ps = 0.f;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) ac[i] = 0.f;
-#pragma unroll
+      for (int i = 0; i < DPL / 2; ++i) ac[i] = make_float2(0.f, 0.f);
+#pragma unroll 4
       for (int r = 0; r < kPage; ++r) {
         if (r < n) {
           const float pr = mysc[16 * x + r];
-          const uint32_t w = lane_codes<D, DPL>(vc + r * (D / 2), lane);
+          float2 cw[DPL / 2];
+          lane_nibbles<DPL>(lane_codes<D, DPL>(vc + r * (D / 2), lane), cw);
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) ac[i] = fmaf(pr, nibble_f(w, i), ac[i]);
+          for (int i = 0; i < DPL / 2; ++i) ac[i] = ffma2(make_float2(pr, pr), cw[i], ac[i]);
           ps += pr;
         }
       }
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
         const float2 z = vq[lane * DPL + i];
-        acc[i] = fmaf(z.x, ac[i], fmaf(z.y, ps, acc[i]));
+        const float a_i = (i & 1) ? ac[i / 2].y : ac[i / 2].x;
+        acc[i] = fmaf(z.x, a_i, fmaf(z.y, ps, acc[i]));
       }
     }
     // coarse entries, in lane order
