@@ -176,25 +176,6 @@ __device__ __forceinline__ uint32_t lane_codes(const uint8_t* row, int lane) {
   }
 }
 
-// Dot product of a whole d-row (owned by one lane) with q held in shared memory.
-template <typename T, int D>
-__device__ __forceinline__ float row_dot(const T* __restrict__ row, const float* __restrict__ qs) {
-  constexpr int VEC = 16 / sizeof(T);
-  uint4 raw[D / VEC];
-#pragma unroll
-  for (int v = 0; v < D / VEC; ++v) raw[v] = __ldg(reinterpret_cast<const uint4*>(row) + v);
-  float2 s = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int v = 0; v < D / VEC; ++v) {
-    float f[VEC];
-    unpack16<T>(raw[v], f);
-#pragma unroll
-    for (int e = 0; e < VEC; e += 2)
-      s = ffma2(make_float2(qs[v * VEC + e], qs[v * VEC + e + 1]), make_float2(f[e], f[e + 1]), s);
-  }
-  return s.x + s.y;
-}
-
 struct UnitInfo {
   int b, kvh;
   int64_t blk, nblk;
@@ -220,8 +201,6 @@ __device__ __forceinline__ UnitInfo unit_info(const AttendArgs& a, int64_t u) {
 struct Cand {
   float s;     // scale * q.mean_k
   int id;      // group id within the unit (chunk * k + slot), -1 = none
-  int pages;   // first page slot | (last page slot + 1) << 16
-  int cnt;     // group size
 };
 
 // ------------------------------------------------------------------ scan

@@ -34,15 +34,16 @@ def _np(t):
     return t.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("name, units", [
-    ("decode_gqa_32k_bf16", [(0, 0), (5, 3), (7, 7)]),
-    ("decode_gqa_128k_bf16", [(0, 1), (3, 6)]),
+@pytest.mark.parametrize("name, units, kv_bits", [
+    ("decode_gqa_32k_bf16", [(0, 0), (5, 3), (7, 7)], 0),
+    ("decode_gqa_128k_bf16", [(0, 1), (3, 6)], 0),
+    ("decode_gqa_128k_bf16", [(1, 2), (2, 5)], 4),   # three-tier INT4
 ])
-def test_decode_full_size(name, units):
+def test_decode_full_size(name, units, kv_bits):
     dev = _dev()
     w = synth.WORKLOADS[name]
     K, V = synth.kv_cache(w)
-    p = lt.params_of(w)
+    p = lt.params_of(w, kv_bits=kv_bits)
     Kd, Vd = K.to(dev), V.to(dev)
     ix = api.Index(p, dev)
     api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix)
@@ -63,6 +64,9 @@ def test_decode_full_size(name, units):
         ou = oracle.build_sequence(cfg, b * w.Hkv + h, Kn, Vn, nch)
         st = lt.compare_builds(gu, ou, cfg, True)
         assert st["diverged"] <= max(2, nch // 20), st
+        if kv_bits == 4:
+            lt.check_int4_pages(ix, b, h, gu, Kn, Vn, cfg)
+            gu = lt.quantized(gu, Kn, Vn, cfg)
         rows = [(_np(q[b, hq]), w.T - 1, _np(out[b, hq]).astype(np.float64), float(lse[b, hq]),
                  sg[b, hq].cpu().numpy(), sp[b, hq].cpu().numpy()) for hq in range(h * w.g, (h + 1) * w.g)]
         print(name, (b, h), st, lt.check_rows(cfg, w.dtype, Kn, Vn, gu, rows))

@@ -330,16 +330,17 @@ def test_zero_variance_decode_equals_dense():
 
 # ------------------------------------------------------------------ prefill
 
-@pytest.mark.parametrize("name, T, split", [
-    ("prefill_128k_bf16", 2048 + 100, None),      # ragged tail, one call
-    ("prefill_128k_bf16", 2048 + 100, 1024),      # two calls: the second continues the first
-    ("decode_tiny_f32", 1536 + 37, None),
-    ("decode_gqa_32k_bf16", 1024 + 300, None),    # g = 8: one position per scan unit
+@pytest.mark.parametrize("name, T, split, kv_bits", [
+    ("prefill_128k_bf16", 2048 + 100, None, 0),      # ragged tail, one call
+    ("prefill_128k_bf16", 2048 + 100, 1024, 0),      # two calls: the second continues the first
+    ("decode_tiny_f32", 1536 + 37, None, 0),
+    ("decode_gqa_32k_bf16", 1024 + 300, None, 0),    # g = 8: one position per scan unit
+    ("prefill_128k_bf16", 2048 + 100, 1024, 4),      # three-tier INT4
 ])
-def test_prefill_matches_oracle(name, T, split):
+def test_prefill_matches_oracle(name, T, split, kv_bits):
     w = synth.WORKLOADS[name]
     w = w.with_(B=1, Hkv=min(w.Hkv, 2), Hq=min(w.Hkv, 2) * w.g, T=T)
-    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T, kv_bits=kv_bits)
     dev = Kd.device
     qc = synth.prefill_queries(w, 0, T)
     q = qc.to(dev)
@@ -361,6 +362,9 @@ def test_prefill_matches_oracle(name, T, split):
         K, V = _np(Kc[0, h]), _np(Vc[0, h])
         u = lt.unit_from_gpu(ix, 0, h, nch, p)
         lt.check_index_consistency(u, K, V, cfg, w.dtype == "bf16")
+        if kv_bits == 4:
+            lt.check_int4_pages(ix, 0, h, u, K, V, cfg)
+            u = lt.quantized(u, K, V, cfg)
         ts = sorted(set(rng.integers(0, T, 48).tolist()) | {0, 255, 256, 511, 512, T - 1})
         rows = []
         for hq in range(h * w.g, (h + 1) * w.g):
