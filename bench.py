@@ -522,6 +522,10 @@ def main():
                     help="decode: device replicas of the inputs used in rotation (1 = flush L2 instead)")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
                     help="N > 1: every rank its own batch (weak scaling) or the KV heads split over ranks (strong)")
+    ap.add_argument("--leg", default=None, choices=["prefill", "build"],
+                    help="run only this secondary leg and print its result (profiler captures)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="with --leg: context length of the leg's workload (0 = its own)")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per step (0 = the workload's own; smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -536,6 +540,17 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w)
+        return
+    if args.leg:  # one secondary leg alone, on one GPU
+        peaks = load_peaks()
+        dev = torch.device("cuda", torch.cuda.current_device())
+        name = "prefill_128k_bf16" if args.leg == "prefill" else "build_128k_bf16"
+        wl = synth.WORKLOADS[name]
+        if args.seq_len:
+            wl = wl.with_(T=args.seq_len)
+        r = (run_prefill(wl, dev, torch.cuda.current_stream(), 2, peaks) if args.leg == "prefill" else
+             run_build(wl, dev, torch.cuda.current_stream(), 5, peaks, 4))
+        print(json.dumps(r), flush=True)
         return
     wg = w
     w = synth.shard(w, args.shard, rank, world)
