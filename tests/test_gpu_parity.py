@@ -132,6 +132,7 @@ def test_decode_on_gpu_index_matches_oracle(name, T, seq_lens):
     dict(Hq=16, Hkv=2, window=256, sinks=0),                                   # g=8, short window, no sinks
     dict(top_pages=0),                                                         # two-tier LoD, g=8
     dict(d=64, dtype="f32", Hq=4, Hkv=2, top_groups=16, top_pages=0),          # two-tier, CUDA-core scan
+    dict(Hq=16, Hkv=2, sinks=100),                                             # more sinks than free lanes
 ])
 def test_decode_parameter_sweep(kw):
     """Head ratios, head sizes, dtypes, cluster counts and selection widths at
