@@ -228,7 +228,7 @@ def params_for(w, k=None, kv_bits=0):
 def run_decode(w, args, dev, stream, world, rank, peaks):
     from hierarchical_long_context_b200 import api, metrics
     qf = world if args.shard == "batch" else 1  # sequences decoded per step, over all ranks, / w.B
-    p = params_for(w)
+    p = params_for(w, kv_bits=args.kv_bits)
     K, V = synth_kv(w)
     Kd, Vd = K.to(dev), V.to(dev)
     ix = api.Index(p, dev)
@@ -330,7 +330,8 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
         status_word=status,
         roofline=dict(bound="hbm", kernel="lod_decode (scan + refine kernels)", achieved=achieved,
                       peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved / peaks["hbm_gbs"],
-                      traffic=profiled_traffic("lod_decode", w.name), algorithmic_bytes_per_launch=touched,
+                      traffic=profiled_traffic("lod_decode_int4" if args.kv_bits == 4 else "lod_decode", w.name),
+                      algorithmic_bytes_per_launch=touched,
                       peak_source=peaks["source"], nominal_peak_gbs=8000.0),
         e2e=dict(value=qf * w.B / (e2e_ms * 1e-3), unit="queries/s",
                  h2d_bytes_per_step=hin.numel() * hin.element_size(),
@@ -526,6 +527,8 @@ def main():
                     help="run only this secondary leg and print its result (profiler captures)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="with --leg: context length of the leg's workload (0 = its own)")
+    ap.add_argument("--kv-bits", type=int, default=0, choices=[0, 4],
+                    help="main decode leg in three-tier INT4 (opened pages from 4-bit codes)")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per step (0 = the workload's own; smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -589,6 +592,7 @@ def main():
                     data="synthetic (seeded Gaussian-mixture keys + RoPE + outlier channels, N(0,1) values)",
                     config=dict(workload=w.name, B=wg.B, Hq=wg.Hq, Hkv=wg.Hkv, d=w.d, seq_len=w.T,
                                 clusters=w.clusters[0], top_groups=w.top_groups, top_pages=w.top_pages,
+                                kv_bits=args.kv_bits,
                                 window=w.window, sinks=w.sinks,
                                 parallelism=("heads x%d" if args.shard == "heads" else "replicas x%d") % world,
                                 l2=res["l2"]),
