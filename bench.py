@@ -292,8 +292,8 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
         qr, Kr, Vr, slr, ixr, wsr, outr = reps[r]
         st = stage[r]
         st.copy_(hin, non_blocking=True)
-        Kr[:, :, w.T - 1].copy_(st[qn:qn + rown].view(w.B, w.Hkv, w.d))
-        Vr[:, :, w.T - 1].copy_(st[qn + rown:].view(w.B, w.Hkv, w.d))
+        api.lod_append_kv(p, Kr, Vr, slr, st[qn:qn + rown].view(w.B, w.Hkv, w.d),
+                          st[qn + rown:].view(w.B, w.Hkv, w.d), stream=strm)
         api.lod_decode(p, st[:qn].view(q.shape), Kr, Vr, slr, ixr, out=outr, ws=wsr, stream=strm)
         hout.copy_(outr, non_blocking=True)
 
@@ -336,8 +336,8 @@ def run_decode(w, args, dev, stream, world, rank, peaks):
         e2e=dict(value=qf * w.B / (e2e_ms * 1e-3), unit="queries/s",
                  h2d_bytes_per_step=hin.numel() * hin.element_size(),
                  d2h_bytes_per_step=hout.numel() * hout.element_size(), ms_per_step=e2e_ms,
-                 step="one CUDA graph per step: pinned input copy, cache-row writes, lod_decode, "
-                      "output copy" if graphs else "eager: pinned input copy, cache-row writes, "
+                 step="one CUDA graph per step: pinned input copy, lod_append_kv, lod_decode, "
+                      "output copy" if graphs else "eager: pinned input copy, lod_append_kv, "
                       "lod_decode, output copy"),
         gpu_launches=2 * args.steps,
         clocks=cs.summary(),

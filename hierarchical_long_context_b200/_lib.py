@@ -19,7 +19,7 @@ LOD_ST_BAD_SEQLEN, LOD_ST_BAD_PAGE, LOD_ST_BAD_MEMBER, LOD_ST_BAD_COUNT = 1, 2, 
 
 # Every symbol include/lod.h declares.
 EXPORTS = ("lod_version", "lod_last_error", "lod_index_sizes", "lod_workspace_bytes",
-           "lod_build_index", "lod_build_ready", "lod_decode", "lod_prefill", "lod_get_status",
+           "lod_build_index", "lod_build_ready", "lod_append_kv", "lod_decode", "lod_prefill", "lod_get_status",
            "lod_decode_noalloc")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -76,6 +76,8 @@ def load():
     lib.lod_build_index.restype = ctypes.c_int32
     lib.lod_build_index.argtypes = [_P(lod_params), _vp, _vp, _P(_i64), _i64, _i64, _P(lod_index),
                                     _vp, ctypes.c_size_t, _vp]
+    lib.lod_append_kv.restype = ctypes.c_int32
+    lib.lod_append_kv.argtypes = [_P(lod_params), _vp, _vp, _P(_i64), _vp, _vp, _vp, _vp]
     lib.lod_build_ready.restype = ctypes.c_int32
     lib.lod_build_ready.argtypes = [_P(lod_params), _vp, _vp, _P(_i64), _vp, _P(lod_index), _vp,
                                     ctypes.c_size_t, _vp]

@@ -138,6 +138,20 @@ def lod_build_index(params: Params, K, V, chunk_begin: int, chunk_end: int, inde
         ctypes.byref(index.c()), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def lod_append_kv(params: Params, K, V, seq_lens, k_new, v_new, stream=None) -> None:
+    """Write the current token's key/value rows k_new, v_new ([B, Hkv, d],
+    cache dtype) into K/V at positions seq_lens - 1 (one kernel)."""
+    lib = load()
+    st = _kv_strides(params, K, V)
+    shape = (params.B, params.Hkv, params.d)
+    for t in (k_new, v_new):
+        if t.shape != shape or t.dtype != params.dtype or not t.is_contiguous():
+            raise ValueError("k_new / v_new must be contiguous %s %s" % (shape, params.dtype))
+    check("lod_append_kv", lib.lod_append_kv(
+        ctypes.byref(params.c()), _ptr(K), _ptr(V), st, _ptr(seq_lens), _ptr(k_new), _ptr(v_new),
+        _stream(stream)))
+
+
 def lod_build_ready(params: Params, K, V, seq_lens, index: Index, ws=None, stream=None) -> None:
     """Online build: for every sequence whose length (seq_lens, device int64
     [B]) is a positive multiple of the chunk, build the chunk it just

@@ -361,6 +361,20 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V, const
   return rc;
 }
 
+int32_t lod_append_kv(const lod_params* p, void* K, void* V, const int64_t kv_strides[3], const int64_t* seq_lens,
+                      const void* k_new, const void* v_new, lod_stream_t stream) {
+  int32_t rc = validate(p);
+  if (!rc) rc = validate_kv(p, K, V, kv_strides);
+  if (rc) return rc;
+  if (!seq_lens || !k_new || !v_new) return fail(LOD_EINVAL, "seq_lens, k_new and v_new must be non-NULL");
+  if (!aligned16(k_new) || !aligned16(v_new)) return fail(LOD_EINVAL, "k_new and v_new must be 16-byte aligned");
+  cudaError_t e = lod::launch_append(K, V, kv_strides, (int)elem_bytes(p), p->d, seq_lens, k_new, v_new, p->B,
+                                     p->Hkv, p->Tmax, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  g_err[0] = 0;
+  return LOD_OK;
+}
+
 int32_t lod_build_ready(const lod_params* p, const void* K, const void* V, const int64_t kv_strides[3],
                         const int64_t* seq_lens, const lod_index* index, void* ws, size_t ws_bytes,
                         lod_stream_t stream) {

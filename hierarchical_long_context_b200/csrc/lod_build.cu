@@ -505,6 +505,35 @@ cudaError_t launch_kmeans_d(const BuildArgs& a, int64_t nchunks, int B, cudaStre
 
 }  // namespace
 
+// The new token's key and value rows of every (b, kvh) written into the cache
+// at position seq_lens[b] - 1 (skipped when that is outside [0, Tmax)).
+// One CTA per sequence; 16-byte copies.
+__global__ void append_kv_kernel(uint4* K, uint4* V, int64_t sb, int64_t sh, int64_t st, const int64_t* seq_lens,
+                                 const uint4* kn, const uint4* vn, int Hkv, int row16, int64_t Tmax) {
+  const int b = blockIdx.x;
+  const int64_t t = seq_lens[b] - 1;
+  if (t < 0 || t >= Tmax) return;
+  for (int i = threadIdx.x; i < Hkv * row16; i += blockDim.x) {
+    const int h = i / row16, c = i % row16;
+    const int64_t dst = b * sb + h * sh + t * st + c;
+    const int64_t src = ((int64_t)b * Hkv + h) * row16 + c;
+    K[dst] = kn[src];
+    V[dst] = vn[src];
+  }
+}
+
+cudaError_t launch_append(void* K, void* V, const int64_t* kv_strides_elems, int elem_bytes, int d,
+                          const int64_t* seq_lens, const void* kn, const void* vn, int B, int Hkv, int64_t Tmax,
+                          cudaStream_t stream) {
+  const int64_t per16 = 16 / elem_bytes;  // elements per 16-byte piece
+  const int row16 = d * elem_bytes / 16;
+  append_kv_kernel<<<B, 128, 0, stream>>>(static_cast<uint4*>(K), static_cast<uint4*>(V), kv_strides_elems[0] / per16,
+                                          kv_strides_elems[1] / per16, kv_strides_elems[2] / per16, seq_lens,
+                                          static_cast<const uint4*>(kn), static_cast<const uint4*>(vn), Hkv, row16,
+                                          Tmax);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
                          cudaStream_t stream) {
   if (dtype == LOD_DTYPE_F32) {

@@ -143,6 +143,9 @@ struct __align__(64) TcMaps {
 
 cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
                          cudaStream_t stream);
+cudaError_t launch_append(void* K, void* V, const int64_t* kv_strides_elems, int elem_bytes, int d,
+                          const int64_t* seq_lens, const void* kn, const void* vn, int B, int Hkv, int64_t Tmax,
+                          cudaStream_t stream);
 // maps == nullptr selects the CUDA-core scan; otherwise bf16, d = 128 run the
 // tensor-core scan.
 cudaError_t launch_attend(const AttendArgs& a, int dtype, int d, int NQ, const TcMaps* maps,

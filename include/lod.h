@@ -203,6 +203,17 @@ int32_t lod_build_index(const lod_params* p, const void* K, const void* V,
                         const lod_index* index, void* ws, size_t ws_bytes, lod_stream_t stream);
 
 /*
+ * Append the current token: for every sequence b, writes k_new[b][h] and
+ * v_new[b][h] (device [B][Hkv][d], cache dtype, contiguous, 16-byte aligned)
+ * into the cache rows K/V[b][h][seq_lens[b] - 1] (seq_lens device [B] int64;
+ * a length outside [1, Tmax] skips that sequence).  One kernel for the whole
+ * batch, asynchronous on `stream`; with lod_decode after it on the same
+ * stream, the decode reads the new rows.
+ */
+int32_t lod_append_kv(const lod_params* p, void* K, void* V, const int64_t kv_strides[3],
+                      const int64_t* seq_lens, const void* k_new, const void* v_new, lod_stream_t stream);
+
+/*
  * Online index build for decode ("How It Works", paragraph 1: the index is
  * built as inference proceeds, after every chunk of 256 tokens): for every
  * sequence b whose length seq_lens[b] (device [B] int64) is a positive

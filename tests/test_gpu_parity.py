@@ -313,6 +313,25 @@ def test_head_shard_builds_the_unsharded_index_slice():
     assert torch.equal(out[:, 8:16], outs)
 
 
+def test_append_kv_writes_the_current_rows_only():
+    """lod_append_kv writes each sequence's new key/value rows at seq_len - 1
+    and nothing else; a length outside [1, Tmax] leaves that sequence alone."""
+    dev = _cuda()
+    p = api.Params(B=3, Hq=16, Hkv=2, d=128, Tmax=1024, dtype=torch.bfloat16)
+    g = torch.Generator(device=dev).manual_seed(5)
+    K = torch.randn(3, 2, 1024, 128, generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn(3, 2, 1024, 128, generator=g, device=dev).to(torch.bfloat16)
+    K0, V0 = K.clone(), V.clone()
+    kn = torch.randn(3, 2, 128, generator=g, device=dev).to(torch.bfloat16)
+    vn = torch.randn(3, 2, 128, generator=g, device=dev).to(torch.bfloat16)
+    sl = torch.tensor([5, 1024, 0], dtype=torch.int64, device=dev)
+    api.lod_append_kv(p, K, V, sl, kn, vn)
+    torch.cuda.synchronize()
+    K0[0, :, 4], V0[0, :, 4] = kn[0], vn[0]
+    K0[1, :, 1023], V0[1, :, 1023] = kn[1], vn[1]
+    assert torch.equal(K, K0) and torch.equal(V, V0)
+
+
 def test_zero_variance_decode_equals_dense():
     """Level of Detail Attention, How It Works: zero-variance groups give full
     attention -- checked on the GPU path directly against dense softmax."""
