@@ -145,9 +145,13 @@ struct BuildSmem {
   static constexpr size_t bytes = off_bar + 8;
 };
 
-// Keys of 256 bytes stay in registers at one CTA per SM; smaller ones fit two.
+// Two CTAs per SM where the packed key (up to 256 bytes, with up to 8
+// clusters; any count for 128-byte keys) fits in half the register file;
+// one otherwise.
 template <typename T, int D, int KMAX>
-__global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1) kmeans_kernel(BuildArgs a) {
+__global__ void __launch_bounds__(kBuildThreads,
+                                  (D * sizeof(T) <= 128 || (D * sizeof(T) <= 256 && KMAX <= 8)) ? 2 : 1)
+    kmeans_kernel(BuildArgs a) {
   constexpr int NW = kBuildWarps;
   constexpr int ROWB = D * (int)sizeof(T);
   constexpr int NWORD = D * (int)sizeof(T) / 4;  // packed 32-bit words per key
@@ -201,6 +205,14 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
     }
   }
   uint32_t kw[NWORD];
+  // Keeps the key packed: without it the compiler hoists the unpacked fp32
+  // key (twice the registers) out of the rounds, which halves the occupancy.
+  auto keep_packed = [&]() {
+    if constexpr (ROWB == 256) {
+#pragma unroll
+      for (int w = 0; w < NWORD; ++w) asm volatile("" : "+r"(kw[w]));
+    }
+  };
   {
     const uint4* row = reinterpret_cast<const uint4*>(Kc + (int64_t)(tid < n ? first + tid : first) * a.st);
 #pragma unroll
@@ -218,10 +230,15 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
     return;
   }
   auto xval = [&](int row, int d) { return Elem<T>::to_f(xs[row * D + d]); };
+  // dims 2p and 2p+1 of a staged key, one shared-memory load
+  auto xpair = [&](int row, int p) {
+    return pair_of<T>(reinterpret_cast<const uint32_t*>(xs + row * D), p);
+  };
 
   // ---- seeded farthest-first initialisation
   float mind = tid < n ? INFINITY : -INFINITY;
   for (int j = 0; j < k; ++j) {
+    keep_packed();
     int pick;
     if (j == 0) {
       // the initialisation's sequence-head index is model-wide under head sharding
@@ -266,6 +283,7 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
   // ---- Lloyd rounds
   int a_prev = -1;
   for (int it = 0; it < a.iters; ++it) {
+    keep_packed();
     int a_new = 0;
     if (tid < n) {
       float2 dot[KMAX];
@@ -331,17 +349,17 @@ __global__ void __launch_bounds__(kBuildThreads, (D * sizeof(T) <= 128) ? 2 : 1)
         const int m0 = off[j], m1 = off[j] + cj;
         int m = m0;
         for (; m + 3 < m1; m += 4) {
-          const int r0 = first + perm_s[m], r1 = first + perm_s[m + 1];
-          const int r2 = first + perm_s[m + 2], r3 = first + perm_s[m + 3];
-          s0.x += xval(r0, 2 * p); s0.y += xval(r0, 2 * p + 1);
-          s1.x += xval(r1, 2 * p); s1.y += xval(r1, 2 * p + 1);
-          s2.x += xval(r2, 2 * p); s2.y += xval(r2, 2 * p + 1);
-          s3.x += xval(r3, 2 * p); s3.y += xval(r3, 2 * p + 1);
+          const float2 x0 = xpair(first + perm_s[m], p), x1 = xpair(first + perm_s[m + 1], p);
+          const float2 x2 = xpair(first + perm_s[m + 2], p), x3 = xpair(first + perm_s[m + 3], p);
+          s0.x += x0.x; s0.y += x0.y;
+          s1.x += x1.x; s1.y += x1.y;
+          s2.x += x2.x; s2.y += x2.y;
+          s3.x += x3.x; s3.y += x3.y;
         }
         for (; m < m1; ++m) {
-          const int r0 = first + perm_s[m];
-          s0.x += xval(r0, 2 * p);
-          s0.y += xval(r0, 2 * p + 1);
+          const float2 x0 = xpair(first + perm_s[m], p);
+          s0.x += x0.x;
+          s0.y += x0.y;
         }
         const float sx = (s0.x + s1.x) + (s2.x + s3.x), sy = (s0.y + s1.y) + (s2.y + s3.y);
         cen2[p * KMAX + j] = make_float2(sx / (float)cj, sy / (float)cj);
@@ -489,7 +507,7 @@ template <typename T, int D, int KMAX>
 cudaError_t launch_kmeans_t(const BuildArgs& a, int64_t nchunks, int B, cudaStream_t stream) {
   const size_t smem = BuildSmem<T, D, KMAX>::bytes;
   auto kern = kmeans_kernel<T, D, KMAX>;
-  cudaError_t e = set_smem_once<kmeans_kernel<T, D, KMAX>>(smem);
+  cudaError_t e = set_smem_once<kmeans_kernel<T, D, KMAX>>(smem, true);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nchunks, (unsigned)a.Hkv, (unsigned)B);
   kern<<<grid, kBuildThreads, smem, stream>>>(a);

@@ -47,9 +47,11 @@ struct BuildArgs {
 
 // Opt kernel `Kern` in to `smem` bytes of dynamic shared memory, once per
 // device (later calls make no CUDA call, so launches stay capturable in a
-// graph).  The flag is per kernel: Kern is a template argument.
+// graph).  The flag is per kernel: Kern is a template argument.  max_shared:
+// also prefer the largest shared-memory carveout (for a kernel whose
+// occupancy is set by its shared memory).
 template <auto Kern>
-cudaError_t set_smem_once(size_t smem) {
+cudaError_t set_smem_once(size_t smem, bool max_shared = false) {
   static std::atomic<uint64_t> done{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -57,6 +59,8 @@ cudaError_t set_smem_once(size_t smem) {
   const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
   if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
   e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && max_shared)
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
   return e;
 }
