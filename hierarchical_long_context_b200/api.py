@@ -140,7 +140,8 @@ def lod_build_index(params: Params, K, V, chunk_begin: int, chunk_end: int, inde
 
 def lod_append_kv(params: Params, K, V, seq_lens, k_new, v_new, stream=None) -> None:
     """Write the current token's key/value rows k_new, v_new ([B, Hkv, d],
-    cache dtype) into K/V at positions seq_lens - 1 (one kernel)."""
+    cache dtype; on the device or in pinned host memory, which the kernel
+    reads directly) into K/V at positions seq_lens - 1 (one kernel)."""
     lib = load()
     st = _kv_strides(params, K, V)
     shape = (params.B, params.Hkv, params.d)
@@ -170,7 +171,10 @@ def lod_build_ready(params: Params, K, V, seq_lens, index: Index, ws=None, strea
 
 def lod_decode(params: Params, q, K, V, seq_lens, index: Index, out=None, lse=None, sel_groups=None,
                sel_pages=None, ws=None, stream=None):
-    """One decode step: q [B, Hq, d] at positions seq_lens - 1.  Returns out."""
+    """One decode step: q [B, Hq, d] at positions seq_lens - 1.  Returns out.
+
+    q and out may be pinned host tensors: the kernels then read q and store
+    out over the host link themselves (no separate copy)."""
     lib = load()
     st = _kv_strides(params, K, V)
     if q.shape != (params.B, params.Hq, params.d) or q.dtype != params.dtype or not q.is_contiguous():
@@ -178,9 +182,9 @@ def lod_decode(params: Params, q, K, V, seq_lens, index: Index, out=None, lse=No
     if seq_lens.dtype != torch.int64 or seq_lens.shape != (params.B,) or not seq_lens.is_cuda:
         raise ValueError("seq_lens must be a device int64 tensor [B]")
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=q.dtype, device=K.device)
     if ws is None:
-        ws = workspace(params, _lib.LOD_OP_DECODE, q.device)
+        ws = workspace(params, _lib.LOD_OP_DECODE, K.device)
     check("lod_decode", lib.lod_decode(
         ctypes.byref(params.c()), _ptr(q), _ptr(K), _ptr(V), st, _ptr(seq_lens),
         ctypes.byref(index.c()), _ptr(out), _ptr(lse), _ptr(sel_groups), _ptr(sel_pages), _ptr(ws),
@@ -198,9 +202,9 @@ def lod_prefill(params: Params, q, q_begin: int, K, V, index: Index, out=None, l
             or q.dtype != params.dtype or not q.is_contiguous():
         raise ValueError("q must be contiguous [B, Hq, Tq, d] of the cache dtype")
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=q.dtype, device=K.device)
     if ws is None:
-        ws = workspace(params, _lib.LOD_OP_PREFILL, q.device)
+        ws = workspace(params, _lib.LOD_OP_PREFILL, K.device)
     check("lod_prefill", lib.lod_prefill(
         ctypes.byref(params.c()), _ptr(q), q_begin, q.shape[2], _ptr(K), _ptr(V), st,
         ctypes.byref(index.c()), _ptr(out), _ptr(lse), _ptr(sel_groups), _ptr(sel_pages), _ptr(ws),

@@ -1,6 +1,8 @@
 // lod_api.cu -- the extern "C" entry points declared in include/lod.h:
 // argument validation, index and workspace sizing, and kernel launches.
 #include <atomic>
+#include <initializer_list>
+#include <utility>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -28,6 +30,41 @@ int32_t cuda_fail(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A per-call buffer the kernels read or write in place: memory of the current
+// device, managed memory, or page-locked host memory mapped at the same
+// address (cudaHostAlloc / cudaMallocHost under unified addressing: the
+// kernels then move its bytes over the host link themselves).  Pageable host
+// memory and another device's memory are refused before anything is enqueued.
+int32_t check_visible(const void* ptr, const char* name) {
+  if (!ptr) return LOD_OK;
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, ptr);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(LOD_EINVAL, "%s: pointer not known to CUDA (%s)", name, cudaGetErrorString(e));
+  }
+  if (at.type == cudaMemoryTypeUnregistered)
+    return fail(LOD_EINVAL, "%s is pageable host memory: pass device or page-locked host memory", name);
+  if (at.type == cudaMemoryTypeHost && at.devicePointer != ptr)
+    return fail(LOD_EINVAL, "%s: page-locked host memory not mapped at its host address", name);
+  if (at.type == cudaMemoryTypeDevice) {
+    int dev = -1;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (at.device != dev) return fail(LOD_EINVAL, "%s is memory of device %d, not the current device %d", name,
+                                      at.device, dev);
+  }
+  return LOD_OK;
+}
+
+int32_t check_visible_all(std::initializer_list<std::pair<const void*, const char*>> bufs) {
+  for (const auto& b : bufs) {
+    const int32_t rc = check_visible(b.first, b.second);
+    if (rc) return rc;
+  }
+  return LOD_OK;
+}
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -368,6 +405,8 @@ int32_t lod_append_kv(const lod_params* p, void* K, void* V, const int64_t kv_st
   if (rc) return rc;
   if (!seq_lens || !k_new || !v_new) return fail(LOD_EINVAL, "seq_lens, k_new and v_new must be non-NULL");
   if (!aligned16(k_new) || !aligned16(v_new)) return fail(LOD_EINVAL, "k_new and v_new must be 16-byte aligned");
+  rc = check_visible_all({{seq_lens, "seq_lens"}, {k_new, "k_new"}, {v_new, "v_new"}});
+  if (rc) return rc;
   cudaError_t e = lod::launch_append(K, V, kv_strides, (int)elem_bytes(p), p->d, seq_lens, k_new, v_new, p->B,
                                      p->Hkv, p->Tmax, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
@@ -403,6 +442,9 @@ int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void
   const AttendShape s = decode_shape(p);
   if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
     return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
+  rc = check_visible_all({{q, "q"}, {out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
+                          {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}});
+  if (rc) return rc;
   lod::AttendArgs a;
   fill_attend(a, p, s, K, V, kv_strides, index, ws);
   a.q = q;
@@ -441,6 +483,9 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   const AttendShape s = prefill_shape(p);
   if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
     return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
+  rc = check_visible_all({{q, "q"}, {out, "out"}, {lse, "lse"}, {sel_groups, "sel_groups"},
+                          {sel_pages, "sel_pages"}});
+  if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   // 1) index of every chunk completed inside the query range (a pure function of K/V)
   const int64_t c0 = q_begin / p->chunk, c1 = (q_begin + Tq) / p->chunk;
@@ -560,6 +605,9 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
                 "decode scratch of %zu bytes exceeds the built-in %zu-byte array of lod_decode_noalloc "
                 "(fewer sequences, KV heads or a smaller Tmax fit; otherwise use lod_decode)",
                 need, kLodNoallocScratchBytes);
+  rc = check_visible_all({{q, "q"}, {out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
+                          {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}, {status, "status"}});
+  if (rc) return rc;
   void* ws = nullptr;
   rc = noalloc_scratch(&ws);
   if (rc) return rc;

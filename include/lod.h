@@ -14,7 +14,15 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every pointer named as "device" must be CUDA device memory (or managed
- *    memory) on the current device; host pointers are marked "host".
+ *    memory) on the current device; host pointers are marked "host".  The
+ *    per-call buffers (q, out, lse, sel_groups, sel_pages, seq_lens, k_new,
+ *    v_new, status) may also be page-locked host memory mapped at its host
+ *    address (cudaHostAlloc / cudaMallocHost under unified addressing): the
+ *    kernels then read or write those bytes over the host link themselves,
+ *    with no separate copy.  The entry points check these buffers and refuse
+ *    pageable host memory and another device's memory (LOD_EINVAL) before
+ *    anything is enqueued.  The KV cache, the index and the workspace must
+ *    be device memory.
  *  - The caller owns every buffer.  The library never allocates or frees
  *    device memory and never synchronises the stream, with one exception:
  *    lod_get_status() copies 4 bytes to the host and waits for them.

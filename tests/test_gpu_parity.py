@@ -332,6 +332,43 @@ def test_append_kv_writes_the_current_rows_only():
     assert torch.equal(K, K0) and torch.equal(V, V0)
 
 
+def test_pinned_host_buffers_are_used_in_place():
+    """q, the new K/V rows and out in pinned host memory: the kernels read and
+    write them directly, with the device buffers' result; pageable host memory
+    and another device's memory are refused before anything is enqueued."""
+    from hierarchical_long_context_b200 import _lib
+    w = synth.WORKLOADS["decode_gqa_32k_bf16"].with_(B=2, Hq=16, Hkv=2, T=4096)
+    p, Kc, Vc, Kd, Vd = _setup(w)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, w.T // 256, ix)
+    q = synth.decode_queries(w).cuda()
+    sl = torch.full((w.B,), w.T, dtype=torch.int64, device="cuda")
+    ref = api.lod_decode(p, q, Kd, Vd, sl, ix)
+    hq = q.cpu().pin_memory()
+    hout = torch.zeros(q.shape, dtype=q.dtype).pin_memory()
+    api.lod_decode(p, hq, Kd, Vd, sl, ix, out=hout)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())
+    g = torch.Generator().manual_seed(3)
+    kn = torch.randn(w.B, w.Hkv, w.d, generator=g).to(w.torch_dtype).pin_memory()
+    vn = torch.randn(w.B, w.Hkv, w.d, generator=g).to(w.torch_dtype).pin_memory()
+    K2, V2 = Kd.clone(), Vd.clone()
+    api.lod_append_kv(p, K2, V2, sl, kn, vn)
+    torch.cuda.synchronize()
+    assert torch.equal(K2[:, :, w.T - 1].cpu(), kn) and torch.equal(V2[:, :, w.T - 1].cpu(), vn)
+    assert torch.equal(K2[:, :, :w.T - 1], Kd[:, :, :w.T - 1])
+    # refused: pageable host memory (no kernel is launched for these calls)
+    pageable_q, pageable_out, pageable_k = q.cpu(), torch.zeros(q.shape, dtype=q.dtype), kn.clone()
+    assert not pageable_q.is_pinned() and not pageable_k.is_pinned()
+    for call in (lambda: api.lod_decode(p, pageable_q, Kd, Vd, sl, ix, out=hout),
+                 lambda: api.lod_decode(p, hq, Kd, Vd, sl, ix, out=pageable_out),
+                 lambda: api.lod_append_kv(p, K2, V2, sl, pageable_k, vn)):
+        with pytest.raises(_lib.LodError) as e:
+            call()
+        assert e.value.code == _lib.LOD_EINVAL and "pageable" in str(e.value)
+    assert torch.equal(pageable_out, torch.zeros_like(pageable_out))
+
+
 def test_zero_variance_decode_equals_dense():
     """Level of Detail Attention, How It Works: zero-variance groups give full
     attention -- checked on the GPU path directly against dense softmax."""
