@@ -134,8 +134,8 @@ struct BuildSmem {
   static constexpr size_t off_x = 0;                                        // T [256][D]
   static constexpr size_t off_cen = (size_t)kChunk * D * sizeof(T);         // float2 [D/2][KMAX]
   static constexpr size_t off_psum = off_cen + sizeof(float) * D * KMAX;    // float [PMAX][D] value sums
-  static constexpr size_t off_cn = off_psum + sizeof(float) * PMAX * D;     // float [KMAX]
-  static constexpr size_t off_red = off_cn + sizeof(float) * KMAX;          // float/int [NW+1] x 2
+  static constexpr size_t off_cn = off_psum + sizeof(float) * PMAX * D;     // float [KMAX][D/64] norm parts
+  static constexpr size_t off_red = off_cn + sizeof(float) * KMAX * (D / 64);  // float/int [NW+1] x 2
   static constexpr size_t off_wc = off_red + 8 * (kBuildWarps + 1);         // int [NW][KMAX]
   static constexpr size_t off_cnt = off_wc + 4 * kBuildWarps * KMAX;        // int [KMAX]
   static constexpr size_t off_off = off_cnt + 4 * KMAX;                     // int [KMAX+1]
@@ -265,19 +265,16 @@ __global__ void __launch_bounds__(kBuildThreads,
       mind = fminf(mind, dd);
     }
   }
-  auto norms = [&]() {
-    for (int j = warp; j < k; j += NW) {
-      float s = 0.f;
-      for (int p = lane; p < NP; p += 32) {
-        const float2 cc = cen2[p * KMAX + j];
-        s = fmaf(cc.x, cc.x, s);
-        s = fmaf(cc.y, cc.y, s);
-      }
-      s = warp_sum(s);
-      if (lane == 0) cnorm[j] = s;
-    }
+  // ||c_j||^2 in D/64 parts of 32 dimension pairs: item (j, p) = j * NP + p;
+  // the 32 items of a warp belong to one cluster (NP is a multiple of 32)
+  constexpr int NSLOT = NP / 32;
+  static_assert(NP % 32 == 0, "dimension pairs per warp");
+  auto norm_part = [&](int item, float2 cc) {
+    const float s = warp_sum(fmaf(cc.x, cc.x, cc.y * cc.y));
+    if (lane == 0) cnorm[item >> 5] = s;
   };
-  norms();
+  for (int item = tid; item < k * NP; item += kBuildThreads)
+    norm_part(item, cen2[(item % NP) * KMAX + item / NP]);
   __syncthreads();
 
   // ---- Lloyd rounds
@@ -296,11 +293,17 @@ __global__ void __launch_bounds__(kBuildThreads,
         for (int j = 0; j < KMAX; ++j)
           if (j < k) dot[j] = ffma2(x, cen2[p * KMAX + j], dot[j]);
       }
-      float best = fmaf(-2.f, dot[0].x + dot[0].y, cnorm[0]);
+      auto cn = [&](int j) {
+        float v = cnorm[j * NSLOT];
+#pragma unroll
+        for (int t = 1; t < NSLOT; ++t) v += cnorm[j * NSLOT + t];
+        return v;
+      };
+      float best = fmaf(-2.f, dot[0].x + dot[0].y, cn(0));
 #pragma unroll
       for (int j = 1; j < KMAX; ++j) {
         if (j < k) {
-          const float dj = fmaf(-2.f, dot[j].x + dot[j].y, cnorm[j]);
+          const float dj = fmaf(-2.f, dot[j].x + dot[j].y, cn(j));
           if (dj < best) {  // strict: ties keep the lower cluster id
             best = dj;
             a_new = j;
@@ -308,42 +311,44 @@ __global__ void __launch_bounds__(kBuildThreads,
         }
       }
     }
-    const int changed = __syncthreads_or(tid < n && a_new != a_prev);
-    if (it > 0 && !changed) break;  // fixed point: later rounds repeat this one exactly
-    a_prev = a_new;
-
-    // stable counting sort of members by cluster (ascending local index)
+    // stable counting sort of members by cluster (ascending local index):
+    // each warp's per-cluster counts, published by the change test's barrier
     int rank = 0;
     for (int j = 0; j < k; ++j) {
       const unsigned m = __ballot_sync(0xffffffffu, tid < n && a_new == j);
       if (lane == 0) wcnt[warp * KMAX + j] = __popc(m);
       if (tid < n && a_new == j) rank = __popc(m & ((1u << lane) - 1u));
     }
-    __syncthreads();
-    if (tid == 0) {
-      int o = 0;
+    const int changed = __syncthreads_or(tid < n && a_new != a_prev);
+    if (it > 0 && !changed) break;  // fixed point: later rounds repeat this one exactly
+    a_prev = a_new;
+    {  // every thread takes its slot from the counts (cluster-major, then warp, then lane)
+      int o = 0, slot = 0;
       for (int j = 0; j < k; ++j) {
-        off[j] = o;
-        int cj = 0;
+        int cj = 0, before = 0;
         for (int w = 0; w < NW; ++w) {
           const int t = wcnt[w * KMAX + j];
-          wcnt[w * KMAX + j] = o + cj;  // becomes the warp's base offset for cluster j
+          before += w < warp ? t : 0;
           cj += t;
         }
-        cnt[j] = cj;
+        if (j == a_new) slot = o + before + rank;
+        if (tid == j) {
+          off[j] = o;
+          cnt[j] = cj;
+        }
         o += cj;
       }
-      off[k] = o;
+      if (tid == 0) off[k] = o;
+      if (tid < n) perm_s[slot] = tid;
     }
-    __syncthreads();
-    if (tid < n) perm_s[wcnt[warp * KMAX + a_new] + rank] = tid;
     __syncthreads();
 
     // centroid := member mean (fp32, fixed order: four interleaved partial sums);
-    // empty clusters keep theirs
+    // empty clusters keep theirs; then the centroid's norm parts
     for (int item = tid; item < k * NP; item += kBuildThreads) {
       const int j = item / NP, p = item % NP;
       const int cj = cnt[j];
+      float2 cc = cen2[p * KMAX + j];
       if (cj > 0) {
         float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
         const int m0 = off[j], m1 = off[j] + cj;
@@ -362,11 +367,11 @@ __global__ void __launch_bounds__(kBuildThreads,
           s0.y += x0.y;
         }
         const float sx = (s0.x + s1.x) + (s2.x + s3.x), sy = (s0.y + s1.y) + (s2.y + s3.y);
-        cen2[p * KMAX + j] = make_float2(sx / (float)cj, sy / (float)cj);
+        cc = make_float2(sx / (float)cj, sy / (float)cj);
+        cen2[p * KMAX + j] = cc;
       }
+      norm_part(item, cc);
     }
-    __syncthreads();
-    norms();
     __syncthreads();
   }
 
