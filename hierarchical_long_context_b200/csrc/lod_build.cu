@@ -533,6 +533,9 @@ cudaError_t launch_kmeans_d(const BuildArgs& a, int64_t nchunks, int B, cudaStre
 // One CTA per sequence; 16-byte copies.
 __global__ void append_kv_kernel(uint4* K, uint4* V, int64_t sb, int64_t sh, int64_t st, const int64_t* seq_lens,
                                  const uint4* kn, const uint4* vn, int Hkv, int row16, int64_t Tmax) {
+  // the next kernel (a decode launched as a programmatic dependent) may start
+  // its input-free set-up now; it reads the cache only after this grid is done
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int64_t t = seq_lens[b] - 1;
   if (t < 0 || t >= Tmax) return;

@@ -70,6 +70,7 @@ template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ AttendArgs a) {
   static_assert(NQ <= 8, "query rows per unit");
+  static_assert(N * (D / 8) % kSoftThreads == 0, "query pieces per softmax thread");
   const int64_t u = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -146,6 +147,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (it waits for this grid's completion before reading what it writes)
   pdl_wait();
   pdl_launch_dependents();
+
+  // the query rows' loads go out first: which rows exist does not depend on
+  // the sequence length, so they overlap its read (rows of an invalid
+  // sequence are zeroed below)
+  constexpr int kQPer = N * (D / 8) / kSoftThreads;  // 16-byte pieces per softmax thread
+  uint4 qv[kQPer];
+  if (warp >= 2) {
+    const int t = tid - 64;
+#pragma unroll
+    for (int i = 0; i < kQPer; ++i) {
+      const int c2 = t + i * kSoftThreads;
+      const int r = c2 / (D / 8), c = c2 % (D / 8);
+      const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
+      const bool row = r < NQ && (a.seq_lens ? r < a.g : (r < a.g * a.NP && pi < a.pos_hi));
+      qv[i] = make_uint4(0, 0, 0, 0);
+      if (row) {
+        const int hq = kvh * a.g + (r % a.g);
+        qv[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                      (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
+      }
+    }
+  }
 
   int64_t t_row[NQ];
   bool ok[NQ];
@@ -229,19 +252,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp >= 2) {
     const int t = tid - 64;
-    for (int c2 = t; c2 < N * (D / 8); c2 += kSoftThreads) {
+#pragma unroll
+    for (int i = 0; i < kQPer; ++i) {
+      const int c2 = t + i * kSoftThreads;
       const int r = c2 / (D / 8), c = c2 % (D / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
       bool okr = false;
 #pragma unroll
       for (int x = 0; x < NQ; ++x)
         if (x == r) okr = ok[x];
-      if (r < NQ && okr) {
-        const int hq = kvh * a.g + (r % a.g);
-        const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
-        v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                  (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
-      }
+      const uint4 v = okr ? qv[i] : make_uint4(0, 0, 0, 0);
       const uint32_t off = (uint32_t)((c >> 3) * (N * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
       *reinterpret_cast<uint4*>(Qs + off) = v;
     }
