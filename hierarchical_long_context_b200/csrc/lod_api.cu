@@ -36,7 +36,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // address (cudaHostAlloc / cudaMallocHost under unified addressing: the
 // kernels then move its bytes over the host link themselves).  Pageable host
 // memory and another device's memory are refused before anything is enqueued.
-int32_t check_visible(const void* ptr, const char* name) {
+int32_t check_visible(const void* ptr, const char* name, int* host = nullptr) {
+  if (host) *host = 0;
   if (!ptr) return LOD_OK;
   cudaPointerAttributes at;
   cudaError_t e = cudaPointerGetAttributes(&at, ptr);
@@ -48,6 +49,7 @@ int32_t check_visible(const void* ptr, const char* name) {
     return fail(LOD_EINVAL, "%s is pageable host memory: pass device or page-locked host memory", name);
   if (at.type == cudaMemoryTypeHost && at.devicePointer != ptr)
     return fail(LOD_EINVAL, "%s: page-locked host memory not mapped at its host address", name);
+  if (host) *host = at.type == cudaMemoryTypeHost;
   if (at.type == cudaMemoryTypeDevice) {
     int dev = -1;
     e = cudaGetDevice(&dev);
@@ -442,12 +444,15 @@ int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void
   const AttendShape s = decode_shape(p);
   if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
     return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
-  rc = check_visible_all({{q, "q"}, {out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
-                          {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}});
+  int q_host = 0;
+  rc = check_visible(q, "q", &q_host);
+  if (!rc) rc = check_visible_all({{out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
+                                   {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}});
   if (rc) return rc;
   lod::AttendArgs a;
   fill_attend(a, p, s, K, V, kv_strides, index, ws);
   a.q = q;
+  a.q_host = q_host;
   a.Tq = 1;
   a.q_begin = 0;
   a.seq_lens = seq_lens;
@@ -483,8 +488,10 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   const AttendShape s = prefill_shape(p);
   if (!ws || !aligned16(ws) || ws_bytes < attend_ws_bytes(p, s))
     return fail(LOD_EINVAL, "workspace too small (%zu < %zu) or misaligned", ws_bytes, attend_ws_bytes(p, s));
-  rc = check_visible_all({{q, "q"}, {out, "out"}, {lse, "lse"}, {sel_groups, "sel_groups"},
-                          {sel_pages, "sel_pages"}});
+  int q_host = 0;
+  rc = check_visible(q, "q", &q_host);
+  if (!rc) rc = check_visible_all({{out, "out"}, {lse, "lse"}, {sel_groups, "sel_groups"},
+                                   {sel_pages, "sel_pages"}});
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   // 1) index of every chunk completed inside the query range (a pure function of K/V)
@@ -497,6 +504,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   lod::AttendArgs a;
   fill_attend(a, p, s, K, V, kv_strides, index, ws);
   a.q = q;
+  a.q_host = q_host;
   a.Tq = Tq;
   a.q_begin = q_begin;
   a.seq_lens = nullptr;
@@ -605,8 +613,10 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
                 "decode scratch of %zu bytes exceeds the built-in %zu-byte array of lod_decode_noalloc "
                 "(fewer sequences, KV heads or a smaller Tmax fit; otherwise use lod_decode)",
                 need, kLodNoallocScratchBytes);
-  rc = check_visible_all({{q, "q"}, {out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
-                          {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}, {status, "status"}});
+  int q_host = 0;
+  rc = check_visible(q, "q", &q_host);
+  if (!rc) rc = check_visible_all({{out, "out"}, {seq_lens, "seq_lens"}, {lse, "lse"},
+                                   {sel_groups, "sel_groups"}, {sel_pages, "sel_pages"}, {status, "status"}});
   if (rc) return rc;
   void* ws = nullptr;
   rc = noalloc_scratch(&ws);
@@ -622,6 +632,7 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
   fill_attend(a, p, s, K, V, kv_strides, index, ws);
   if (status) a.status = status;
   a.q = q;
+  a.q_host = q_host;
   a.Tq = 1;
   a.q_begin = 0;
   a.seq_lens = seq_lens;

@@ -97,6 +97,7 @@ constexpr int kScanSlab = 64;
 //           unit is head (r % g) at position block*NP + r / g.
 struct AttendArgs {
   const void* q;            // [B][Hq][Tq][d]
+  int q_host;               // 1: q is mapped page-locked host memory (read over the host link)
   int64_t Tq;               // positions per sequence in q/out (1 for decode)
   int64_t q_begin;          // position of q's first row (prefill)
   const int64_t* seq_lens;  // decode: device [B]; prefill: null

@@ -148,26 +148,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  // the query rows' loads go out first: which rows exist does not depend on
-  // the sequence length, so they overlap its read (rows of an invalid
-  // sequence are zeroed below)
+  // query piece i of this softmax thread (16 bytes; zero for a missing row)
   constexpr int kQPer = N * (D / 8) / kSoftThreads;  // 16-byte pieces per softmax thread
+  auto load_q = [&](int i) {
+    const int c2 = (tid - 64) + i * kSoftThreads;
+    const int r = c2 / (D / 8), c = c2 % (D / 8);
+    const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
+    const bool row = r < NQ && (a.seq_lens ? r < a.g : (r < a.g * a.NP && pi < a.pos_hi));
+    if (!row) return make_uint4(0, 0, 0, 0);
+    const int hq = kvh * a.g + (r % a.g);
+    return __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                 (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
+  };
+  // q in host memory: its loads go out first (which rows exist does not
+  // depend on the sequence length, so they overlap its read; rows of an
+  // invalid sequence are zeroed below); q in device memory is read after
   uint4 qv[kQPer];
-  if (warp >= 2) {
-    const int t = tid - 64;
 #pragma unroll
-    for (int i = 0; i < kQPer; ++i) {
-      const int c2 = t + i * kSoftThreads;
-      const int r = c2 / (D / 8), c = c2 % (D / 8);
-      const int64_t pi = a.seq_lens ? 0 : a.pos_lo + blk * a.NP + r / a.g;
-      const bool row = r < NQ && (a.seq_lens ? r < a.g : (r < a.g * a.NP && pi < a.pos_hi));
-      qv[i] = make_uint4(0, 0, 0, 0);
-      if (row) {
-        const int hq = kvh * a.g + (r % a.g);
-        qv[i] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                      (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
-      }
-    }
+  for (int i = 0; i < kQPer; ++i) qv[i] = make_uint4(0, 0, 0, 0);
+  if (warp >= 2 && a.q_host) {
+#pragma unroll
+    for (int i = 0; i < kQPer; ++i) qv[i] = load_q(i);
   }
 
   int64_t t_row[NQ];
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int x = 0; x < NQ; ++x)
         if (x == r) okr = ok[x];
+      if (okr && !a.q_host) qv[i] = load_q(i);
       const uint4 v = okr ? qv[i] : make_uint4(0, 0, 0, 0);
       const uint32_t off = (uint32_t)((c >> 3) * (N * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
       *reinterpret_cast<uint4*>(Qs + off) = v;
