@@ -561,8 +561,9 @@ int32_t lod_get_status(void* ws, lod_stream_t stream, uint32_t* status) {
 // library.  The array is `static __device__`, so each GPU that loads this
 // library holds its kLodNoallocScratchBytes until the process exits.  Host
 // code cannot use the array's name as an address; the device address is
-// looked up once per device with cudaGetSymbolAddress, with that device
-// current, on the first call made on that device.
+// looked up with cudaGetSymbolAddress, with that device current, on the
+// first call made on that device (and again whenever the device's current
+// context has changed since, as after cudaDeviceReset).
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -570,25 +571,50 @@ constexpr size_t kLodNoallocScratchBytes = LOD_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kLodNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;
+// Per device: the context the address was looked up in, and the address.
+// A context that is destroyed and created again (cudaDeviceReset, or a
+// driver-API context switch) maps the array at a new address, so the cached
+// one is used only while the device's current context is the same.
 void* g_noalloc_ptr[kMaxDevices] = {};
-std::atomic<int> g_noalloc_ready[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of this device's copy of the scratch array (set-up on first use).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
+
+// The calling thread's current context (null when none is current yet).
+int32_t current_context(CUcontext* ctx) {
+  std::call_once(g_ctx_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  });
+  if (!g_ctx_current) return fail(LOD_ECUDA, "cuCtxGetCurrent is not available from the driver");
+  if (g_ctx_current(ctx) != CUDA_SUCCESS) return fail(LOD_ECUDA, "cuCtxGetCurrent failed");
+  return LOD_OK;
+}
+
+// Device address of the current device's copy of the scratch array, looked
+// up on the first call made in the device's current context.
 int32_t noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(LOD_EUNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
-  if (!g_noalloc_ready[dev].load(std::memory_order_acquire)) {
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ready[dev].load(std::memory_order_relaxed)) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
-      g_noalloc_ptr[dev] = p;
-      g_noalloc_ready[dev].store(1, std::memory_order_release);
-    }
+  CUcontext ctx = nullptr;
+  int32_t rc = current_context(&ctx);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (ctx == nullptr || ctx != g_noalloc_ctx[dev] || g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    rc = current_context(&ctx);  // the lookup made the device's primary context current if none was
+    if (rc) return rc;
+    g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return LOD_OK;
@@ -606,6 +632,7 @@ extern "C" int32_t lod_decode_noalloc(const lod_params* p, const void* q, const 
   if (rc) return rc;
   if (!q || !out || !seq_lens) return fail(LOD_EINVAL, "q, out and seq_lens must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(LOD_EINVAL, "q and out must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(status) & 3u) return fail(LOD_EINVAL, "status must be 4-byte aligned");
   const AttendShape s = decode_shape(p);
   const size_t need = attend_ws_bytes(p, s);
   if (need > kLodNoallocScratchBytes)

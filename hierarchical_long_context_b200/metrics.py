@@ -108,15 +108,31 @@ def prefill_flops(p, q_begin: int, Tq: int) -> float:
 
 
 def build_bytes(p, nchunks: int) -> int:
-    """Bytes of one lod_build_index call over chunks [0, nchunks) of every
-    sequence: read K and V once, write the summaries, counts, offsets, member
-    lists and the member-ordered K/V copies (every clustered token once)."""
+    """Algorithmic bytes of one lod_build_index call over chunks [0, nchunks)
+    of every sequence: the method's own reads and writes -- K and V read
+    once, the group and page summaries, counts, page offsets, group page
+    ranges and the member list written once."""
     e = 4 if str(p.dtype).endswith("float32") else 2
     units = p.B * p.Hkv
     k, P, C, d = p.clusters, p.page_slots, p.chunk, p.d
     per_chunk = 2 * C * d * e + 2 * k * d * e + k * 4 + 2 * P * d * e + P * (4 + 2) + (k + 1) * 2 + C * 2
-    copies = 2 * (nchunks * C - (p.sinks if nchunks else 0)) * d * e
-    return units * (nchunks * per_chunk + copies)
+    return units * nchunks * per_chunk
+
+
+def build_design_bytes(p, nchunks: int) -> int:
+    """Bytes the build writes beyond the method's own: the member-ordered K/V
+    copies (every clustered token once, cache dtype; with kv_bits = 4 the
+    4-bit codes and the per-page (scale, low) quantisers instead) and the
+    packed group words.  These serve the decode's contiguous page reads."""
+    e = 4 if str(p.dtype).endswith("float32") else 2
+    units = p.B * p.Hkv
+    k, P, C, d = p.clusters, p.page_slots, p.chunk, p.d
+    toks = nchunks * C - (p.sinks if nchunks else 0)
+    if p.kv_bits == 4:
+        copies = 2 * toks * (d // 2) + 2 * nchunks * P * d * 8
+    else:
+        copies = 2 * toks * d * e
+    return units * (copies + nchunks * k * 4)
 
 
 def build_flops(p, nchunks: int) -> float:

@@ -305,15 +305,19 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
  *     Shapes whose scratch (lod_workspace_bytes(LOD_OP_DECODE)) exceeds it
  *     are rejected with LOD_EINVAL and a message naming both sizes; nothing
  *     is enqueued then.  (The 128K-context decode of 4 sequences x 8 KV heads
- *     x 8 query heads per KV head needs about 3.3 MB.)
- *   - status: nullable device pointer to a uint32_t that receives (bitwise
- *     OR) this call's LOD_ST_* bits; the caller zeroes it.  When NULL the
+ *     x 8 query heads per KV head needs about 4.7 MB; a 1M-context decode of
+ *     one sequence with the same heads needs about 9.0 MB, more than the
+ *     array holds, and must use lod_decode.)
+ *   - status: nullable device pointer to a 4-byte aligned uint32_t that
+ *     receives (bitwise OR) this call's LOD_ST_* bits; the caller zeroes it
+ *     (a misaligned pointer is rejected with LOD_EINVAL).  When NULL the
  *     bits are recorded in the built-in array and not reported.
  * No device memory is allocated or freed by this call, by the library or by
  * any library it calls.  The first call on each device looks up that
  * device's address of the built-in array (cudaGetSymbolAddress, with that
- * device current); make the first call on a device outside any stream
- * capture.  All calls on one device share the one array and it keeps the
+ * device current), and so does the first call after the device's current
+ * context has changed (after cudaDeviceReset, or a context switch through
+ * the driver API); make those calls outside any stream capture.  All calls on one device share the one array and it keeps the
  * last call's contents: calls whose executions can overlap on the GPU
  * (different streams without ordering, or concurrent host threads) race on
  * it and produce undefined results.  Order them on one stream.

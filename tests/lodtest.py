@@ -226,9 +226,10 @@ def compare_builds(gu: dict, ou: dict, cfg: oracle.Config, bf16: bool) -> dict:
             np.testing.assert_array_equal(gu["pCnt"][c * P:(c + 1) * P], ou["pCnt"][c * P:(c + 1) * P])
             for key, n in (("gK", k), ("gV", k), ("pK", P), ("pV", P)):
                 g_, o_ = gu[key][c * n:(c + 1) * n], ou[key][c * n:(c + 1) * n]
-                # both sides round an fp32 sum (taken in different orders) to
-                # bf16: the results may straddle a rounding boundary and differ
-                # by one bf16 ulp, at most 2^-7 of the value
+                # the GPU rounds an fp32 sum and the oracle an fp64 sum of the
+                # same members to bf16: the two sums differ by fp32 rounding,
+                # so the results may straddle a rounding boundary and differ by
+                # one bf16 ulp, at most 2^-7 of the value
                 tol = (2.0 ** -7 * np.abs(o_) + 1e-6) if bf16 else (2e-6 * np.abs(o_) + 1e-6)
                 assert np.all(np.abs(g_ - o_) <= tol), (c, key)
     return stats
@@ -244,13 +245,30 @@ def check_rows(cfg: oracle.Config, dtype: str, K: np.ndarray, V: np.ndarray, u: 
 
     qk = dict(kq=u["kq"], vq=u["vq"]) if "kq" in u else {}
 
+    def gscore(q, gid):
+        return float(np.dot(q.astype(np.float64), u["gK"][gid])) * sc
+
+    def check_order(q, t, sg, gsg):
+        """The ABI's order of sel_groups: the opened groups best first, then
+        -1 padding; as many opened groups as the oracle opens.  Neighbours
+        may swap only within a score tie (TIE)."""
+        gsg = np.asarray(gsg)
+        nv = int((np.asarray(sg) >= 0).sum())
+        assert np.all(gsg[:nv] >= 0) and np.all(gsg[nv:] == -1), (t, gsg, sg)
+        s = [gscore(q, int(x)) for x in gsg[:nv]]
+        for i in range(nv - 1):
+            assert s[i] >= s[i + 1] - TIE, (t, gsg, s)
+            if s[i] == s[i + 1]:
+                assert gsg[i] < gsg[i + 1], (t, gsg)
+
     def one(row):
         q, t, gout, glse, gsg, gsp = row
         out, lse, sg, sp, st = oracle.attend_row(cfg, q, t, K, V, u, **qk)
+        check_order(q, t, sg, gsg)
         forced = False
         if not (np.array_equal(np.sort(sg), np.sort(gsg))):
             # differing opened groups must be score ties within TIE
-            s = lambda gid: float(np.dot(q.astype(np.float64), u["gK"][gid])) * sc
+            s = lambda gid: gscore(q, gid)
             og = [x for x in sg if x >= 0 and x not in gsg]
             gg = [x for x in gsg if x >= 0 and x not in sg]
             assert len(og) == len(gg), (sg, gsg)

@@ -79,5 +79,10 @@ def test_build_bytes_by_hand():
                  + 18 * (4 + 2)          # page counts and offsets
                  + 3 * 2                 # group page ranges
                  + 256 * 2)              # member list
+    assert metrics.build_bytes(p, 2) == 2 * per_chunk == 283892
     copies = 2 * (2 * 256 - 1) * 64 * 4  # member-ordered K and V, sinks excluded
-    assert metrics.build_bytes(p, 2) == 2 * per_chunk + copies == 545524
+    words = 2 * 2 * 4                    # packed group words (2 chunks x 2 groups)
+    assert metrics.build_design_bytes(p, 2) == copies + words == 261648
+    # three-tier INT4: 32 + 32 bytes of codes per token, (scale, low) per slot and channel
+    p4 = _params(kv_bits=4)
+    assert metrics.build_design_bytes(p4, 2) == 2 * 511 * 32 + 2 * 2 * 18 * 64 * 8 + words
