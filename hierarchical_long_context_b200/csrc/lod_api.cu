@@ -207,7 +207,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
 int32_t encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides_bytes) {
+                   const cuuint64_t* strides_bytes, cuuint32_t box_rows = 128) {
   std::call_once(g_encode_once, [] {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
@@ -216,7 +216,7 @@ int32_t encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t*
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
   if (!g_encode) return fail(LOD_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint32_t box4[4] = {64, 128, 1, 1};
+  const cuuint32_t box4[4] = {64, box_rows, 1, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
                         strides_bytes, box4, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -237,6 +237,97 @@ int32_t make_tc_maps(const lod_params* p, const void* K, const void* V, const in
   const cuuint64_t kstr[3] = {(cuuint64_t)kv[2] * 2, (cuuint64_t)kv[1] * 2, (cuuint64_t)kv[0] * 2};
   if (!rc) rc = encode_map(&m->K, K, 4, kdims, kstr);
   if (!rc) rc = encode_map(&m->V, V, 4, kdims, kstr);
+  return rc;
+}
+
+// ---------------------------------------------------------------- grouped prefill
+
+// The grouped tensor-core prefill runs for bf16 caches with d = 128 and the
+// cache-dtype member copies (kv_bits = 0), when every row index it forms
+// fits in 32 bits.
+bool use_tc_prefill(const lod_params* p) {
+  const int64_t Cmax = p->Tmax / p->chunk;
+  return use_tc(p) && p->kv_bits == 0 && (int64_t)p->B * p->Hkv * p->Tmax < ((int64_t)1 << 31) &&
+         (int64_t)p->B * p->Hkv * Cmax * page_slots(p) < ((int64_t)1 << 31);
+}
+
+constexpr int kItemRows = 1024;                    // pairs per work item of the pair kernel
+constexpr int64_t kPrefillWaveBudget = (int64_t)1 << 30;  // workspace bytes a wave may use
+
+// Workspace bytes per wave row: state (132 floats), and per opened group
+// its id, its place in the group's run, its log-sum-exp, its bf16 output and
+// its pair-list entry.
+int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 2 * p->d + 4); }
+
+// Query positions per wave: a multiple of chunk, as many as the budget allows
+// (at least one chunk, at most 64), never more than the cache holds.
+int64_t pf_wave(const lod_params* p) {
+  const int64_t rows = (int64_t)p->B * p->Hq;
+  int64_t nw = kPrefillWaveBudget / (rows * pf_row_bytes(p)) / p->chunk * p->chunk;
+  const int64_t most = (((int64_t)1 << 31) - 1) / (rows * p->top_groups) / p->chunk * p->chunk;
+  if (nw > most) nw = most;
+  if (nw > 64 * (int64_t)p->chunk) nw = 64 * (int64_t)p->chunk;
+  if (nw > p->Tmax) nw = p->Tmax;
+  if (nw < p->chunk) nw = p->chunk;
+  return nw;
+}
+
+struct PfLayout {
+  size_t state, sel, pos, plse, po, list, cnt, off, items, n_items, total;
+  int64_t NW, Gtot, max_items;
+};
+
+PfLayout pf_layout(const lod_params* p) {
+  PfLayout L;
+  L.NW = pf_wave(p);
+  const int64_t rows = (int64_t)p->B * p->Hq * L.NW;
+  const int64_t pairs = rows * p->top_groups;
+  L.Gtot = (int64_t)p->B * p->Hkv * (p->Tmax / p->chunk) * p->clusters;
+  L.max_items = pairs / kItemRows + L.Gtot + 1;
+  size_t o = lod::kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += (bytes + 255) & ~size_t(255);
+    return at;
+  };
+  L.state = take(sizeof(float) * 132 * (size_t)rows);
+  L.sel = take(sizeof(int32_t) * (size_t)pairs);
+  L.pos = take(sizeof(int32_t) * (size_t)pairs);
+  L.plse = take(sizeof(float) * (size_t)pairs);
+  L.po = take((size_t)2 * p->d * (size_t)pairs);
+  L.list = take(sizeof(int32_t) * (size_t)pairs);
+  L.cnt = take(sizeof(int32_t) * (size_t)L.Gtot);
+  L.off = take(sizeof(int32_t) * (size_t)L.Gtot);
+  L.items = take(16 * (size_t)L.max_items);
+  L.n_items = take(16);
+  L.total = o;
+  return L;
+}
+
+int g_num_sms[64] = {};
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+// Tensor maps of the pair kernel: member-ordered copies and page summaries.
+int32_t make_pair_maps(const lod_params* p, const lod_index* ix, lod::PairMaps* m) {
+  const cuuint64_t Cmax = (cuuint64_t)(p->Tmax / p->chunk);
+  const cuuint64_t mrows = (cuuint64_t)p->B * p->Hkv * Cmax * p->chunk;
+  const cuuint64_t prows = (cuuint64_t)p->B * p->Hkv * Cmax * page_slots(p);
+  const cuuint64_t str[1] = {(cuuint64_t)p->d * 2};
+  const cuuint64_t md[2] = {(cuuint64_t)p->d, mrows}, pd[2] = {(cuuint64_t)p->d, prows};
+  int32_t rc = encode_map(&m->mK, ix->mK, 2, md, str, 32);
+  if (!rc) rc = encode_map(&m->mV, ix->mV, 2, md, str, 32);
+  if (!rc) rc = encode_map(&m->pK, ix->pK, 2, pd, str, 16);
+  if (!rc) rc = encode_map(&m->pV, ix->pV, 2, pd, str, 16);
   return rc;
 }
 
@@ -375,7 +466,16 @@ int32_t lod_workspace_bytes(const lod_params* p, int32_t op, size_t* bytes) {
   switch (op) {
     case LOD_OP_BUILD: *bytes = lod::kWsHeader; break;
     case LOD_OP_DECODE: *bytes = attend_ws_bytes(p, decode_shape(p)); break;
-    case LOD_OP_PREFILL: *bytes = attend_ws_bytes(p, prefill_shape(p)); break;
+    case LOD_OP_PREFILL: {
+      // the grouped path's waves, or the per-chunk path (q in host memory)
+      size_t b = attend_ws_bytes(p, prefill_shape(p));
+      if (use_tc_prefill(p)) {
+        const size_t t = pf_layout(p).total;
+        if (t > b) b = t;
+      }
+      *bytes = b;
+      break;
+    }
     default: return fail(LOD_EINVAL, "unknown op %d", op);
   }
   g_err[0] = 0;
@@ -499,6 +599,65 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
   if (c1 > c0) {
     rc = do_build(p, K, V, kv_strides, c0, c1, index, ws, st);
     if (rc) return rc;
+  }
+  if (use_tc_prefill(p) && !q_host) {
+    // 2) grouped tensor-core attention, one wave of query chunks at a time
+    const PfLayout L = pf_layout(p);
+    lod::TcMaps maps;
+    lod::PairMaps pmaps;
+    rc = make_tc_maps(p, K, V, kv_strides, index, &maps);
+    if (!rc) rc = make_pair_maps(p, index, &pmaps);
+    if (rc) return rc;
+    char* w = static_cast<char*>(ws);
+    lod::PrefillArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.Tq = Tq;
+    a.q_begin = q_begin;
+    a.B = p->B;
+    a.Hq = p->Hq;
+    a.Hkv = p->Hkv;
+    a.g = g_of(p);
+    a.Tmax = p->Tmax;
+    a.Cmax = p->Tmax / p->chunk;
+    a.k = p->clusters;
+    a.P = page_slots(p);
+    a.G = p->top_groups;
+    a.TP = p->top_pages;
+    a.window = p->window;
+    a.sinks = p->sinks;
+    a.scale_log2 = (p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d)) * 1.4426950408889634f;
+    a.gMeta = index->gMeta;
+    a.gV = static_cast<const __nv_bfloat16*>(index->gV);
+    a.pBeg = index->pBeg;
+    a.pCnt = index->pCnt;
+    a.NW = L.NW;
+    a.state = reinterpret_cast<float*>(w + L.state);
+    a.sel = reinterpret_cast<int32_t*>(w + L.sel);
+    a.pos = reinterpret_cast<int32_t*>(w + L.pos);
+    a.plse = reinterpret_cast<float*>(w + L.plse);
+    a.po = reinterpret_cast<__nv_bfloat16*>(w + L.po);
+    a.list = reinterpret_cast<int32_t*>(w + L.list);
+    a.cnt = reinterpret_cast<int32_t*>(w + L.cnt);
+    a.off = reinterpret_cast<int32_t*>(w + L.off);
+    a.items = reinterpret_cast<int4*>(w + L.items);
+    a.n_items = reinterpret_cast<int32_t*>(w + L.n_items);
+    a.Gtot = L.Gtot;
+    a.item_rows = kItemRows;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.sel_groups = sel_groups;
+    a.sel_pages = sel_pages;
+    a.status = reinterpret_cast<uint32_t*>(w);
+    const int nsm = num_sms();
+    for (int64_t lo = 0; lo < Tq; lo += L.NW) {
+      a.w_lo = lo;
+      a.w_hi = lo + L.NW < Tq ? lo + L.NW : Tq;
+      cudaError_t e = lod::launch_prefill_tc_wave(a, maps, pmaps, nsm, st);
+      if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    }
+    g_err[0] = 0;
+    return LOD_OK;
   }
   // 2) attention, one launch pair per query chunk
   lod::AttendArgs a;

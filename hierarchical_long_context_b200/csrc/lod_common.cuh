@@ -154,6 +154,13 @@ __device__ __forceinline__ void cp_async4_zfill(void* dst, const void* src, bool
                "r"(valid ? 4u : 0u)
                : "memory");
 }
+// Sixteen-byte asynchronous copy global -> shared (both 16-byte aligned),
+// bypassing L1; `valid` false writes zeros (nothing is read from `src`).
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16u : 0u)
+               : "memory");
+}
 // One arrival on `bar` once every cp.async this thread issued before has
 // landed (the arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
@@ -179,6 +186,20 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+// 2^x on the special-function unit (approximate, flushes denormals; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two floats rounded (RNE) to bf16 and packed, `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Bring the 128-byte line holding `p` into L2 (no register result, no wait).

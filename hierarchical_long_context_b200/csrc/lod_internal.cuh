@@ -146,6 +146,52 @@ struct __align__(64) TcMaps {
   CUtensorMap gK, gV, K, V;
 };
 
+// Grouped tensor-core prefill (bf16, d = 128), one wave of query positions
+// [w_lo, w_hi) of q at a time.  A wave row is (b * Hq + hq) * NW + (pi - w_lo).
+struct PrefillArgs {
+  const __nv_bfloat16* q;   // [B][Hq][Tq][d] (device)
+  int64_t Tq, q_begin;
+  int B, Hq, Hkv, g;
+  int64_t Tmax, Cmax;
+  int k, P, G, TP, window, sinks;
+  float scale_log2;         // softmax scale * log2 e
+  const int32_t* gMeta;
+  const __nv_bfloat16* gV;
+  const int16_t* pBeg;
+  const int32_t* pCnt;
+  int64_t w_lo, w_hi, NW;   // this wave's q positions; NW = wave rows per (b, hq)
+  // workspace
+  float* state;             // [rows][132]: m, l (log2 units), -, -, acc[d] (opened groups removed)
+  int32_t* sel;             // [rows][G] opened group ids, best first, -1 padded
+  int32_t* pos;             // [rows][G] place of the pair in its group's run
+  float* plse;              // [rows][G] pair log-sum-exp (log2 units)
+  __nv_bfloat16* po;        // [rows][G][d] pair output (normalised)
+  int32_t* list;            // pair ids (row * G + rank) grouped by (unit, group)
+  int32_t* cnt;             // [Gtot] pairs per (unit, group)
+  int32_t* off;             // [Gtot] first pair of each (unit, group)
+  int4* items;              // work items {unit * Cmax * k + group, first pair, pairs, 0}
+  int32_t* n_items;
+  int64_t Gtot;             // B * Hkv * Cmax * k
+  int item_rows;            // pairs per work item (at most)
+  // outputs
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* sel_groups;
+  int32_t* sel_pages;
+  uint32_t* status;
+};
+
+// TMA tensor maps of the pair kernel: member-ordered K/V copies (32-row
+// boxes) and page summaries (16-row boxes), 64 columns, 128B swizzle.
+struct __align__(64) PairMaps {
+  CUtensorMap mK, mV, pK, pV;
+};
+
+cudaError_t launch_prefill_tc_wave(const PrefillArgs& a, const TcMaps& maps, const PairMaps& pmaps, int num_sms,
+                                   cudaStream_t stream);
+size_t prefill_tc_scan_smem();
+size_t prefill_tc_pair_smem();
+
 cudaError_t launch_build(const BuildArgs& a, int dtype, int d, int64_t nchunks, int B,
                          cudaStream_t stream);
 cudaError_t launch_append(void* K, void* V, const int64_t* kv_strides_elems, int elem_bytes, int d,

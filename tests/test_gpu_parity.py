@@ -431,6 +431,78 @@ def test_prefill_matches_oracle(name, T, split, kv_bits):
         print(lt.check_rows(cfg, w.dtype, K, V, u, rows))
 
 
+@pytest.mark.parametrize("kw, T", [
+    (dict(Hq=2, Hkv=2), 2048 + 100),                                       # g = 1: 128 positions per tile
+    (dict(Hq=4, Hkv=2), 2048 + 100),                                       # g = 2
+    (dict(top_pages=0), 2048 + 100),                                       # two-tier LoD: groups opened whole
+    (dict(clusters=(16,), top_groups=16, top_pages=4), 2048 + 100),        # k = 16, widest selection
+    (dict(clusters=(1,), top_groups=2, top_pages=1), 3072 + 5),            # k = 1: groups of 252-256 members
+    (dict(clusters=(2,), sinks=100, window=256), 2048 + 100),              # a sink tile with 100 live rows
+    (dict(Hq=8, Hkv=2, window=1024), 2048 + 100),                          # window of four chunks
+])
+def test_grouped_prefill_sweep(kw, T):
+    """The grouped tensor-core prefill over the head ratios, selection widths,
+    cluster counts (group sizes up to a whole chunk), windows and sinks that
+    lod_params accepts, each against the oracle on sampled rows."""
+    w = synth.WORKLOADS["prefill_128k_bf16"].with_(B=1, Hkv=2, Hq=8).with_(**kw)
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    dev = Kd.device
+    q = synth.prefill_queries(w, 0, T).to(dev)
+    ix = api.Index(p)
+    lse = torch.empty(w.B, w.Hq, T, dtype=torch.float32, device=dev)
+    sg = torch.empty(w.B, w.Hq, T, p.top_groups, dtype=torch.int32, device=dev)
+    sp = torch.empty(w.B, w.Hq, T, p.top_groups, max(p.top_pages, 1), dtype=torch.int32, device=dev)
+    ws = api.workspace(p, api._lib.LOD_OP_PREFILL)
+    out = api.lod_prefill(p, q, 0, Kd, Vd, ix, lse=lse, sel_groups=sg, sel_pages=sp if p.top_pages else None,
+                          ws=ws)
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws) == 0
+    assert torch.isfinite(out.float()).all()
+    cfg = lt.oracle_cfg(w)
+    rng = np.random.default_rng(5)
+    nch = T // 256
+    for h in range(w.Hkv):
+        K, V = _np(Kc[0, h]), _np(Vc[0, h])
+        u = lt.unit_from_gpu(ix, 0, h, nch, p)
+        ts = sorted(set(rng.integers(0, T, 24).tolist()) | {0, 511, 512, 767, 1024, T - 1})
+        rows = []
+        for hq in range(h * w.g, (h + 1) * w.g):
+            for t in ts:
+                gsp = sp[0, hq, t].cpu().numpy() if p.top_pages else np.zeros((p.top_groups, 0), np.int32)
+                rows.append((_np(q[0, hq, t]), t, _np(out[0, hq, t]).astype(np.float64),
+                             float(lse[0, hq, t]), sg[0, hq, t].cpu().numpy(), gsp))
+        print(kw, lt.check_rows(cfg, w.dtype, K, V, u, rows))
+
+
+def test_grouped_prefill_several_waves_match_one_call_per_chunk():
+    """A prefill longer than one wave of query chunks (64 chunks) equals the
+    same queries prefilled one chunk per call: the wave boundaries and the
+    pair bookkeeping leave every row's result unchanged, bit for bit."""
+    w = synth.WORKLOADS["prefill_128k_bf16"].with_(B=1, Hkv=1, Hq=4)
+    T = 64 * 256 + 700
+    p, Kc, Vc, Kd, Vd = _setup(w, None, T)
+    dev = Kd.device
+    q = synth.prefill_queries(w, 0, T).to(dev)
+    ws = api.workspace(p, api._lib.LOD_OP_PREFILL)
+    ix = api.Index(p)
+    lse = torch.empty(w.B, w.Hq, T, dtype=torch.float32, device=dev)
+    out = api.lod_prefill(p, q, 0, Kd, Vd, ix, lse=lse, ws=ws)
+    ix2 = api.Index(p)
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    for lo in range(0, T, 256):
+        hi = min(T, lo + 256)
+        o = torch.empty_like(q[:, :, lo:hi].contiguous())
+        l_ = torch.empty(w.B, w.Hq, hi - lo, dtype=torch.float32, device=dev)
+        api.lod_prefill(p, q[:, :, lo:hi].contiguous(), lo, Kd, Vd, ix2, out=o, lse=l_, ws=ws)
+        out2[:, :, lo:hi] = o
+        lse2[:, :, lo:hi] = l_
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws) == 0
+    assert torch.equal(out, out2)
+    assert torch.equal(lse, lse2)
+
+
 def _prefill_piece(p, q, lo, hi, Kd, Vd, ix, out, lse, sg, sp, ws):
     o = torch.empty_like(q[:, :, lo:hi].contiguous())
     l_ = torch.empty(q.shape[0], q.shape[1], hi - lo, dtype=torch.float32, device=q.device)
