@@ -252,28 +252,28 @@ bool use_tc_prefill(const lod_params* p) {
 }
 
 constexpr int kItemRows = 1024;                    // pairs per work item of the pair kernel
-constexpr int64_t kPrefillWaveBudget = (int64_t)1 << 30;  // workspace bytes a wave may use
+constexpr int64_t kPrefillWaveBudget = (int64_t)2 << 30;  // workspace bytes a wave may use
 
 // Workspace bytes per wave row: state (132 floats), and per opened group
-// its id, its place in the group's run, its log-sum-exp, its bf16 output and
-// its pair-list entry.
+// its id, its coarse weight, its log-sum-exp, its bf16 output and its
+// pair-list entry.
 int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 2 * p->d + 4); }
 
 // Query positions per wave: a multiple of chunk, as many as the budget allows
-// (at least one chunk, at most 64), never more than the cache holds.
+// (at least one chunk, at most 128), never more than the cache holds.
 int64_t pf_wave(const lod_params* p) {
   const int64_t rows = (int64_t)p->B * p->Hq;
   int64_t nw = kPrefillWaveBudget / (rows * pf_row_bytes(p)) / p->chunk * p->chunk;
   const int64_t most = (((int64_t)1 << 31) - 1) / (rows * p->top_groups) / p->chunk * p->chunk;
   if (nw > most) nw = most;
-  if (nw > 64 * (int64_t)p->chunk) nw = 64 * (int64_t)p->chunk;
+  if (nw > 128 * (int64_t)p->chunk) nw = 128 * (int64_t)p->chunk;
   if (nw > p->Tmax) nw = p->Tmax;
   if (nw < p->chunk) nw = p->chunk;
   return nw;
 }
 
 struct PfLayout {
-  size_t state, sel, pos, plse, po, list, cnt, off, items, n_items, total;
+  size_t state, sel, cw, plse, po, list, cnt, off, items, n_items, total;
   int64_t NW, Gtot, max_items;
 };
 
@@ -292,13 +292,13 @@ PfLayout pf_layout(const lod_params* p) {
   };
   L.state = take(sizeof(float) * 132 * (size_t)rows);
   L.sel = take(sizeof(int32_t) * (size_t)pairs);
-  L.pos = take(sizeof(int32_t) * (size_t)pairs);
+  L.cw = take(sizeof(float) * (size_t)pairs);
   L.plse = take(sizeof(float) * (size_t)pairs);
   L.po = take((size_t)2 * p->d * (size_t)pairs);
   L.list = take(sizeof(int32_t) * (size_t)pairs);
   L.cnt = take(sizeof(int32_t) * (size_t)L.Gtot);
   L.off = take(sizeof(int32_t) * (size_t)L.Gtot);
-  L.items = take(16 * (size_t)L.max_items);
+  L.items = take(16 * 2 * (size_t)L.max_items);  // small-group items, then large-group items
   L.n_items = take(16);
   L.total = o;
   return L;
@@ -634,13 +634,14 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.NW = L.NW;
     a.state = reinterpret_cast<float*>(w + L.state);
     a.sel = reinterpret_cast<int32_t*>(w + L.sel);
-    a.pos = reinterpret_cast<int32_t*>(w + L.pos);
+    a.cw = reinterpret_cast<float*>(w + L.cw);
     a.plse = reinterpret_cast<float*>(w + L.plse);
     a.po = reinterpret_cast<__nv_bfloat16*>(w + L.po);
     a.list = reinterpret_cast<int32_t*>(w + L.list);
     a.cnt = reinterpret_cast<int32_t*>(w + L.cnt);
     a.off = reinterpret_cast<int32_t*>(w + L.off);
     a.items = reinterpret_cast<int4*>(w + L.items);
+    a.big_items = L.max_items;
     a.n_items = reinterpret_cast<int32_t*>(w + L.n_items);
     a.Gtot = L.Gtot;
     a.item_rows = kItemRows;

@@ -161,16 +161,18 @@ struct PrefillArgs {
   const int32_t* pCnt;
   int64_t w_lo, w_hi, NW;   // this wave's q positions; NW = wave rows per (b, hq)
   // workspace
-  float* state;             // [rows][132]: m, l (log2 units), -, -, acc[d] (opened groups removed)
+  float* state;             // [rows][132]: m, l (log2 units), -, -, acc[d] (opened groups included)
   int32_t* sel;             // [rows][G] opened group ids, best first, -1 padded
-  int32_t* pos;             // [rows][G] place of the pair in its group's run
+  float* cw;                // [rows][G] weight of the opened group's coarse term, relative to m
   float* plse;              // [rows][G] pair log-sum-exp (log2 units)
   __nv_bfloat16* po;        // [rows][G][d] pair output (normalised)
   int32_t* list;            // pair ids (row * G + rank) grouped by (unit, group)
   int32_t* cnt;             // [Gtot] pairs per (unit, group)
-  int32_t* off;             // [Gtot] first pair of each (unit, group)
-  int4* items;              // work items {unit * Cmax * k + group, first pair, pairs, 0}
-  int32_t* n_items;
+  int32_t* off;             // [Gtot] first pair of each (unit, group); advanced by the scatter
+  int4* items;              // work items {unit * Cmax * k + group, first pair, pairs, 0}: small groups
+                            // from items[0], large groups from items[big_items]
+  int64_t big_items;
+  int32_t* n_items;         // [2] work items of small and of large groups
   int64_t Gtot;             // B * Hkv * Cmax * k
   int item_rows;            // pairs per work item (at most)
   // outputs

@@ -53,6 +53,7 @@ constexpr uint32_t kTileBytes = 128 * D * 2;    // one 128 x 128 bf16 operand ti
 constexpr uint32_t kHalf = kTileBytes / 2;      // one 64-column half of it
 constexpr float kTau2 = 12.f;                   // weights reach at most 2^kTau2 before the reference max moves
 constexpr int kStateStride = 132;               // floats per row state: m, l, -, -, acc[128]
+constexpr int kSmallN = 112;  // pair kernel: groups up to this size run two CTAs per SM (members + 16 page columns fit 128)
 
 __device__ __forceinline__ uint32_t sw_off(int row, int chunk16) {  // 16-byte chunk of a 128B-swizzled row
   return (uint32_t)(row * 128 + (((chunk16 & 7) ^ (row & 7)) << 4));
@@ -60,19 +61,25 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk16) {  // 16-byte c
 
 // ================================================================== phase A
 
-constexpr int kThreadsA = 192;   // warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax
-constexpr int kBarSoftA = 1;
+constexpr int kThreadsA = 320;   // warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax, 6-9 top-G + epilogue
+constexpr int kCandCap = 32;     // buffered top-G candidates per row
+constexpr int kBarLncA = 1;      // named barrier of the softmax warps
+constexpr int kBarEpiA = 2;      // named barrier of warps 2-9 (hand-over of the softmax state)
+
+// Tensor memory of the scan: S double-buffered in columns [0, 256), O in
+// [256, 384), the query tile (bf16 pairs, MMA 1's A operand) in [384, 448).
+constexpr uint32_t kColO = 256, kColQ = 384;
 
 struct SmemA {
-  static constexpr size_t off_Q = 0;                          // [2 halves][128][128 B]
-  static constexpr size_t off_K = off_Q + kTileBytes;         // [2 stages]
+  static constexpr size_t off_K = 0;                          // [2 stages][2 halves][128][128 B]
   static constexpr size_t off_V = off_K + 2 * kTileBytes;     // [2 stages]
   static constexpr size_t off_P = off_V + 2 * kTileBytes;     // [2 halves][128][128 B]
-  static constexpr size_t off_meta = off_P + kTileBytes;      // int [2][128]
+  static constexpr size_t off_cand = off_P + kTileBytes;      // float2 [128][kCandCap + 1] (+1: a junk slot)
+  static constexpr size_t off_meta = off_cand + 128 * (kCandCap + 1) * 8;  // int [2][128]
   static constexpr size_t off_lnc = off_meta + 2 * 128 * 4;   // float [2][128]
-  static constexpr size_t off_stash = off_lnc + 2 * 128 * 4;  // float [128][33]
-  static constexpr int kBars = 15;
-  static constexpr size_t off_bar = off_stash + 128 * 33 * 4;
+  static constexpr size_t off_ml = off_lnc + 2 * 128 * 4;   // float2 [128] softmax state handed over
+  static constexpr int kBars = 17;
+  static constexpr size_t off_bar = off_ml + 128 * 8;
   static constexpr size_t off_misc = off_bar + 8 * kBars;     // tmem slot, abort flag
   static constexpr size_t bytes = off_misc + 16 + 1024;
   static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -80,33 +87,46 @@ struct SmemA {
 
 // Insert (v, id) into the descending list (s, ix) of GM entries: every entry
 // from the first one v beats moves down by one place.  Ties keep the earlier
-// entry first (ids arrive in increasing order, so the lower id wins).
+// entry first (ids arrive in increasing order, so the lower id wins).  A
+// list of G < GM entries occupies the last G slots below GM - G sentinels of
+// +inf, so that its G-th best is always s[GM - 1] (a runtime index into a
+// register array would move the list to local memory).
 template <int GM>
 __device__ __forceinline__ void topk_insert(float (&s)[GM], int (&ix)[GM], float v, int id) {
   bool act = false;
   float cs = v;
   int ci = id;
 #pragma unroll
-  for (int k = 0; k < GM; ++k) {
+  for (int k = 0; k < GM; ++k) {  // selects only: the list stays in registers
     act = act || (v > s[k]);
-    const float ts = s[k];
-    const int ti = ix[k];
-    if (act) {
-      s[k] = cs;
-      ix[k] = ci;
-      cs = ts;
-      ci = ti;
-    }
+    const float ns = act ? cs : s[k];
+    const int ni = act ? ci : ix[k];
+    cs = act ? s[k] : cs;
+    ci = act ? ix[k] : ci;
+    s[k] = ns;
+    ix[k] = ni;
   }
 }
 
+// Merge a row's buffered candidates (ascending ids: ties keep the earlier
+// one) into its sorted list; the whole warp calls it.
 template <int GM>
-__device__ __forceinline__ float topk_kth(const float (&s)[GM], int G) {
-  float t = s[GM - 1];
+__device__ __forceinline__ void topk_merge(float (&s)[GM], int (&ix)[GM], float& thr, int& n, const float2* buf) {
+  const int nmax = (int)__reduce_max_sync(0xffffffffu, (unsigned)n);
+  for (int j0 = 0; j0 < nmax; j0 += 4) {
+    float2 cv[4];
 #pragma unroll
-  for (int k = 0; k < GM; ++k)
-    if (k == G - 1) t = s[k];
-  return t;
+    for (int q = 0; q < 4; ++q) cv[q] = j0 + q < n ? buf[j0 + q] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (cv[q].x > thr) {
+        topk_insert<GM>(s, ix, cv[q].x, __float_as_int(cv[q].y));
+        thr = s[GM - 1];
+      }
+    }
+  }
+  n = 0;
+  __syncwarp();
 }
 
 template <int GM>
@@ -116,13 +136,13 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
-  unsigned char* Qs = sm + SmemA::off_Q;
   unsigned char* Kring = sm + SmemA::off_K;
   unsigned char* Vring = sm + SmemA::off_V;
   unsigned char* Ps = sm + SmemA::off_P;
+  float2* cand_s = reinterpret_cast<float2*>(sm + SmemA::off_cand);
   int* meta_s = reinterpret_cast<int*>(sm + SmemA::off_meta);
   float* lnc_s = reinterpret_cast<float*>(sm + SmemA::off_lnc);
-  float* stash = reinterpret_cast<float*>(sm + SmemA::off_stash);
+  float2* ml_s = reinterpret_cast<float2*>(sm + SmemA::off_ml);
   uint64_t* kfull = reinterpret_cast<uint64_t*>(sm + SmemA::off_bar);
   uint64_t* kempty = kfull + 2;
   uint64_t* vfull = kempty + 2;
@@ -132,6 +152,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 1;
   uint64_t* fin = o_done + 1;
+  uint64_t* lnc_ready = fin + 1;  // [2]: ln counts of a group tile written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SmemA::off_misc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + SmemA::off_misc + 4);
 
@@ -163,9 +184,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
       mbar_init(&vfull[i], 1 + 32);
-      mbar_init(&vempty[i], 1);
+      mbar_init(&vempty[i], 1 + 4);  // MMA 2 done + the four top-G warps done with the tile's counts
+      mbar_init(&lnc_ready[i], 4);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], 8);
     }
     mbar_init(p_full, 4);
     mbar_init(o_done, 1);
@@ -178,24 +200,41 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     tc::prefetch_tensormap(&maps.V);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
-  // ---- the query tile (softmax warps): row r = position r / g, head r % g
-  if (warp >= 2) {
-    const int r = tid - 64;  // 0..127: each thread stages one row
+  // the query rows, loaded while TMEM is allocated (row r = position r / g, head r % g)
+  uint4 qrow[16];
+  if (warp >= 2 && warp < 6) {
+    const int r = 32 * (warp & 3) + lane;
     const int64_t pi = pos0 + r / a.g;
     const int hq = kvh * a.g + r % a.g;
     const bool okr = pi < pos_end;
     const __nv_bfloat16* src = a.q + (((int64_t)b * a.Hq + hq) * a.Tq + (okr ? pi : 0)) * D;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint4 v = okr ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(Qs + (c >> 3) * kHalf + sw_off(r, c)) = v;
-    }
+    for (int c = 0; c < 16; ++c) qrow[c] = okr ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
   }
-  tc::fence_proxy_async();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // ---- the query tile into TMEM lane r (MMA 1's A operand)
+  if (warp >= 2 && warp < 6) {
+    const uint32_t tl = (uint32_t)(32 * (warp & 3)) << 16;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float qv[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w = qrow[8 * h + c];
+        qv[4 * c] = __uint_as_float(w.x);
+        qv[4 * c + 1] = __uint_as_float(w.y);
+        qv[4 * c + 2] = __uint_as_float(w.z);
+        qv[4 * c + 3] = __uint_as_float(w.w);
+      }
+      tc::tmem_st32(tmem + tl + kColQ + 32 * h, qv);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*abort_s) return false;
@@ -263,7 +302,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idO = tc::idesc_bf16(128, 128, false, true);
-      const uint32_t qb = smem_u32(Qs), pb = smem_u32(Ps);
+      const uint32_t pb = smem_u32(Ps);
       auto mma2 = [&](int j) -> bool {  // O += P_j V_j
         if (!wait(p_full, (uint32_t)j & 1u)) return false;
         if (!wait(&vfull[j & 1], (uint32_t)(j >> 1) & 1u)) return false;
@@ -273,7 +312,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ad = tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32);
           const uint64_t bd = tc::desc_mnmajor_sw128(vb + kk * 2048, kHalf);
-          tc::mma_bf16(tmem + 256, ad, bd, idO, j > 0 || kk > 0);
+          tc::mma_bf16(tmem + kColO, ad, bd, idO, j > 0 || kk > 0);
         }
         tc::mma_commit(&vempty[j & 1]);
         tc::mma_commit(o_done);
@@ -287,9 +326,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         const uint32_t kb = smem_u32(Kring + (i & 1) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = tc::desc_kmajor_sw128(qb + (kk >> 2) * kHalf + (kk & 3) * 32);
           const uint64_t bd = tc::desc_kmajor_sw128(kb + (kk >> 2) * kHalf + (kk & 3) * 32);
-          tc::mma_bf16(tmem + (uint32_t)(i & 1) * 128, ad, bd, idS, kk > 0);
+          tc::mma_bf16_ts(tmem + (uint32_t)(i & 1) * 128, tmem + kColQ + 8 * kk, bd, idS, kk > 0);
         }
         tc::mma_commit(&kempty[i & 1]);
         tc::mma_commit(&s_full[i & 1]);
@@ -303,50 +341,24 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       }
     }
     __syncwarp();
-  } else {
-    // ================================================================ softmax
+  } else if (warp < 6) {
+    // ================================================================ softmax (warps 2-5)
     const int q4 = warp & 3;
-    const int r = 32 * q4 + lane;  // query row of this thread (and key row it stages)
+    const int r = 32 * q4 + lane;  // query row of this thread (and the key row it stages)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
-    const int64_t pi = pos0 + r / a.g;
-    const int hq = kvh * a.g + r % a.g;
-    const bool valid = pi < pos_end;
-    const int64_t t_row = a.q_begin + pi;
+    const int64_t t_row = a.q_begin + pos0 + r / a.g;
     const float scl = a.scale_log2;
     float m = -INFINITY, l = 0.f;
-    float ts[GM];
-    int ti[GM];
-#pragma unroll
-    for (int k = 0; k < GM; ++k) {
-      ts[k] = -INFINITY;
-      ti[k] = -1;
-    }
-    float thr = -INFINITY;
-    float* my_stash = stash + r * 33;
     bool alive = true;
     for (int i = 0; i < ntile; ++i) {
       const int st = i & 1;
       const bool grp = i < gt, snk = !grp && i < gt + st_;
       const int64_t kpos0 = grp ? 0 : (snk ? (int64_t)(i - gt) * 128 : ws + (int64_t)(i - gt - st_) * 128);
-      // (a failed wait in a group tile is carried to that tile's softmax
-      // barrier, where the four warps leave the loop together)
+      // (a failed wait in a group tile is carried to that tile's barrier,
+      // where the eight warps leave the loop together)
       alive = __all_sync(0xffffffffu, wait(&s_full[st], (uint32_t)(i >> 1) & 1u) &&
                                           wait(&vfull[st], (uint32_t)(i >> 1) & 1u));
       if (!alive && !grp) break;
-      float s[128];
-      if (alive) {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(tmem + tl + (uint32_t)st * 128 + 32 * c, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[32 * c + e] = v[e];
-        }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[st]);
-      }
       // key row r of this tile: its bias (group tiles) and whether it is in
       // no row's softmax (its value row is then zeroed: MMA 2 must not meet
       // NaN or Inf from rows that are not inputs of this call)
@@ -367,78 +379,52 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       if (dead) {
         unsigned char* vd = Vring + st * kTileBytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(vd + h * kHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 16; ++c)  // (swizzled order: the warp's rows spread over the banks)
+          *reinterpret_cast<uint4*>(vd + (c >> 3) * kHalf + sw_off(r, c)) = make_uint4(0, 0, 0, 0);
       }
-      float xm = -INFINITY;
-      if (grp) {
-        // every group's ln count is in lnc_s past this barrier
-        if (bar_red_or(kBarSoftA, 128, !alive)) {
+      if (grp) {  // every group's ln count is in lnc_s past here
+        if (bar_red_or(kBarLncA, 128, !alive)) {
           alive = false;
           break;
         }
-        const float* lc = lnc_s + st * 128;
+        if (lane == 0) mbar_arrive(&lnc_ready[st]);
+      }
+      tc::fence_after_sync();
+      const uint32_t sb = tmem + tl + (uint32_t)st * 128;
+      const float* lc = lnc_s + st * 128;
+      // window and sink keys at positions kpos0 + j <= lim are in this row's softmax
+      const int64_t lim = snk ? nsk - 1 : t_row;
+      const int rel = grp ? 127 : (int)(lim - kpos0 < -1 ? -1 : (lim - kpos0 > 127 ? 127 : lim - kpos0));
+      // the logits (log2 units) of key columns [64 h, 64 h + 64), minus `sub`
+      auto logits = [&](int h, float (&x)[64], float sub) {
+        tc::tmem_ld32xN<2>(sb + 64 * h, x);
+        if (grp) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float lv[32];
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lc + 64 * h + 4 * e4);
+            const float lv[4] = {l4.x - sub, l4.y - sub, l4.z - sub, l4.w - sub};
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(lc + 32 * c + 4 * e4);
-            lv[4 * e4] = l4.x;
-            lv[4 * e4 + 1] = l4.y;
-            lv[4 * e4 + 2] = l4.z;
-            lv[4 * e4 + 3] = l4.w;
+            for (int e = 0; e < 4; ++e)  // fmaxf drops NaN: a group outside the softmax gives -inf
+              x[4 * e4 + e] = fmaxf(fmaf(x[4 * e4 + e], scl, lv[e]), -INFINITY);
           }
-          // the raw scores of the groups in this row's softmax (-inf otherwise)
-          float cm = -INFINITY;
+        } else if (rel >= 127) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            s[32 * c + e] = (valid && lv[e] != -INFINITY) ? s[32 * c + e] : -INFINITY;
-            cm = fmaxf(cm, s[32 * c + e]);
-          }
-          // top-G: only a chunk holding a score above the current G-th best
-          // is scanned (rare once the first tiles have filled the list)
-          const bool cand = cm > thr;
-          if (__any_sync(0xffffffffu, cand)) {
-            if (cand) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) my_stash[e] = s[32 * c + e];
-              for (int e = 0; e < 32; ++e) {
-                const float v = my_stash[e];
-                if (v > thr) {
-                  topk_insert<GM>(ts, ti, v, (int)((int64_t)i * 128 + 32 * c + e));
-                  thr = topk_kth<GM>(ts, a.G);
-                }
-              }
-            }
-            __syncwarp();
-          }
-          // the logits in log2 units: score * scale * log2 e + log2 count
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            s[32 * c + e] = fmaf(s[32 * c + e], scl, lv[e]);
-            xm = fmaxf(xm, s[32 * c + e]);
-          }
-        }
-      } else {
-        const int64_t lim = snk ? nsk - 1 : t_row;  // keys at positions kpos0 + j <= lim
-        const int64_t rel = valid ? lim - kpos0 : -1;
-        if (rel >= 127) {
-#pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            s[j] *= scl;
-            xm = fmaxf(xm, s[j]);
-          }
+          for (int e = 0; e < 64; ++e) x[e] = fmaf(x[e], scl, -sub);
         } else {
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            s[j] = j <= rel ? s[j] * scl : -INFINITY;
-            xm = fmaxf(xm, s[j]);
-          }
+          for (int e = 0; e < 64; ++e) x[e] = 64 * h + e <= rel ? fmaf(x[e], scl, -sub) : -INFINITY;
         }
+      };
+      // ---- pass 1: the logit max
+      float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent max chains
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float x[64];
+        logits(h, x, 0.f);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) xa[e & 3] = fmaxf(xa[e & 3], x[e]);
       }
+      const float xm = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
       // the reference max moves when a logit exceeds it by more than kTau2
       const bool need = xm > m + kTau2;
       bool waited = false;
@@ -455,82 +441,148 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               float ov[32];
-              tc::tmem_ld32(tmem + tl + 256 + 32 * c, ov);
+              tc::tmem_ld32(tmem + tl + kColO + 32 * c, ov);
 #pragma unroll
               for (int e = 0; e < 32; ++e) ov[e] *= corr;
-              tc::tmem_st32(tmem + tl + 256 + 32 * c, ov);
+              tc::tmem_st32(tmem + tl + kColO + 32 * c, ov);
             }
           }
         }
       }
-      // the weights into P (free once MMA 2 of the previous tile is done)
+      // P is free once MMA 2 of the previous tile is done
       if (i > 0 && !waited) alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u)) && alive;
       if (!alive) break;
       const float mu = m == -INFINITY ? 0.f : m;
+      // ---- pass 2: the weights 2^(logit - m) into P
+      float la[4] = {0.f, 0.f, 0.f, 0.f};  // independent sum chains
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float x[64];
+        logits(h, x, mu);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float p[8];
+        for (int q = 0; q < 8; ++q) {
+          float p[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = ex2_approx(s[8 * c + e] - mu);
-          l += p[e];
+          for (int e = 0; e < 8; ++e) {
+            p[e] = ex2_approx(x[8 * q + e]);
+            la[e & 3] += p[e];
+          }
+          const int ch = 8 * h + q;
+          *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
+              make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                         pack_bf16x2(p[6], p[7]));
         }
-        const uint4 w = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                                   pack_bf16x2(p[6], p[7]));
-        *reinterpret_cast<uint4*>(Ps + (c >> 3) * kHalf + sw_off(r, c)) = w;
       }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      l += (la[0] + la[1]) + (la[2] + la[3]);
       tc::fence_proxy_async();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // ---------------------------------------------------------------- epilogue
-    if (alive && ntile > 0) alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(ntile - 1) & 1u));
-    tc::fence_after_sync();
-    const int64_t wr = ((int64_t)b * a.Hq + hq) * a.NW + (pi - a.w_lo);  // wave row
-    const int64_t orow = ((int64_t)b * a.Hq + hq) * a.Tq + pi;
-    float w[GM], lcnt[GM];
-    int nsel = 0;
+    // the row's softmax state goes to the selection warps, which write it
+    ml_s[r] = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+    bar_named_sync(kBarEpiA, 256);
+  } else {
+    // ================================================================ top-G and epilogue (warps 6-9)
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;
+    const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    const int64_t pi = pos0 + r / a.g;
+    const int hq = kvh * a.g + r % a.g;
+    const bool valid = pi < pos_end;
+    const float scl = a.scale_log2;
+    float ts[GM];
+    int ti[GM];
 #pragma unroll
     for (int k = 0; k < GM; ++k) {
-      w[k] = 0.f;
-      lcnt[k] = 0.f;
-      if (k < a.G && ti[k] >= 0) {
-        const int c = a.gMeta[grow0 + ti[k]] & 0xffff;
-        lcnt[k] = log2f((float)(c > 0 ? c : 1));
-        ++nsel;
-      }
+      ts[k] = k < GM - a.G ? INFINITY : -INFINITY;
+      ti[k] = -1;
     }
-    const float mu = m == -INFINITY ? 0.f : m;
+    float thr = -INFINITY;
+    // this row's buffer of candidates (scores above the running G-th best,
+    // not yet merged into the sorted list ts/ti)
+    float2* cbuf = cand_s + r * (kCandCap + 1);
+    int ncand = 0;
+    bool alive = true;
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i & 1;
+      const bool grp = i < gt;
+      alive = __all_sync(0xffffffffu, wait(&s_full[st], (uint32_t)(i >> 1) & 1u));
+      if (alive && grp) alive = __all_sync(0xffffffffu, wait(&lnc_ready[st], (uint32_t)(i >> 1) & 1u));
+      if (!alive) break;
+      if (grp) {
+        tc::fence_after_sync();
+        const float* lc = lnc_s + st * 128;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float v[64];
+          tc::tmem_ld32xN<2>(tmem + tl + (uint32_t)st * 128 + 64 * h, v);
 #pragma unroll
-    for (int k = 0; k < GM; ++k) {
-      if (k < nsel) {
-        w[k] = ex2_approx(fmaf(ts[k], scl, lcnt[k]) - mu);
-        l -= w[k];
-      }
-    }
-    float* stp = a.state + wr * kStateStride;
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c = 2 * h + c2;
+            // the raw scores of the groups in the softmax (-inf: outside)
+            float ca[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float ov[32];
-      tc::tmem_ld32(tmem + tl + 256 + 32 * c, ov);
-      if (valid && alive) {
-#pragma unroll
-        for (int k = 0; k < GM; ++k) {
-          if (k < nsel) {
-            const uint4* gv = reinterpret_cast<const uint4*>(a.gV + (grow0 + ti[k]) * D + 32 * c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 raw = __ldg(gv + q);
-              const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(lc + 32 * c + 4 * e4);
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                ov[8 * q + 2 * e] = fmaf(-w[k], __uint_as_float(wd[e] << 16), ov[8 * q + 2 * e]);
-                ov[8 * q + 2 * e + 1] = fmaf(-w[k], __uint_as_float(wd[e] & 0xffff0000u), ov[8 * q + 2 * e + 1]);
+                float& x = v[32 * c2 + 4 * e4 + e];
+                x = (valid && lv[e] != -INFINITY) ? x : -INFINITY;
+                ca[e] = fmaxf(ca[e], x);
+              }
+            }
+            const float cm = fmaxf(fmaxf(ca[0], ca[1]), fmaxf(ca[2], ca[3]));
+            // candidates: scores above the running G-th best go to the buffer
+            // (merged into the sorted list whenever 16 more might not fit)
+            if (__any_sync(0xffffffffu, cm > thr)) {
+              const int id0 = i * 128 + 32 * c;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                if (__any_sync(0xffffffffu, ncand > kCandCap - 16)) topk_merge<GM>(ts, ti, thr, ncand, cbuf);
+#pragma unroll
+                for (int e = 16 * hh; e < 16 * hh + 16; ++e) {  // (branch-free: a miss writes the junk slot)
+                  const float x = v[32 * c2 + e];
+                  const bool hit = x > thr;
+                  cbuf[hit ? ncand : kCandCap] = make_float2(x, __int_as_float(id0 + e));
+                  ncand += hit ? 1 : 0;
+                }
               }
             }
           }
         }
+        if (i == gt - 1) topk_merge<GM>(ts, ti, thr, ncand, cbuf);  // the list is final
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[st]);
+        mbar_arrive(&vempty[st]);  // (the stage's counts may be overwritten)
+      }
+    }
+    // ---------------------------------------------------------------- epilogue
+    bar_named_sync(kBarEpiA, 256);
+    const float2 ml = ml_s[r];
+    const float m = ml.x;
+    float l = ml.y;
+    if (ml.x == -INFINITY && ml.y == 0.f && gt + st_ < ntile) alive = false;  // the softmax gave up
+    if (alive && ntile > 0) alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(ntile - 1) & 1u));
+    tc::fence_after_sync();
+    const int64_t wr = ((int64_t)b * a.Hq + hq) * a.NW + (pi - a.w_lo);  // wave row
+    const int64_t orow = ((int64_t)b * a.Hq + hq) * a.Tq + pi;
+    // the row state (m, l, acc) and the opened groups (list slots GM - G ..
+    // GM - 1, best first, -1: none) with the weights of their coarse terms
+    // relative to m: the merge removes those terms (finer entries replace them)
+    float* stp = a.state + wr * kStateStride;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float ov[32];
+      tc::tmem_ld32(tmem + tl + kColO + 32 * c, ov);
+      if (valid && alive) {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           *reinterpret_cast<float4*>(stp + 4 + 32 * c + 4 * q) =
@@ -538,20 +590,22 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       }
     }
     if (valid) {
-      if (alive) {
-        stp[0] = m;
-        stp[1] = l;
-      } else {
-        stp[0] = -INFINITY;
-        stp[1] = 0.f;
-      }
+      *reinterpret_cast<float2*>(stp) = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+      const float mu = m == -INFINITY ? 0.f : m;
 #pragma unroll
       for (int k = 0; k < GM; ++k) {
-        if (k < a.G) {
-          const int gid = (alive && k < nsel) ? ti[k] : -1;
-          a.sel[wr * a.G + k] = gid;
-          if (a.sel_groups) a.sel_groups[orow * a.G + k] = gid;
-          a.pos[wr * a.G + k] = gid >= 0 ? atomicAdd(a.cnt + grow0 + gid, 1) : -1;
+        if (k >= GM - a.G) {
+          const int j = k - (GM - a.G);  // rank
+          const int gid = alive ? ti[k] : -1;
+          float wk = 0.f;
+          if (gid >= 0) {
+            const int c = a.gMeta[grow0 + gid] & 0xffff;
+            wk = ex2_approx(fmaf(ts[k], scl, log2f((float)(c > 0 ? c : 1))) - mu);
+          }
+          a.sel[wr * a.G + j] = gid;
+          a.cw[wr * a.G + j] = wk;
+          if (a.sel_groups) a.sel_groups[orow * a.G + j] = gid;
+          if (gid >= 0) atomicAdd(a.cnt + grow0 + gid, 1);  // (result unused: a reduction, no round trip)
         }
       }
     }
@@ -569,63 +623,67 @@ constexpr int kPlanThreads = 1024;
 // items: group gflat with c pairs gives ceil(c / item_rows) items
 // {gflat, first pair, pairs}.
 __global__ void __launch_bounds__(kPlanThreads) pf_plan_kernel(const __grid_constant__ PrefillArgs a) {
-  __shared__ int wsum[2][32];
-  __shared__ long long carry[2];
+  __shared__ int wsum[3][32];
+  __shared__ long long carry[3];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) carry[0] = carry[1] = 0;
+  if (tid < 3) carry[tid] = 0;
   __syncthreads();
   for (int64_t base = 0; base < a.Gtot; base += kPlanThreads) {
     const int64_t gf = base + tid;
     const int c = gf < a.Gtot ? a.cnt[gf] : 0;
+    const bool big = c > 0 && (a.gMeta[gf] & 0xffff) > kSmallN;
     const int ni = (c + a.item_rows - 1) / a.item_rows;
-    int xp = c, xi = ni;  // inclusive warp scans
+    int x[3] = {c, big ? 0 : ni, big ? ni : 0};  // pairs, small items, big items
+    int y[3] = {x[0], x[1], x[2]};                // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int yp = __shfl_up_sync(0xffffffffu, xp, o), yi = __shfl_up_sync(0xffffffffu, xi, o);
-      if (lane >= o) {
-        xp += yp;
-        xi += yi;
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const int z = __shfl_up_sync(0xffffffffu, y[q], o);
+        if (lane >= o) y[q] += z;
       }
     }
     if (lane == 31) {
-      wsum[0][warp] = xp;
-      wsum[1][warp] = xi;
+#pragma unroll
+      for (int q = 0; q < 3; ++q) wsum[q][warp] = y[q];
     }
     __syncthreads();
     if (warp == 0) {
-      int sp = wsum[0][lane], si = wsum[1][lane];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yp = __shfl_up_sync(0xffffffffu, sp, o), yi = __shfl_up_sync(0xffffffffu, si, o);
-        if (lane >= o) {
-          sp += yp;
-          si += yi;
+      for (int q = 0; q < 3; ++q) {
+        int sv = wsum[q][lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int z = __shfl_up_sync(0xffffffffu, sv, o);
+          if (lane >= o) sv += z;
         }
+        wsum[q][lane] = sv;
       }
-      wsum[0][lane] = sp;
-      wsum[1][lane] = si;
     }
     __syncthreads();
-    const long long bp = carry[0] + (warp > 0 ? wsum[0][warp - 1] : 0) + xp - c;
-    const long long bi = carry[1] + (warp > 0 ? wsum[1][warp - 1] : 0) + xi - ni;
+    long long ex[3];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) ex[q] = carry[q] + (warp > 0 ? wsum[q][warp - 1] : 0) + y[q] - x[q];
     if (gf < a.Gtot) {
-      a.off[gf] = (int32_t)bp;
-      for (int x = 0; x < ni; ++x) {
-        const int n = c - x * a.item_rows < a.item_rows ? c - x * a.item_rows : a.item_rows;
-        a.items[bi + x] = make_int4((int)gf, (int)(bp + (long long)x * a.item_rows), n, 0);
+      a.off[gf] = (int32_t)ex[0];  // the scatter advances it to the run's end
+      int4* dst = big ? a.items + a.big_items + ex[2] : a.items + ex[1];
+      for (int t = 0; t < ni; ++t) {
+        const int n = c - t * a.item_rows < a.item_rows ? c - t * a.item_rows : a.item_rows;
+        dst[t] = make_int4((int)gf, (int)(ex[0] + (long long)t * a.item_rows), n, 0);
       }
     }
     __syncthreads();
-    if (tid == 0) {
-      carry[0] += wsum[0][31];
-      carry[1] += wsum[1][31];
-    }
+    if (tid < 3) carry[tid] += wsum[tid][31];
     __syncthreads();
   }
-  if (tid == 0) *a.n_items = (int32_t)carry[1];
+  if (tid == 0) {
+    a.n_items[0] = (int32_t)carry[1];
+    a.n_items[1] = (int32_t)carry[2];
+  }
 }
 
-// Every (row, group) pair into its group's run of the pair list.
+// Every (row, group) pair into its group's run of the pair list (the order
+// inside a run is arbitrary: every pair is computed on its own).
 __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__ PrefillArgs a) {
   const int64_t n = (int64_t)a.B * a.Hq * a.NW * a.G;
   for (int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * 256) {
@@ -636,7 +694,7 @@ __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__
     if (gid < 0) continue;
     const int64_t bh = wr / a.NW;
     const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
-    a.list[a.off[u * a.Cmax * a.k + gid] + a.pos[idx]] = (int32_t)idx;
+    a.list[atomicAdd(a.off + u * a.Cmax * a.k + gid, 1)] = (int32_t)idx;
   }
 }
 
@@ -644,16 +702,27 @@ __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__
 
 constexpr int kThreadsB = 160;   // warp 0 TMA + MMA issue, warps 1-4 one pair per thread
 constexpr int kBarSoftB = 2;
-constexpr size_t kSmemBData = 216 * 1024;  // operand regions (laid out per work item)
 
-struct SmemB {
-  static constexpr size_t off_misc = kSmemBData;           // per-item info, page counts, barriers
-  static constexpr size_t off_lpc = off_misc + 64;         // float [16] log2 page counts
+// Shared memory and tensor memory of the pair kernel.  SMALL (groups of at
+// most kSmallN members, two CTAs per SM): a fixed 104 KB layout, the query
+// tile and P share one region (P is written after S has been computed), S
+// in TMEM columns [0, 128), O in [128, 256) with the page scores in its
+// first 16 columns until MMA 2 overwrites them.  BIG (one CTA per SM, up to
+// a whole chunk): the layout follows the group size, S in [0, 256), the
+// page scores in [256, 272), O in [384, 512).
+template <bool BIG>
+struct PairCfg {
+  static constexpr size_t kData = BIG ? 216 * 1024 : 104 * 1024;
+  static constexpr uint32_t kTmemCols = BIG ? 512 : 256;
+  static constexpr uint32_t kColSp = BIG ? 256 : 128;
+  static constexpr uint32_t kColO = BIG ? 384 : 128;
+  static constexpr size_t off_misc = kData;            // per-item info
+  static constexpr size_t off_lpc = off_misc + 96;     // float [16] log2 page counts
   static constexpr size_t off_bar = off_lpc + 64;
   static constexpr int kBars = 6;
   static constexpr size_t off_tmem = off_bar + 8 * kBars;
   static constexpr size_t bytes = off_tmem + 16 + 1024;
-  static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
+  static_assert(bytes <= (BIG ? 227 * 1024 : 113 * 1024), "shared memory of the CTAs of one SM");
 };
 
 struct ItemInfo {
@@ -663,21 +732,23 @@ struct ItemInfo {
   uint32_t off_kg, off_vg, off_q, off_p;
 };
 
-__global__ void __launch_bounds__(kThreadsB, 1)
+template <bool BIG>
+__global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
     pf_pair_kernel(const __grid_constant__ PairMaps maps, const __grid_constant__ PrefillArgs a) {
+  using Cfg = PairCfg<BIG>;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~uintptr_t(1023));
-  ItemInfo* info = reinterpret_cast<ItemInfo*>(sm + SmemB::off_misc);
-  float* lpc_s = reinterpret_cast<float*>(sm + SmemB::off_lpc);
-  uint64_t* gfull = reinterpret_cast<uint64_t*>(sm + SmemB::off_bar);
+  ItemInfo* info = reinterpret_cast<ItemInfo*>(sm + Cfg::off_misc);
+  float* lpc_s = reinterpret_cast<float*>(sm + Cfg::off_lpc);
+  uint64_t* gfull = reinterpret_cast<uint64_t*>(sm + Cfg::off_bar);
   uint64_t* q_full = gfull + 1;
   uint64_t* s_full = q_full + 1;
   uint64_t* p_full = s_full + 1;
   uint64_t* o_done = p_full + 1;
   uint64_t* o_free = o_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SmemB::off_tmem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::off_tmem);
   unsigned char* PKs = sm;             // [2 halves][16 rows][128 B]
   unsigned char* PVs = sm + 4096;
 
@@ -694,29 +765,30 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     tc::prefetch_tensormap(&maps.pK);
     tc::prefetch_tensormap(&maps.pV);
   }
-  if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+  if (warp == 0) tc::tmem_alloc(tmem_slot, Cfg::kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int n_items = *a.n_items;
+  const int n_items = a.n_items[BIG ? 1 : 0];
+  const int4* items = a.items + (BIG ? a.big_items : 0);
   const int64_t Gcap = a.Cmax * a.k;
   const float scl = a.scale_log2;
   const int G = a.G, TP = a.TP;
   uint32_t T = 0;      // tiles processed by this CTA (barrier phases)
-  uint32_t ngrp = 0;   // items with a staged group (gfull phases)
+  uint32_t ngrp = 0;   // items processed (gfull phases)
   bool alive = true;
 
   for (int it = blockIdx.x; it < n_items && alive; it += gridDim.x) {
     // ---- the item: its group, bounds-checked, and the operand layout
     if (tid == 0) {
-      const int4 item = a.items[it];
+      const int4 item = items[it];
       const int64_t gflat = item.x;
       const int64_t u = gflat / Gcap, gid = gflat % Gcap, c = gid / a.k;
       const int meta = a.gMeta[gflat];
       const int n = meta & 0xffff, p0 = (meta >> 16) & 0xff, p1 = (meta >> 24) & 0xff;
       const int64_t pslot = (u * a.Cmax + c) * a.P;
-      bool ok = n >= 1 && n <= kChunk && p0 < p1 && p1 <= a.P && p1 - p0 == (n + kPage - 1) / kPage;
+      bool ok = n >= 1 && n <= (BIG ? kChunk : kSmallN) && p0 < p1 && p1 <= a.P && p1 - p0 == (n + kPage - 1) / kPage;
       if (!ok) set_status(a.status, n > kChunk ? LOD_ST_BAD_COUNT : LOD_ST_BAD_PAGE);
       const int off = ok ? (int)a.pBeg[pslot + p0] : 0;
       if (ok && (off < 0 || off + n > kChunk)) {
@@ -733,23 +805,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       f.c = c;
       f.u = u;
       f.R = ok ? (n + 31) / 32 * 32 : 32;
-      const uint32_t kg = (uint32_t)f.R * 256;  // one operand: 2 halves x R rows x 128 B
+      const uint32_t kg = BIG ? (uint32_t)f.R * 256 : 128 * 256;  // one operand: 2 halves x R rows x 128 B
       const int n16 = (f.n + 15) / 16 * 16;
       const uint32_t pbytes = (uint32_t)((n16 + 16 + 63) / 64) * kHalf;
       f.off_kg = 8192;
       f.off_vg = 8192 + kg;
       f.off_q = 8192 + 2 * kg;
-      f.shared_qp = f.off_q + kTileBytes + pbytes > kSmemBData;
+      f.shared_qp = !BIG || f.off_q + kTileBytes + pbytes > Cfg::kData;
       f.off_p = f.shared_qp ? f.off_q : f.off_q + kTileBytes;
       *info = f;
+      const int rs = BIG ? f.R : 128;  // rows of one operand half in shared memory
       if (ok) {
-        mbar_arrive_expect(gfull, 2 * kg + 2 * 4096);
+        mbar_arrive_expect(gfull, 2 * (uint32_t)f.R * 256 + 2 * 4096);
         const int row0 = (int)((u * a.Cmax + c) * kChunk + off);
         for (int bx = 0; bx < f.R / 32; ++bx)
           for (int h = 0; h < 2; ++h) {
-            tc::tma_load_2d(sm + f.off_kg + h * (f.R * 128) + bx * 4096, &maps.mK, 64 * h, row0 + 32 * bx, gfull,
+            tc::tma_load_2d(sm + f.off_kg + h * (rs * 128) + bx * 4096, &maps.mK, 64 * h, row0 + 32 * bx, gfull,
                             0x1000000000000000ull);
-            tc::tma_load_2d(sm + f.off_vg + h * (f.R * 128) + bx * 4096, &maps.mV, 64 * h, row0 + 32 * bx, gfull,
+            tc::tma_load_2d(sm + f.off_vg + h * (rs * 128) + bx * 4096, &maps.mV, 64 * h, row0 + 32 * bx, gfull,
                             0x1000000000000000ull);
           }
         for (int h = 0; h < 2; ++h) {
@@ -764,6 +837,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const ItemInfo f = *info;
     const int n16 = (f.n + 15) / 16 * 16;
     const int ntiles = (f.count + kRows - 1) / kRows;
+    const int rs = BIG ? f.R : 128;
     unsigned char* KG = sm + f.off_kg;
     unsigned char* VG = sm + f.off_vg;
     unsigned char* Qs = sm + f.off_q;
@@ -778,30 +852,32 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const uint32_t idO = tc::idesc_bf16(128, 128, false, true);
         const uint32_t qb = smem_u32(Qs), kb = smem_u32(KG), vb = smem_u32(VG), pb = smem_u32(Ps);
         const uint32_t pkb = smem_u32(PKs), pvb = smem_u32(PVs);
-        const uint32_t hs = (uint32_t)f.R * 128;
+        const uint32_t hs = (uint32_t)rs * 128;
         for (int t = 0; t < ntiles && go; ++t) {
           const uint32_t Tt = T + t;
           go = mbar_wait(q_full, Tt & 1u, a.status);
+          // (O is free once the epilogue of the previous tile has read it; the
+          // page scores share its columns in the SMALL layout)
+          if (go && Tt > 0) go = mbar_wait(o_free, (Tt - 1) & 1u, a.status);
           if (!go) break;
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t ad = tc::desc_kmajor_sw128(qb + (kk >> 2) * kHalf + (kk & 3) * 32);
             tc::mma_bf16(tmem, ad, tc::desc_kmajor_sw128(kb + (kk >> 2) * hs + (kk & 3) * 32), idS, kk > 0);
-            tc::mma_bf16(tmem + 256, ad, tc::desc_kmajor_sw128(pkb + (kk >> 2) * 2048 + (kk & 3) * 32), idP,
+            tc::mma_bf16(tmem + Cfg::kColSp, ad, tc::desc_kmajor_sw128(pkb + (kk >> 2) * 2048 + (kk & 3) * 32), idP,
                          kk > 0);
           }
           tc::mma_commit(s_full);
           go = mbar_wait(p_full, Tt & 1u, a.status);
-          if (go && Tt > 0) go = mbar_wait(o_free, (Tt - 1) & 1u, a.status);
           if (!go) break;
           tc::fence_after_sync();
           for (int kk = 0; kk < n16 / 16; ++kk)
-            tc::mma_bf16(tmem + 384, tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32),
+            tc::mma_bf16(tmem + Cfg::kColO, tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32),
                          tc::desc_mnmajor_sw128(vb + kk * 2048, hs), idO, kk > 0);
           {
             const int kk = n16 / 16;  // the coarse pages' weights and mean values
-            tc::mma_bf16(tmem + 384, tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32),
+            tc::mma_bf16(tmem + Cfg::kColO, tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32),
                          tc::desc_mnmajor_sw128(pvb, 2048), idO, true);
           }
           tc::mma_commit(o_done);
@@ -846,7 +922,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       // not inputs of this group: zero their values for MMA 2
       alive = mbar_wait(gfull, ngrp & 1u, a.status);
       if (alive) {
-        const int hs = f.R * 128;
+        const int hs = rs * 128;
         for (int x = r; x < (n16 - f.n) * 16; x += 128) {
           const int row = f.n + x / 16, ch = x % 16;
           *reinterpret_cast<uint4*>(VG + (ch >> 3) * hs + sw_off(row, ch)) = make_uint4(0, 0, 0, 0);
@@ -858,6 +934,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tc::fence_proxy_async();
       }
       bar_named_sync(kBarSoftB, 128);
+      const int nblk = (f.np + 3) / 4;  // 64-column blocks of member scores (4 pages each)
       for (int t = 0; t < ntiles && alive; ++t) {
         const uint32_t Tt = T + t;
         alive = __all_sync(0xffffffffu, mbar_wait(s_full, Tt & 1u, a.status));
@@ -866,7 +943,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (t + 1 < ntiles && !f.shared_qp) gather(t + 1, pid_next);
         // page scores and this row's top-TP pages (score desc, slot asc)
         float sp[16];
-        tc::tmem_ld16(tmem + tl + 256, sp);
+        tc::tmem_ld16(tmem + tl + Cfg::kColSp, sp);
         uint32_t selm = 0;
         if (TP == 0 || TP >= f.np) {
           selm = (1u << f.np) - 1u;
@@ -888,41 +965,52 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
         // pass 1: the row's max over its exact members and coarse pages
         float xc[16];
-        float m = -INFINITY;
+        float ma[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const bool coarse = TP > 0 && j < f.np && !((selm >> j) & 1u);
           xc[j] = coarse ? fmaf(sp[j], scl, lpc_s[j]) : -INFINITY;
-          m = fmaxf(m, xc[j]);
+          ma[j & 3] = fmaxf(ma[j & 3], xc[j]);
         }
-        for (int j = 0; j < f.np; ++j) {
-          float v[16];
-          tc::tmem_ld16(tmem + tl + 16 * j, v);
-          if ((selm >> j) & 1u) {
+        for (int bb = 0; bb < nblk; ++bb) {
+          float v[64];
+          tc::tmem_ld32xN<2>(tmem + tl + 64 * bb, v);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (16 * j + e < f.n) m = fmaxf(m, v[e] * scl);
+          for (int jj = 0; jj < 4; ++jj) {
+            const int j = 4 * bb + jj;
+            if ((selm >> j) & 1u) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (16 * j + e < f.n) ma[e & 3] = fmaxf(ma[e & 3], v[16 * jj + e] * scl);
+            }
           }
         }
+        const float m = fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3]));
         const float mu = m == -INFINITY ? 0.f : m;
         // pass 2: the weights into P (members, then the coarse pages)
-        float l = 0.f;
-        for (int j = 0; j < f.np; ++j) {
-          float v[16];
-          tc::tmem_ld16(tmem + tl + 16 * j, v);
-          const bool on = (selm >> j) & 1u;
-          float p[16];
+        float la[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int bb = 0; bb < nblk; ++bb) {
+          float v[64];
+          tc::tmem_ld32xN<2>(tmem + tl + 64 * bb, v);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            p[e] = (on && 16 * j + e < f.n) ? ex2_approx(fmaf(v[e], scl, -mu)) : 0.f;
-            l += p[e];
-          }
+          for (int jj = 0; jj < 4; ++jj) {
+            const int j = 4 * bb + jj;
+            if (j < f.np) {
+              const bool on = (selm >> j) & 1u;
+              float p[16];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int ch = 2 * j + h;
-            *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
-                make_uint4(pack_bf16x2(p[8 * h], p[8 * h + 1]), pack_bf16x2(p[8 * h + 2], p[8 * h + 3]),
-                           pack_bf16x2(p[8 * h + 4], p[8 * h + 5]), pack_bf16x2(p[8 * h + 6], p[8 * h + 7]));
+              for (int e = 0; e < 16; ++e) {
+                p[e] = (on && 16 * j + e < f.n) ? ex2_approx(fmaf(v[16 * jj + e], scl, -mu)) : 0.f;
+                la[e & 3] += p[e];
+              }
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int ch = 2 * j + h;
+                *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
+                    make_uint4(pack_bf16x2(p[8 * h], p[8 * h + 1]), pack_bf16x2(p[8 * h + 2], p[8 * h + 3]),
+                               pack_bf16x2(p[8 * h + 4], p[8 * h + 5]), pack_bf16x2(p[8 * h + 6], p[8 * h + 7]));
+              }
+            }
           }
         }
         {
@@ -930,7 +1018,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             p[e] = xc[e] == -INFINITY ? 0.f : ex2_approx(xc[e] - mu);
-            l += p[e];
+            la[e & 3] += p[e];
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -940,6 +1028,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                            pack_bf16x2(p[8 * h + 4], p[8 * h + 5]), pack_bf16x2(p[8 * h + 6], p[8 * h + 7]));
           }
         }
+        const float l = (la[0] + la[1]) + (la[2] + la[3]);
         tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncwarp();
@@ -951,22 +1040,25 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const bool vp = pid_cur >= 0 && f.ok;
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float ov[32];
-          tc::tmem_ld32(tmem + tl + 384 + 32 * c, ov);
+        for (int hh = 0; hh < 2; ++hh) {
+          float ov[64];
+          tc::tmem_ld32xN<2>(tmem + tl + Cfg::kColO + 64 * hh, ov);
+          if (hh == 1) {
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+          }
           if (vp) {
-            uint4* dst = reinterpret_cast<uint4*>(a.po + pid_cur * D + 32 * c);
+            uint4* dst = reinterpret_cast<uint4*>(a.po + pid_cur * D + 64 * hh);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 8; ++q)
               dst[q] = make_uint4(pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
                                   pack_bf16x2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv),
                                   pack_bf16x2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv),
                                   pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
           }
         }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(o_free);
+        if (t + 1 < ntiles && f.shared_qp) gather(t + 1, pid_next);
         if (pid_cur >= 0) {
           a.plse[pid_cur] = vp && l > 0.f ? m + log2f(l) : -INFINITY;
           if (a.sel_pages) {
@@ -990,7 +1082,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             }
           }
         }
-        if (t + 1 < ntiles && f.shared_qp) gather(t + 1, pid_next);
         pid_cur = pid_next;
       }
       // (a gathered tile that was never consumed: let its copies land)
@@ -1003,7 +1094,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   if (!alive && tid == 0) set_status(a.status, LOD_ST_TIMEOUT);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 512);
+  if (warp == 0) tc::tmem_dealloc(tmem, Cfg::kTmemCols);
 }
 
 // ================================================================== merge
@@ -1027,8 +1118,26 @@ __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ P
   for (int k = 0; k < a.G; ++k)
     if (a.sel[wr * a.G + k] >= 0) M = fmaxf(M, a.plse[wr * a.G + k]);
   const float cs = m == -INFINITY ? 0.f : ex2_approx(m - M);
-  float L = l * cs;
-  float o0 = acc.x * cs, o1 = acc.y * cs, o2 = acc.z * cs, o3 = acc.w * cs;
+  // the opened groups' coarse terms leave the row state (finer entries,
+  // the pairs' partials, replace them)
+  float L = l, o0 = acc.x, o1 = acc.y, o2 = acc.z, o3 = acc.w;
+  const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
+  for (int k = 0; k < a.G; ++k) {
+    const int gid = a.sel[wr * a.G + k];
+    if (gid < 0 || m == -INFINITY) continue;
+    const float wk = a.cw[wr * a.G + k];
+    const uint2 raw = *reinterpret_cast<const uint2*>(a.gV + ((u * a.Cmax * a.k + gid) * D + 4 * lane));
+    L -= wk;
+    o0 = fmaf(-wk, __uint_as_float(raw.x << 16), o0);
+    o1 = fmaf(-wk, __uint_as_float(raw.x & 0xffff0000u), o1);
+    o2 = fmaf(-wk, __uint_as_float(raw.y << 16), o2);
+    o3 = fmaf(-wk, __uint_as_float(raw.y & 0xffff0000u), o3);
+  }
+  L *= cs;
+  o0 *= cs;
+  o1 *= cs;
+  o2 *= cs;
+  o3 *= cs;
   for (int k = 0; k < a.G; ++k) {
     if (a.sel[wr * a.G + k] < 0) {
       if (a.sel_pages && lane < a.TP) a.sel_pages[(orow * a.G + k) * a.TP + lane] = -1;
@@ -1053,7 +1162,7 @@ __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ P
 }  // namespace
 
 size_t prefill_tc_scan_smem() { return SmemA::bytes; }
-size_t prefill_tc_pair_smem() { return SmemB::bytes; }
+size_t prefill_tc_pair_smem() { return PairCfg<true>::bytes; }
 
 cudaError_t launch_prefill_tc_wave(const PrefillArgs& a, const TcMaps& maps, const PairMaps& pmaps, int num_sms,
                                    cudaStream_t stream) {
@@ -1081,9 +1190,13 @@ cudaError_t launch_prefill_tc_wave(const PrefillArgs& a, const TcMaps& maps, con
   pf_scatter_kernel<<<(unsigned)(sblocks > 0 ? sblocks : 1), 256, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = set_smem_once<pf_pair_kernel>(SmemB::bytes);
+  e = set_smem_once<pf_pair_kernel<false>>(PairCfg<false>::bytes, true);
+  if (e == cudaSuccess) e = set_smem_once<pf_pair_kernel<true>>(PairCfg<true>::bytes, true);
   if (e != cudaSuccess) return e;
-  pf_pair_kernel<<<(unsigned)num_sms, kThreadsB, SmemB::bytes, stream>>>(pmaps, a);
+  pf_pair_kernel<false><<<(unsigned)(2 * num_sms), kThreadsB, PairCfg<false>::bytes, stream>>>(pmaps, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  pf_pair_kernel<true><<<(unsigned)num_sms, kThreadsB, PairCfg<true>::bytes, stream>>>(pmaps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)a.B * a.Hq * a.NW;

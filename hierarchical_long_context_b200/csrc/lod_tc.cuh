@@ -63,6 +63,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M rows x K, bf16) read from tensor
+// memory, row i in lane i, K elements packed two per 32-bit column (the
+// lower k in the low half); one K = 16 step reads 8 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u));
+}
+
 // Arrive once on `bar` when every MMA this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -144,6 +156,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 * N consecutive fp32 columns of this thread's TMEM lane, as N loads
+// in flight together and one wait.  Each value then passes through an empty
+// asm that reads and writes it, so no use is scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld32xN(uint32_t taddr, float (&v)[32 * N]) {
+  uint32_t r[32 * N];
+#pragma unroll
+  for (int b = 0; b < N; ++b)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[32 * b + 0]), "=r"(r[32 * b + 1]), "=r"(r[32 * b + 2]), "=r"(r[32 * b + 3]),
+          "=r"(r[32 * b + 4]), "=r"(r[32 * b + 5]), "=r"(r[32 * b + 6]), "=r"(r[32 * b + 7]),
+          "=r"(r[32 * b + 8]), "=r"(r[32 * b + 9]), "=r"(r[32 * b + 10]), "=r"(r[32 * b + 11]),
+          "=r"(r[32 * b + 12]), "=r"(r[32 * b + 13]), "=r"(r[32 * b + 14]), "=r"(r[32 * b + 15]),
+          "=r"(r[32 * b + 16]), "=r"(r[32 * b + 17]), "=r"(r[32 * b + 18]), "=r"(r[32 * b + 19]),
+          "=r"(r[32 * b + 20]), "=r"(r[32 * b + 21]), "=r"(r[32 * b + 22]), "=r"(r[32 * b + 23]),
+          "=r"(r[32 * b + 24]), "=r"(r[32 * b + 25]), "=r"(r[32 * b + 26]), "=r"(r[32 * b + 27]),
+          "=r"(r[32 * b + 28]), "=r"(r[32 * b + 29]), "=r"(r[32 * b + 30]), "=r"(r[32 * b + 31])
+        : "r"(taddr + 32 * b));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32 * N; ++i) {
+    asm volatile("" : "+r"(r[i]));
+    v[i] = __uint_as_float(r[i]);
+  }
 }
 
 // Store 32 consecutive fp32 columns of this thread's TMEM lane and wait for them.
