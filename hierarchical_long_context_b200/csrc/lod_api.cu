@@ -255,9 +255,9 @@ constexpr int kItemRows = 1024;                    // pairs per work item of the
 constexpr int64_t kPrefillWaveBudget = (int64_t)2 << 30;  // workspace bytes a wave may use
 
 // Workspace bytes per wave row: state (132 floats), and per opened group
-// its id, its coarse weight, its log-sum-exp, its bf16 output and its
-// pair-list entry.
-int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 2 * p->d + 4); }
+// its id, its coarse weight, its place in the group's run, its log-sum-exp,
+// its bf16 output and its pair-list entry.
+int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 4 + 2 * p->d + 4); }
 
 // Query positions per wave: a multiple of chunk, as many as the budget allows
 // (at least one chunk, at most 128), never more than the cache holds.
@@ -273,7 +273,7 @@ int64_t pf_wave(const lod_params* p) {
 }
 
 struct PfLayout {
-  size_t state, sel, cw, plse, po, list, cnt, off, items, n_items, total;
+  size_t state, sel, cw, pos, plse, po, list, cnt, off, items, n_items, total;
   int64_t NW, Gtot, max_items;
 };
 
@@ -293,6 +293,7 @@ PfLayout pf_layout(const lod_params* p) {
   L.state = take(sizeof(float) * 132 * (size_t)rows);
   L.sel = take(sizeof(int32_t) * (size_t)pairs);
   L.cw = take(sizeof(float) * (size_t)pairs);
+  L.pos = take(sizeof(int32_t) * (size_t)pairs);
   L.plse = take(sizeof(float) * (size_t)pairs);
   L.po = take((size_t)2 * p->d * (size_t)pairs);
   L.list = take(sizeof(int32_t) * (size_t)pairs);
@@ -635,6 +636,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.state = reinterpret_cast<float*>(w + L.state);
     a.sel = reinterpret_cast<int32_t*>(w + L.sel);
     a.cw = reinterpret_cast<float*>(w + L.cw);
+    a.pos = reinterpret_cast<int32_t*>(w + L.pos);
     a.plse = reinterpret_cast<float*>(w + L.plse);
     a.po = reinterpret_cast<__nv_bfloat16*>(w + L.po);
     a.list = reinterpret_cast<int32_t*>(w + L.list);

@@ -164,11 +164,12 @@ struct PrefillArgs {
   float* state;             // [rows][132]: m, l (log2 units), -, -, acc[d] (opened groups included)
   int32_t* sel;             // [rows][G] opened group ids, best first, -1 padded
   float* cw;                // [rows][G] weight of the opened group's coarse term, relative to m
+  int32_t* pos;             // [rows][G] place of the pair in its group's run
   float* plse;              // [rows][G] pair log-sum-exp (log2 units)
   __nv_bfloat16* po;        // [rows][G][d] pair output (normalised)
   int32_t* list;            // pair ids (row * G + rank) grouped by (unit, group)
   int32_t* cnt;             // [Gtot] pairs per (unit, group)
-  int32_t* off;             // [Gtot] first pair of each (unit, group); advanced by the scatter
+  int32_t* off;             // [Gtot] first pair of each (unit, group)
   int4* items;              // work items {unit * Cmax * k + group, first pair, pairs, 0}: small groups
                             // from items[0], large groups from items[big_items]
   int64_t big_items;

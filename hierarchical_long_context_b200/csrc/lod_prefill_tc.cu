@@ -61,10 +61,18 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk16) {  // 16-byte c
 
 // ================================================================== phase A
 
-constexpr int kThreadsA = 320;   // warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax, 6-9 top-G + epilogue
-constexpr int kCandCap = 32;     // buffered top-G candidates per row
+// Warpgroups of the scan: 0 (warps 0-3) warp 0 TMA copies, warp 1 MMA
+// issue; 1 (warps 4-7) softmax; 2 and 3 (warps 8-15) the top-G groups of
+// key columns [0, 64) and [64, 128) of every group tile, and (group 2) the
+// epilogue.  Registers move from warpgroup 0 to the others:
+// 128 x (40 + 200 + 136 + 136) = 65536, the register file.
+constexpr int kThreadsA = 512;
+constexpr int kRegCtl = 40, kRegSoft = 200, kRegSel = 136;
+constexpr int kCandCap = 28;     // buffered top-G candidates per row and column half
 constexpr int kBarLncA = 1;      // named barrier of the softmax warps
-constexpr int kBarEpiA = 2;      // named barrier of warps 2-9 (hand-over of the softmax state)
+constexpr int kBarEpiA = 2;      // named barrier of warpgroups 1 and 2 (hand-over of the softmax state)
+constexpr int kBarSelA = 3;      // named barrier of warpgroups 2 and 3 (merge of the two column halves)
+constexpr int kBarEndA = 4;      // named barrier of warpgroups 0-2 before TMEM is released
 
 // Tensor memory of the scan: S double-buffered in columns [0, 256), O in
 // [256, 384), the query tile (bf16 pairs, MMA 1's A operand) in [384, 448).
@@ -74,11 +82,11 @@ struct SmemA {
   static constexpr size_t off_K = 0;                          // [2 stages][2 halves][128][128 B]
   static constexpr size_t off_V = off_K + 2 * kTileBytes;     // [2 stages]
   static constexpr size_t off_P = off_V + 2 * kTileBytes;     // [2 halves][128][128 B]
-  static constexpr size_t off_cand = off_P + kTileBytes;      // float2 [128][kCandCap + 1] (+1: a junk slot)
-  static constexpr size_t off_meta = off_cand + 128 * (kCandCap + 1) * 8;  // int [2][128]
+  static constexpr size_t off_cand = off_P + kTileBytes;      // float2 [2][128][kCandCap + 1] (+1: a junk slot)
+  static constexpr size_t off_meta = off_cand + 2 * 128 * (kCandCap + 1) * 8;  // int [2][128]
   static constexpr size_t off_lnc = off_meta + 2 * 128 * 4;   // float [2][128]
   static constexpr size_t off_ml = off_lnc + 2 * 128 * 4;   // float2 [128] softmax state handed over
-  static constexpr int kBars = 17;
+  static constexpr int kBars = 18;
   static constexpr size_t off_bar = off_ml + 128 * 8;
   static constexpr size_t off_misc = off_bar + 8 * kBars;     // tmem slot, abort flag
   static constexpr size_t bytes = off_misc + 16 + 1024;
@@ -106,6 +114,34 @@ __device__ __forceinline__ void topk_insert(float (&s)[GM], int (&ix)[GM], float
     s[k] = ns;
     ix[k] = ni;
   }
+}
+
+// Insert (v, id) by the full ranking (score desc, id asc), for entries that
+// do not arrive in id order.
+template <int GM>
+__device__ __forceinline__ void topk_insert_ranked(float (&s)[GM], int (&ix)[GM], float v, int id) {
+  bool act = false;
+  float cs = v;
+  int ci = id;
+#pragma unroll
+  for (int k = 0; k < GM; ++k) {
+    act = act || v > s[k] || (v == s[k] && (unsigned)id < (unsigned)ix[k]);
+    const float ns = act ? cs : s[k];
+    const int ni = act ? ci : ix[k];
+    cs = act ? s[k] : cs;
+    ci = act ? ix[k] : ci;
+    s[k] = ns;
+    ix[k] = ni;
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Merge a row's buffered candidates (ascending ids: ties keep the earlier
@@ -153,6 +189,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   uint64_t* o_done = p_full + 1;
   uint64_t* fin = o_done + 1;
   uint64_t* lnc_ready = fin + 1;  // [2]: ln counts of a group tile written
+  uint64_t* q_ready = lnc_ready + 2;  // the query tile is in TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SmemA::off_misc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + SmemA::off_misc + 4);
 
@@ -184,14 +221,15 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
       mbar_init(&vfull[i], 1 + 32);
-      mbar_init(&vempty[i], 1 + 4);  // MMA 2 done + the four top-G warps done with the tile's counts
+      mbar_init(&vempty[i], 1);
       mbar_init(&lnc_ready[i], 4);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 8);
+      mbar_init(&s_free[i], 12);  // four softmax warps + eight top-G warps
     }
     mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
+    mbar_init(q_ready, 4);
     *abort_s = 0;
     fence_mbar_init();
     tc::prefetch_tensormap(&maps.gK);
@@ -200,41 +238,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     tc::prefetch_tensormap(&maps.V);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
-  // the query rows, loaded while TMEM is allocated (row r = position r / g, head r % g)
-  uint4 qrow[16];
-  if (warp >= 2 && warp < 6) {
-    const int r = 32 * (warp & 3) + lane;
-    const int64_t pi = pos0 + r / a.g;
-    const int hq = kvh * a.g + r % a.g;
-    const bool okr = pi < pos_end;
-    const __nv_bfloat16* src = a.q + (((int64_t)b * a.Hq + hq) * a.Tq + (okr ? pi : 0)) * D;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) qrow[c] = okr ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  // ---- the query tile into TMEM lane r (MMA 1's A operand)
-  if (warp >= 2 && warp < 6) {
-    const uint32_t tl = (uint32_t)(32 * (warp & 3)) << 16;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float qv[32];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w = qrow[8 * h + c];
-        qv[4 * c] = __uint_as_float(w.x);
-        qv[4 * c + 1] = __uint_as_float(w.y);
-        qv[4 * c + 2] = __uint_as_float(w.z);
-        qv[4 * c + 3] = __uint_as_float(w.w);
-      }
-      tc::tmem_st32(tmem + tl + kColQ + 32 * h, qv);
-    }
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
 
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*abort_s) return false;
@@ -244,6 +251,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   };
   const uint64_t l2pol = l2_policy_evict_first();
 
+  if (warp < 4) regs_dec<kRegCtl>();  // (each warpgroup's branch opens with its register count)
   if (warp == 0) {
     // ================================================================ producer
     const int32_t* gM = a.gMeta + grow0;
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         tc::mma_commit(o_done);
         return true;
       };
-      bool go = true, any = false;
+      bool go = wait(q_ready, 0), any = false;  // the query tile, staged by the softmax warps
       for (int i = 0; i < ntile && go; ++i) {
         if (!wait(&kfull[i & 1], (uint32_t)(i >> 1) & 1u)) break;
         if (i >= 2 && !wait(&s_free[i & 1], (uint32_t)((i - 2) >> 1) & 1u)) break;
@@ -341,11 +349,37 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ================================================================ softmax (warps 2-5)
+  } else if (warp < 4) {
+    // (warps 2 and 3: no role)
+  } else if (warp < 8) {
+    // ================================================================ softmax (warps 4-7)
+    regs_inc<kRegSoft>();
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;  // query row of this thread (and the key row it stages)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
+    {
+      // the query tile into TMEM lane r (MMA 1's A operand): row r = position r / g, head r % g
+      const int64_t pi = pos0 + r / a.g;
+      const int hq = kvh * a.g + r % a.g;
+      const bool okr = pi < pos_end;
+      const __nv_bfloat16* src = a.q + (((int64_t)b * a.Hq + hq) * a.Tq + (okr ? pi : 0)) * D;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float qv[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = okr ? __ldg(reinterpret_cast<const uint4*>(src) + 8 * h + c) : make_uint4(0, 0, 0, 0);
+          qv[4 * c] = __uint_as_float(w.x);
+          qv[4 * c + 1] = __uint_as_float(w.y);
+          qv[4 * c + 2] = __uint_as_float(w.z);
+          qv[4 * c + 3] = __uint_as_float(w.w);
+        }
+        tc::tmem_st32(tmem + tl + kColQ + 32 * h, qv);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
     const int64_t t_row = a.q_begin + pos0 + r / a.g;
     const float scl = a.scale_log2;
     float m = -INFINITY, l = 0.f;
@@ -395,34 +429,33 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       // window and sink keys at positions kpos0 + j <= lim are in this row's softmax
       const int64_t lim = snk ? nsk - 1 : t_row;
       const int rel = grp ? 127 : (int)(lim - kpos0 < -1 ? -1 : (lim - kpos0 > 127 ? 127 : lim - kpos0));
-      // the logits (log2 units) of key columns [64 h, 64 h + 64), minus `sub`
-      auto logits = [&](int h, float (&x)[64], float sub) {
-        tc::tmem_ld32xN<2>(sb + 64 * h, x);
+      // the logits (log2 units) of key columns [32 c, 32 c + 32), minus `sub`
+      // (one copy of the code: the loops over chunks are not unrolled)
+      auto logits = [&](int c, float (&y)[32], float sub) {
+        tc::tmem_ld32(sb + 32 * c, y);
         if (grp) {
 #pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(lc + 64 * h + 4 * e4);
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lc + 32 * c + 4 * e4);
             const float lv[4] = {l4.x - sub, l4.y - sub, l4.z - sub, l4.w - sub};
 #pragma unroll
             for (int e = 0; e < 4; ++e)  // fmaxf drops NaN: a group outside the softmax gives -inf
-              x[4 * e4 + e] = fmaxf(fmaf(x[4 * e4 + e], scl, lv[e]), -INFINITY);
+              y[4 * e4 + e] = fmaxf(fmaf(y[4 * e4 + e], scl, lv[e]), -INFINITY);
           }
-        } else if (rel >= 127) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = fmaf(x[e], scl, -sub);
         } else {
+          const int rc = rel - 32 * c;  // columns e <= rc are in
 #pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = 64 * h + e <= rel ? fmaf(x[e], scl, -sub) : -INFINITY;
+          for (int e = 0; e < 32; ++e) y[e] = e <= rc ? fmaf(y[e], scl, -sub) : -INFINITY;
         }
       };
       // ---- pass 1: the logit max
       float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent max chains
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float x[64];
-        logits(h, x, 0.f);
+      for (int c = 0; c < 4; ++c) {
+        float y[32];
+        logits(c, y, 0.f);
 #pragma unroll
-        for (int e = 0; e < 64; ++e) xa[e & 3] = fmaxf(xa[e & 3], x[e]);
+        for (int e = 0; e < 32; ++e) xa[e & 3] = fmaxf(xa[e & 3], y[e]);
       }
       const float xm = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
       // the reference max moves when a logit exceeds it by more than kTau2
@@ -456,18 +489,18 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       // ---- pass 2: the weights 2^(logit - m) into P
       float la[4] = {0.f, 0.f, 0.f, 0.f};  // independent sum chains
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float x[64];
-        logits(h, x, mu);
+      for (int c = 0; c < 4; ++c) {
+        float y[32];
+        logits(c, y, mu);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = ex2_approx(x[8 * q + e]);
+            p[e] = ex2_approx(y[8 * q + e]);
             la[e & 3] += p[e];
           }
-          const int ch = 8 * h + q;
+          const int ch = 4 * c + q;
           *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
               make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
                          pack_bf16x2(p[6], p[7]));
@@ -486,9 +519,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     ml_s[r] = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
     bar_named_sync(kBarEpiA, 256);
   } else {
-    // ================================================================ top-G and epilogue (warps 6-9)
+    // ================================================================ top-G (warps 8-15) and epilogue (8-11)
+    regs_inc<kRegSel>();
     const int q4 = warp & 3;
     const int r = 32 * q4 + lane;
+    const int half = (warp - 8) >> 2;  // key columns [64 half, 64 half + 64) of every group tile
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     const int64_t pi = pos0 + r / a.g;
     const int hq = kvh * a.g + r % a.g;
@@ -504,7 +539,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     float thr = -INFINITY;
     // this row's buffer of candidates (scores above the running G-th best,
     // not yet merged into the sorted list ts/ti)
-    float2* cbuf = cand_s + r * (kCandCap + 1);
+    float2* cbuf = cand_s + (half * 128 + r) * (kCandCap + 1);
     int ncand = 0;
     bool alive = true;
     for (int i = 0; i < ntile; ++i) {
@@ -515,54 +550,63 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       if (!alive) break;
       if (grp) {
         tc::fence_after_sync();
-        const float* lc = lnc_s + st * 128;
+        const float* lc = lnc_s + st * 128 + 64 * half;
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float v[64];
-          tc::tmem_ld32xN<2>(tmem + tl + (uint32_t)st * 128 + 64 * h, v);
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float v[32];
+          tc::tmem_ld32(tmem + tl + (uint32_t)st * 128 + 64 * half + 32 * c2, v);
+          // the raw scores of the groups in the softmax (-inf: outside)
+          float ca[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const int c = 2 * h + c2;
-            // the raw scores of the groups in the softmax (-inf: outside)
-            float ca[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lc + 32 * c2 + 4 * e4);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 l4 = *reinterpret_cast<const float4*>(lc + 32 * c + 4 * e4);
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float& x = v[32 * c2 + 4 * e4 + e];
-                x = (valid && lv[e] != -INFINITY) ? x : -INFINITY;
-                ca[e] = fmaxf(ca[e], x);
-              }
+            for (int e = 0; e < 4; ++e) {
+              float& y = v[4 * e4 + e];
+              y = (valid && lv[e] != -INFINITY) ? y : -INFINITY;
+              ca[e] = fmaxf(ca[e], y);
             }
-            const float cm = fmaxf(fmaxf(ca[0], ca[1]), fmaxf(ca[2], ca[3]));
-            // candidates: scores above the running G-th best go to the buffer
-            // (merged into the sorted list whenever 16 more might not fit)
-            if (__any_sync(0xffffffffu, cm > thr)) {
-              const int id0 = i * 128 + 32 * c;
+          }
+          const float cm = fmaxf(fmaxf(ca[0], ca[1]), fmaxf(ca[2], ca[3]));
+          // candidates: scores above the running G-th best go to the buffer
+          // (merged into the sorted list whenever 16 more might not fit)
+          if (__any_sync(0xffffffffu, cm > thr)) {
+            const int id0 = i * 128 + 64 * half + 32 * c2;
 #pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                if (__any_sync(0xffffffffu, ncand > kCandCap - 16)) topk_merge<GM>(ts, ti, thr, ncand, cbuf);
+            for (int hh = 0; hh < 2; ++hh) {
+              if (__any_sync(0xffffffffu, ncand > kCandCap - 16)) topk_merge<GM>(ts, ti, thr, ncand, cbuf);
 #pragma unroll
-                for (int e = 16 * hh; e < 16 * hh + 16; ++e) {  // (branch-free: a miss writes the junk slot)
-                  const float x = v[32 * c2 + e];
-                  const bool hit = x > thr;
-                  cbuf[hit ? ncand : kCandCap] = make_float2(x, __int_as_float(id0 + e));
-                  ncand += hit ? 1 : 0;
-                }
+              for (int e = 16 * hh; e < 16 * hh + 16; ++e) {  // (branch-free: a miss writes the junk slot)
+                const float y = v[e];
+                const bool hit = y > thr;
+                cbuf[hit ? ncand : kCandCap] = make_float2(y, __int_as_float(id0 + e));
+                ncand += hit ? 1 : 0;
               }
             }
           }
         }
-        if (i == gt - 1) topk_merge<GM>(ts, ti, thr, ncand, cbuf);  // the list is final
+        if (i == gt - 1) topk_merge<GM>(ts, ti, thr, ncand, cbuf);  // this half's list is final
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_free[st]);
-        mbar_arrive(&vempty[st]);  // (the stage's counts may be overwritten)
-      }
+      if (lane == 0) mbar_arrive(&s_free[st]);
+    }
+    // ---- the two halves' lists into one (warpgroup 3 hands its list over)
+    float2* hand = cand_s + (128 + r) * (kCandCap + 1);  // (warpgroup 3's buffer, free now)
+    if (half == 1) {
+#pragma unroll
+      for (int k = 0; k < GM; ++k) hand[k] = make_float2(ts[k], __int_as_float(ti[k]));
+      hand[GM] = make_float2(alive ? 1.f : 0.f, 0.f);
+    }
+    bar_named_sync(kBarSelA, 256);
+    if (half == 1) return;  // (warpgroup 3 is done; the CTA's last barrier counts warpgroups 0-2 only)
+    if (hand[GM].x == 0.f) alive = false;
+#pragma unroll
+    for (int k = 0; k < GM; ++k) {
+      const float2 e = hand[k];
+      const int id = __float_as_int(e.y);
+      if (id >= 0) topk_insert_ranked<GM>(ts, ti, e.x, id);
     }
     // ---------------------------------------------------------------- epilogue
     bar_named_sync(kBarEpiA, 256);
@@ -590,6 +634,14 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       }
     }
     if (valid) {
+      // the pairs' places in their groups' runs: every atomic is issued
+      // before any result is used, so their round trips overlap
+      int pos[GM];
+#pragma unroll
+      for (int k = 0; k < GM; ++k) {
+        const int gid = alive ? ti[k] : -1;
+        pos[k] = (k >= GM - a.G && gid >= 0) ? atomicAdd(a.cnt + grow0 + gid, 1) : -1;
+      }
       *reinterpret_cast<float2*>(stp) = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
       const float mu = m == -INFINITY ? 0.f : m;
 #pragma unroll
@@ -604,14 +656,14 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           }
           a.sel[wr * a.G + j] = gid;
           a.cw[wr * a.G + j] = wk;
+          a.pos[wr * a.G + j] = pos[k];
           if (a.sel_groups) a.sel_groups[orow * a.G + j] = gid;
-          if (gid >= 0) atomicAdd(a.cnt + grow0 + gid, 1);  // (result unused: a reduction, no round trip)
         }
       }
     }
   }
   tc::fence_before_sync();
-  __syncthreads();
+  bar_named_sync(kBarEndA, 384);  // warpgroups 0-2 (warpgroup 3 has left)
   if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
@@ -665,7 +717,7 @@ __global__ void __launch_bounds__(kPlanThreads) pf_plan_kernel(const __grid_cons
 #pragma unroll
     for (int q = 0; q < 3; ++q) ex[q] = carry[q] + (warp > 0 ? wsum[q][warp - 1] : 0) + y[q] - x[q];
     if (gf < a.Gtot) {
-      a.off[gf] = (int32_t)ex[0];  // the scatter advances it to the run's end
+      a.off[gf] = (int32_t)ex[0];
       int4* dst = big ? a.items + a.big_items + ex[2] : a.items + ex[1];
       for (int t = 0; t < ni; ++t) {
         const int n = c - t * a.item_rows < a.item_rows ? c - t * a.item_rows : a.item_rows;
@@ -682,8 +734,9 @@ __global__ void __launch_bounds__(kPlanThreads) pf_plan_kernel(const __grid_cons
   }
 }
 
-// Every (row, group) pair into its group's run of the pair list (the order
-// inside a run is arbitrary: every pair is computed on its own).
+// Every (row, group) pair into its group's run of the pair list, at the
+// place its counting atomic returned (the order inside a run is arbitrary:
+// every pair is computed on its own).
 __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__ PrefillArgs a) {
   const int64_t n = (int64_t)a.B * a.Hq * a.NW * a.G;
   for (int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * 256) {
@@ -694,7 +747,7 @@ __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__
     if (gid < 0) continue;
     const int64_t bh = wr / a.NW;
     const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
-    a.list[atomicAdd(a.off + u * a.Cmax * a.k + gid, 1)] = (int32_t)idx;
+    a.list[a.off[u * a.Cmax * a.k + gid] + a.pos[idx]] = (int32_t)idx;
   }
 }
 
@@ -1099,8 +1152,11 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
 
 // ================================================================== merge
 
-// One warp per row: the row state (m, l, acc) and the partials of the
-// row's opened groups in one softmax.
+// One warp per row: the row state (m, l, acc), minus the opened groups'
+// coarse terms, and the partials of those groups in one softmax.  Lane k
+// reads rank k's bookkeeping; every value slice is requested before any is
+// used, so the row's loads are in flight together.
+template <int GM>
 __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ PrefillArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)a.B * a.Hq * a.NW;
@@ -1109,54 +1165,74 @@ __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ P
   const int64_t bh = wr / a.NW, pi = a.w_lo + wr % a.NW;
   if (pi >= a.w_hi) return;
   const int64_t orow = bh * a.Tq + pi;
+  const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
   const float* stp = a.state + wr * kStateStride;
-  const float m = stp[0], l = stp[1];
-  // (a row whose scan gave up holds m = -inf and no accumulator)
+  const int G = a.G;
+  // rank `lane`: group, coarse weight, partial's log-sum-exp
+  const int gid_l = lane < G ? a.sel[wr * G + lane] : -1;
+  const float cw_l = lane < G ? a.cw[wr * G + lane] : 0.f;
+  const float pl_l = lane < G ? a.plse[wr * G + lane] : -INFINITY;
+  const float2 ml = *reinterpret_cast<const float2*>(stp);
+  const float m = ml.x;
   const float4 acc = m == -INFINITY ? make_float4(0.f, 0.f, 0.f, 0.f)
                                     : *reinterpret_cast<const float4*>(stp + 4 + 4 * lane);
+  uint2 gv[GM], po[GM];
+#pragma unroll
+  for (int k = 0; k < GM; ++k) {
+    const int gid = __shfl_sync(0xffffffffu, gid_l, k);
+    gv[k] = make_uint2(0u, 0u);
+    po[k] = make_uint2(0u, 0u);
+    if (k < G && gid >= 0) {
+      gv[k] = *reinterpret_cast<const uint2*>(a.gV + ((u * a.Cmax * a.k + gid) * D + 4 * lane));
+      po[k] = *reinterpret_cast<const uint2*>(a.po + (wr * G + k) * D + 4 * lane);
+    }
+  }
+  // the common max over the state and the partials
   float M = m;
-  for (int k = 0; k < a.G; ++k)
-    if (a.sel[wr * a.G + k] >= 0) M = fmaxf(M, a.plse[wr * a.G + k]);
+  {
+    const float pv = gid_l >= 0 ? pl_l : -INFINITY;
+    M = fmaxf(M, warp_max(pv));
+  }
   const float cs = m == -INFINITY ? 0.f : ex2_approx(m - M);
-  // the opened groups' coarse terms leave the row state (finer entries,
-  // the pairs' partials, replace them)
-  float L = l, o0 = acc.x, o1 = acc.y, o2 = acc.z, o3 = acc.w;
-  const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
-  for (int k = 0; k < a.G; ++k) {
-    const int gid = a.sel[wr * a.G + k];
-    if (gid < 0 || m == -INFINITY) continue;
-    const float wk = a.cw[wr * a.G + k];
-    const uint2 raw = *reinterpret_cast<const uint2*>(a.gV + ((u * a.Cmax * a.k + gid) * D + 4 * lane));
-    L -= wk;
-    o0 = fmaf(-wk, __uint_as_float(raw.x << 16), o0);
-    o1 = fmaf(-wk, __uint_as_float(raw.x & 0xffff0000u), o1);
-    o2 = fmaf(-wk, __uint_as_float(raw.y << 16), o2);
-    o3 = fmaf(-wk, __uint_as_float(raw.y & 0xffff0000u), o3);
+  float L = ml.y, o0 = acc.x, o1 = acc.y, o2 = acc.z, o3 = acc.w;
+#pragma unroll
+  for (int k = 0; k < GM; ++k) {  // the opened groups' coarse terms leave the state
+    const int gid = __shfl_sync(0xffffffffu, gid_l, k);
+    const float wk = __shfl_sync(0xffffffffu, cw_l, k);
+    if (k < G && gid >= 0 && m != -INFINITY) {
+      L -= wk;
+      o0 = fmaf(-wk, __uint_as_float(gv[k].x << 16), o0);
+      o1 = fmaf(-wk, __uint_as_float(gv[k].x & 0xffff0000u), o1);
+      o2 = fmaf(-wk, __uint_as_float(gv[k].y << 16), o2);
+      o3 = fmaf(-wk, __uint_as_float(gv[k].y & 0xffff0000u), o3);
+    }
   }
   L *= cs;
   o0 *= cs;
   o1 *= cs;
   o2 *= cs;
   o3 *= cs;
-  for (int k = 0; k < a.G; ++k) {
-    if (a.sel[wr * a.G + k] < 0) {
-      if (a.sel_pages && lane < a.TP) a.sel_pages[(orow * a.G + k) * a.TP + lane] = -1;
-      continue;
+#pragma unroll
+  for (int k = 0; k < GM; ++k) {  // the finer entries: the pairs' partials
+    const int gid = __shfl_sync(0xffffffffu, gid_l, k);
+    const float ls = __shfl_sync(0xffffffffu, pl_l, k);
+    if (k < G && gid >= 0 && ls != -INFINITY) {
+      const float w = ex2_approx(ls - M);
+      L += w;
+      o0 = fmaf(w, __uint_as_float(po[k].x << 16), o0);
+      o1 = fmaf(w, __uint_as_float(po[k].x & 0xffff0000u), o1);
+      o2 = fmaf(w, __uint_as_float(po[k].y << 16), o2);
+      o3 = fmaf(w, __uint_as_float(po[k].y & 0xffff0000u), o3);
     }
-    const float ls = a.plse[wr * a.G + k];
-    if (ls == -INFINITY) continue;
-    const float w = ex2_approx(ls - M);
-    L += w;
-    const uint2 raw = *reinterpret_cast<const uint2*>(a.po + (wr * a.G + k) * D + 4 * lane);
-    o0 = fmaf(w, __uint_as_float(raw.x << 16), o0);
-    o1 = fmaf(w, __uint_as_float(raw.x & 0xffff0000u), o1);
-    o2 = fmaf(w, __uint_as_float(raw.y << 16), o2);
-    o3 = fmaf(w, __uint_as_float(raw.y & 0xffff0000u), o3);
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   *reinterpret_cast<uint2*>(a.out + orow * D + 4 * lane) =
       make_uint2(pack_bf16x2(o0 * inv, o1 * inv), pack_bf16x2(o2 * inv, o3 * inv));
   if (lane == 0 && a.lse) a.lse[orow] = (M + log2f(L)) * 0.69314718055994531f;
+  // sel_pages of the ranks with no opened group (the pair kernel writes the others)
+  if (a.sel_pages)
+    for (int k = 0; k < G; ++k)
+      if (__shfl_sync(0xffffffffu, gid_l, k) < 0 && lane < a.TP) a.sel_pages[(orow * G + k) * a.TP + lane] = -1;
 }
 
 }  // namespace
@@ -1186,7 +1262,7 @@ cudaError_t launch_prefill_tc_wave(const PrefillArgs& a, const TcMaps& maps, con
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t npairs = (int64_t)a.B * a.Hq * a.NW * a.G;
-  const int64_t sblocks = (npairs + 255) / 256 < 4 * num_sms ? (npairs + 255) / 256 : 4 * num_sms;
+  const int64_t sblocks = (npairs + 255) / 256 < 64 * num_sms ? (npairs + 255) / 256 : 64 * num_sms;
   pf_scatter_kernel<<<(unsigned)(sblocks > 0 ? sblocks : 1), 256, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1200,7 +1276,10 @@ cudaError_t launch_prefill_tc_wave(const PrefillArgs& a, const TcMaps& maps, con
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)a.B * a.Hq * a.NW;
-  pf_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(a);
+  if (a.G <= 8)
+    pf_merge_kernel<8><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(a);
+  else
+    pf_merge_kernel<16><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
