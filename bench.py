@@ -471,14 +471,63 @@ def run_build(w, dev, stream, steps, peaks, k):
     flush = l2_flusher(dev)
     ts = time_steps(lambda i: api.lod_build_index(p, Kd, Vd, 0, nch, ix, stream=stream), steps, 2, flush, stream)
     ms = float(np.mean(ts))
-    by = metrics.build_bytes(p, nch)
+    by = metrics.build_bytes(p, nch)          # the method's own reads and writes
+    dby = metrics.build_design_bytes(p, nch)  # this design's member-ordered copies
     gbs = by / (ms * 1e-3) / 1e9
     fl = metrics.build_flops(p, nch)
+    alu = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # FP32 FMA lanes x 2 x clock
     return dict(workload="%s k=%d" % (w.name, k), value=gbs, unit="GB/s", ms_per_step=ms,
                 chunks_per_s=p.B * p.Hkv * nch / (ms * 1e-3),
                 roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
                               frac=gbs / peaks["hbm_gbs"], algorithmic_bytes=by,
-                              fp32_tflops=fl / (ms * 1e-3) / 1e12))
+                              design_bytes=dby,
+                              with_design_bytes=dict(achieved=(by + dby) / (ms * 1e-3) / 1e9,
+                                                     frac=(by + dby) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]),
+                              fp32_tflops=fl / (ms * 1e-3) / 1e12, fp32_alu_peak_tflops=alu,
+                              fp32_alu_frac=fl / (ms * 1e-3) / 1e12 / alu))
+
+
+def run_dense(dev, stream):
+    """Dense attention as the second reference (torch SDPA on the GPU): one
+    decode step at 32K (batch 8) and at 128K (batch 4), 64 query / 8 KV heads,
+    and the causal 128K prefill of 32 query / 8 KV heads, all bf16, d = 128."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    res = {}
+    backends = [SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]
+
+    def one(B, Hq, Hkv, T, Tq, causal, steps):
+        g = torch.Generator(device=dev).manual_seed(7)
+        q = torch.randn(B, Hq, Tq, 128, device=dev, dtype=torch.bfloat16, generator=g) / 8
+        k = torch.randn(B, Hkv, T, 128, device=dev, dtype=torch.bfloat16, generator=g)
+        v = torch.randn(B, Hkv, T, 128, device=dev, dtype=torch.bfloat16, generator=g)
+        # query heads share their KV head: expanded once, outside the timed region
+        k = k.repeat_interleave(Hq // Hkv, dim=1)
+        v = v.repeat_interleave(Hq // Hkv, dim=1)
+        with sdpa_kernel(backends):
+            fn = lambda i: F.scaled_dot_product_attention(q, k, v, is_causal=causal)
+            ms = time_region(fn, steps, 2, stream) / steps
+        del q, k, v
+        torch.cuda.empty_cache()
+        return ms
+
+    for name, args in (("decode_gqa_32k_bf16", (8, 64, 8, 32768, 1, False, 50)),
+                       ("decode_gqa_128k_bf16", (4, 64, 8, 131072, 1, False, 20)),
+                       ("prefill_128k_bf16", (1, 32, 8, 131072, 131072, True, 2))):
+        try:
+            ms = one(*args)
+            B, Hq, Hkv, T, Tq, causal, _ = args
+            entry = dict(ms_per_step=ms, B=B, Hq=Hq, Hkv=Hkv, seq_len=T, impl="torch SDPA (cuDNN/flash backends), "
+                         "KV heads expanded to the query heads outside the timed region")
+            if Tq == 1:
+                entry.update(value=B / (ms * 1e-3), unit="queries/s")
+            else:
+                fl = 4.0 * 128 * Hq * T * T / 2
+                entry.update(value=T * B / (ms * 1e-3), unit="tok/s", tflops=fl / (ms * 1e-3) / 1e12)
+            res[name] = entry
+        except Exception as ex:  # no memory-efficient backend for this shape here
+            res[name] = dict(unavailable=str(ex).splitlines()[0][:200])
+    return res
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -521,6 +570,77 @@ def oracle_decode_rate(w, budget_s=15.0):
     return n / dt, "%d decode steps of one sequence (all %d heads) at t=%d" % (n, w.Hq, w.T - 1), cores
 
 
+def oracle_index_all(w, cfg, nch, threads):
+    """The oracle's index of every KV head of sequence 0 (threads over heads),
+    and the time it took."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    K, V = synth_kv(w)
+    Kn = [K[0, h].float().numpy() for h in range(w.Hkv)]
+    Vn = [V[0, h].float().numpy() for h in range(w.Hkv)]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        idx = list(ex.map(lambda h: oracle.build_sequence(cfg, h, Kn[h], Vn[h], nch), range(w.Hkv)))
+    return idx, Kn, Vn, time.perf_counter() - t0
+
+
+def oracle_prefill_and_build(budget_rows=0):
+    """The oracle on the host cores for the prefill and the index build
+    (workloads prefill_128k_bf16 and build_128k_bf16).  Prefill: every row
+    (all 32 heads) of query chunks {1, 2, 3, 64, 256, 511}, timed; the time of
+    the whole 512-chunk prefill is extrapolated from them (a row's cost grows
+    linearly with its chunk's visible groups: least squares over the sampled
+    chunks).  Build: the whole 128K index of the 8 KV heads (threads over
+    heads), k = 4, timed.  Dense: the oracle's dense attention for 64 rows at
+    the last position, the second reference."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    from hierarchical_long_context_b200 import synth
+    cores = host_cores()
+    out = {}
+    wb = synth.WORKLOADS["build_128k_bf16"]
+    cfgb = oracle.Config(d=wb.d, clusters=4, iters=wb.iters, top_groups=wb.top_groups, top_pages=wb.top_pages,
+                         window=wb.window, sinks=wb.sinks, store_bf16=True, seed=wb.seed)
+    _, _, _, tb = oracle_index_all(wb, cfgb, wb.T // 256, cores)
+    out["build"] = dict(value=wb.Hkv * (wb.T // 256) / tb, unit="chunks/s", seconds=tb, cores=min(cores, wb.Hkv),
+                        kind="oracle", sample="the whole 128K index of 8 KV heads, k = 4 (threads over heads)")
+    w = synth.WORKLOADS["prefill_128k_bf16"]
+    cfg = oracle.Config(d=w.d, clusters=w.clusters[0], iters=w.iters, top_groups=w.top_groups,
+                        top_pages=w.top_pages, window=w.window, sinks=w.sinks, store_bf16=True, seed=w.seed)
+    nch = w.T // 256
+    idx, Kn, Vn, _ = oracle_index_all(w, cfg, nch, cores)
+    chunks = (1, 2, 3, 64, 256, 511)
+    per_chunk = {}
+    for c in chunks:
+        q = synth.prefill_queries(w, c * 256, 256)[0].float().numpy()  # [Hq, 256, d]
+        rows = [(hq, t) for hq in range(w.Hq) for t in range(256)]
+        t0 = time.perf_counter()
+        with ThreadPoolExecutor(cores) as ex:
+            list(ex.map(lambda rt: oracle.attend_row(cfg, q[rt[0], rt[1]], c * 256 + rt[1], Kn[rt[0] // w.g],
+                                                      Vn[rt[0] // w.g], idx[rt[0] // w.g]), rows))
+        per_chunk[c] = time.perf_counter() - t0
+    # least squares: time(c) = a + b * visible groups of chunk c
+    xs = np.array([max(0, c - w.window // 256 + 1) * cfg.clusters for c in chunks], dtype=np.float64)
+    ys = np.array([per_chunk[c] for c in chunks])
+    A = np.stack([np.ones_like(xs), xs], 1)
+    coef = np.linalg.lstsq(A, ys, rcond=None)[0]
+    allx = np.array([max(0, c - w.window // 256 + 1) * cfg.clusters for c in range(nch)], dtype=np.float64)
+    total = float(np.sum(np.maximum(coef[0] + coef[1] * allx, 0.0)))
+    out["prefill"] = dict(value=w.T / total, unit="tok/s", extrapolated=True, seconds_full_estimate=total,
+                          sampled_seconds={str(c): per_chunk[c] for c in chunks}, cores=cores, kind="oracle",
+                          sample="all rows (32 heads x 256 positions) of query chunks 1, 2, 3, 64, 256, 511; "
+                                 "the 512-chunk total is extrapolated (linear in visible groups)")
+    qd = synth.prefill_queries(w, w.T - 64, 64)[0].float().numpy()
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        list(ex.map(lambda j: oracle.dense_row(cfg, qd[j % w.Hq, j], w.T - 64 + j, Kn[(j % w.Hq) // w.g],
+                                               Vn[(j % w.Hq) // w.g]), range(64)))
+    td = time.perf_counter() - t0
+    out["dense_rows"] = dict(value=64 / td, unit="rows/s", cores=cores, kind="oracle dense attention",
+                             sample="64 rows at positions 131008-131071 (causal over the whole context)")
+    return out
+
+
 def run_reference(args, w):
     rate, sample, cores = oracle_decode_rate(w, budget_s=max(5.0, min(60.0, 3.0 * args.steps)))
     line = dict(impl="reference", metric="LoD decode queries/s (batch 4 x 64 heads at 128K context, one layer)",
@@ -554,6 +674,7 @@ def main():
                     help="with --leg: context length of the leg's workload (0 = its own)")
     ap.add_argument("--kv-bits", type=int, default=0, choices=[0, 4],
                     help="main decode leg in three-tier INT4 (opened pages from 4-bit codes)")
+    ap.add_argument("--clusters", type=int, default=4, help="with --leg build: clusters per chunk")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per step (0 = the workload's own; smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -577,7 +698,7 @@ def main():
         if args.seq_len:
             wl = wl.with_(T=args.seq_len)
         r = (run_prefill(wl, dev, torch.cuda.current_stream(), 2, peaks) if args.leg == "prefill" else
-             run_build(wl, dev, torch.cuda.current_stream(), 5, peaks, 4))
+             run_build(wl, dev, torch.cuda.current_stream(), 5, peaks, args.clusters))
         print(json.dumps(r), flush=True)
         return
     wg = w
@@ -601,13 +722,26 @@ def main():
             synth.WORKLOADS["decode_gqa_1m_bf16"], dev, stream, peaks, 500, 4,
             "decode_gqa_1m_bf16: one sequence at 1M context (device-generated inputs)", device_gen=True)
         torch.cuda.empty_cache()
+        extras["decode_32k"] = run_decode_variant(
+            synth.WORKLOADS["decode_gqa_32k_bf16"], dev, stream, peaks, 1000, 4,
+            "decode_gqa_32k_bf16: batch 8 at 32K context")
+        torch.cuda.empty_cache()
         wp = synth.WORKLOADS["prefill_128k_bf16"]
-        extras["prefill"] = run_prefill(wp, dev, stream, 2, peaks)
+        extras["prefill"] = run_prefill(wp, dev, stream, 3, peaks)
         wb = synth.WORKLOADS["build_128k_bf16"]
         extras["build"] = run_build(wb, dev, stream, 5, peaks, 4)
+        extras["build_k8"] = run_build(wb, dev, stream, 5, peaks, 8)
+        torch.cuda.empty_cache()
+        extras["dense_reference"] = run_dense(dev, stream)
+        for nm, leg in (("decode_gqa_32k_bf16", extras["decode_32k"]), ("decode_gqa_128k_bf16", res),
+                        ("prefill_128k_bf16", extras["prefill"])):
+            dref = extras["dense_reference"].get(nm, {})
+            if "ms_per_step" in dref:
+                dref["lod_speedup"] = dref["ms_per_step"] / leg["ms_per_step"]
         if rank == 0 and world == 1:
             rate, sample, cores = oracle_decode_rate(w)
             extras["cpu_baseline"] = dict(value=rate, unit="queries/s", cores=cores, kind="oracle", sample=sample)
+            extras["cpu_oracle"] = oracle_prefill_and_build()
     barrier(world)
     if rank == 0:
         line = dict(metric=res["metric"], value=res["value"], unit=res["unit"], n_gpus=world,

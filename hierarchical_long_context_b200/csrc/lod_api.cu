@@ -307,6 +307,26 @@ PfLayout pf_layout(const lod_params* p) {
 
 int g_num_sms[64] = {};
 
+// A second stream of the current device for work that overlaps the caller's
+// stream inside one call (created once per device, never destroyed; it only
+// ever waits on events of the caller's stream).
+cudaStream_t g_side[64] = {};
+std::mutex g_side_mu;
+
+int32_t side_stream(cudaStream_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LOD_EUNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  if (!g_side[dev]) {
+    e = cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+  }
+  *out = g_side[dev];
+  return LOD_OK;
+}
+
 int num_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
@@ -595,12 +615,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
                                    {sel_pages, "sel_pages"}});
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  // 1) index of every chunk completed inside the query range (a pure function of K/V)
   const int64_t c0 = q_begin / p->chunk, c1 = (q_begin + Tq) / p->chunk;
-  if (c1 > c0) {
-    rc = do_build(p, K, V, kv_strides, c0, c1, index, ws, st);
-    if (rc) return rc;
-  }
   if (use_tc_prefill(p) && !q_host) {
     // 2) grouped tensor-core attention, one wave of query chunks at a time
     const PfLayout L = pf_layout(p);
@@ -653,14 +668,70 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.sel_pages = sel_pages;
     a.status = reinterpret_cast<uint32_t*>(w);
     const int nsm = num_sms();
-    for (int64_t lo = 0; lo < Tq; lo += L.NW) {
+    // The index of the chunks a wave completes is built before the wave
+    // attends; the next wave's chunks are built on a second stream while
+    // this wave attends.  Its queries see a chunk only window/chunk chunks
+    // after it completes, so no wave reads a chunk that is being built.
+    auto wave_chunks = [&](int64_t lo, int64_t hi, int64_t& b0, int64_t& b1) {
+      b0 = (q_begin + lo) / p->chunk;
+      b1 = (q_begin + hi) / p->chunk;
+    };
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+    if (Tq > L.NW) {
+      rc = side_stream(&side);
+      if (!rc && cudaEventCreateWithFlags(&ev[0], cudaEventDisableTiming) != cudaSuccess) rc = fail(LOD_ECUDA, "event");
+      if (!rc && cudaEventCreateWithFlags(&ev[1], cudaEventDisableTiming) != cudaSuccess) rc = fail(LOD_ECUDA, "event");
+      if (rc) {
+        if (ev[0]) cudaEventDestroy(ev[0]);
+        return rc;
+      }
+    }
+    auto done = [&](int32_t code) {
+      for (cudaEvent_t e : ev)
+        if (e) cudaEventDestroy(e);  // (released once their work has completed)
+      return code;
+    };
+    int64_t b0, b1;
+    wave_chunks(0, L.NW < Tq ? L.NW : Tq, b0, b1);
+    if (b1 > b0) {
+      rc = do_build(p, K, V, kv_strides, b0, b1, index, ws, st);
+      if (rc) return done(rc);
+    }
+    int k = 0;
+    for (int64_t lo = 0; lo < Tq; lo += L.NW, k ^= 1) {
       a.w_lo = lo;
       a.w_hi = lo + L.NW < Tq ? lo + L.NW : Tq;
+      const int64_t nlo = a.w_hi, nhi = nlo + L.NW < Tq ? nlo + L.NW : Tq;
+      bool built_next = false;
+      if (nlo < Tq) {  // the next wave's chunks, on the second stream
+        wave_chunks(nlo, nhi, b0, b1);
+        if (b1 > b0) {
+          cudaError_t e = cudaEventRecord(ev[k], st);
+          if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev[k], 0);
+          if (e != cudaSuccess) return done(cuda_fail(e, "prefill stream fork"));
+          rc = do_build(p, K, V, kv_strides, b0, b1, index, ws, side);
+          if (rc) return done(rc);
+          e = cudaEventRecord(ev[k], side);
+          if (e != cudaSuccess) return done(cuda_fail(e, "prefill stream join"));
+          built_next = true;
+        }
+      }
       cudaError_t e = lod::launch_prefill_tc_wave(a, maps, pmaps, nsm, st);
-      if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+      if (e != cudaSuccess) return done(cuda_fail(e, "prefill launch"));
+      if (built_next) {
+        e = cudaStreamWaitEvent(st, ev[k], 0);
+        if (e != cudaSuccess) return done(cuda_fail(e, "prefill stream join"));
+      }
     }
     g_err[0] = 0;
-    return LOD_OK;
+    return done(LOD_OK);
+  }
+  // per-chunk path: 1) the index of every chunk completed inside the query
+  // range (a pure function of K/V), 2) attention per query chunk
+  if (c1 > c0) {
+    rc = do_build(p, K, V, kv_strides, c0, c1, index, ws, st);
+    if (rc) return rc;
   }
   // 2) attention, one launch pair per query chunk
   lod::AttendArgs a;

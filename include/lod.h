@@ -278,6 +278,13 @@ int32_t lod_decode(const lod_params* p, const void* q, const void* K, const void
  *   sel_pages  device [B][Hq][Tq][top_groups][top_pages] int32 (nullable)
  *   index      its chunks [q_begin/chunk, (q_begin+Tq)/chunk) are written
  *   ws         device workspace of at least lod_workspace_bytes(LOD_OP_PREFILL)
+ * With bf16 caches and d = 128 (and q in device memory) the rows are
+ * processed in waves of query chunks, and the rows that opened the same
+ * group share tensor-core tiles (the grouped prefill); the index of the
+ * next wave's chunks is built on a second stream of the library (created
+ * once per device) while a wave attends, and that stream is joined back to
+ * `stream` before the call's work ends.  Other configurations build the
+ * whole range first and then attend per query chunk.
  */
 int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t Tq,
                     const void* K, const void* V, const int64_t kv_strides[3],

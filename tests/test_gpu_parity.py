@@ -475,11 +475,12 @@ def test_grouped_prefill_sweep(kw, T):
 
 
 def test_grouped_prefill_several_waves_match_one_call_per_chunk():
-    """A prefill longer than one wave of query chunks (64 chunks) equals the
-    same queries prefilled one chunk per call: the wave boundaries and the
-    pair bookkeeping leave every row's result unchanged, bit for bit."""
+    """A prefill longer than one wave of query chunks (at most 128 chunks)
+    equals the same queries prefilled one chunk per call: the wave boundaries,
+    the next wave's index built on a second stream while a wave attends, and
+    the pair bookkeeping leave every row's result unchanged, bit for bit."""
     w = synth.WORKLOADS["prefill_128k_bf16"].with_(B=1, Hkv=1, Hq=4)
-    T = 64 * 256 + 700
+    T = 2 * 128 * 256 + 700
     p, Kc, Vc, Kd, Vd = _setup(w, None, T)
     dev = Kd.device
     q = synth.prefill_queries(w, 0, T).to(dev)
