@@ -248,6 +248,7 @@ int32_t make_tc_maps(const lod_params* p, const void* K, const void* V, const in
 bool use_tc_prefill(const lod_params* p) {
   const int64_t Cmax = p->Tmax / p->chunk;
   return use_tc(p) && p->kv_bits == 0 && (int64_t)p->B * p->Hkv * p->Tmax < ((int64_t)1 << 31) &&
+         (int64_t)p->B * p->Hq * p->Tmax < ((int64_t)1 << 31) &&
          (int64_t)p->B * p->Hkv * Cmax * page_slots(p) < ((int64_t)1 << 31);
 }
 
@@ -256,8 +257,8 @@ constexpr int64_t kPrefillWaveBudget = (int64_t)2 << 30;  // workspace bytes a w
 
 // Workspace bytes per wave row: state (132 floats), and per opened group
 // its id, its coarse weight, its place in the group's run, its log-sum-exp,
-// its bf16 output and its pair-list entry.
-int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 4 + 2 * p->d + 4); }
+// its bf16 output and its two pair-list entries (pair id, row of q).
+int64_t pf_row_bytes(const lod_params* p) { return 132 * 4 + (int64_t)p->top_groups * (4 + 4 + 4 + 4 + 2 * p->d + 4 + 4); }
 
 // Query positions per wave: a multiple of chunk, as many as the budget allows
 // (at least one chunk, at most 128), never more than the cache holds.
@@ -273,7 +274,7 @@ int64_t pf_wave(const lod_params* p) {
 }
 
 struct PfLayout {
-  size_t state, sel, cw, pos, plse, po, list, cnt, off, items, n_items, total;
+  size_t state, sel, cw, pos, plse, po, list, list_q, cnt, off, items, n_items, total;
   int64_t NW, Gtot, max_items;
 };
 
@@ -297,6 +298,7 @@ PfLayout pf_layout(const lod_params* p) {
   L.plse = take(sizeof(float) * (size_t)pairs);
   L.po = take((size_t)2 * p->d * (size_t)pairs);
   L.list = take(sizeof(int32_t) * (size_t)pairs);
+  L.list_q = take(sizeof(int32_t) * (size_t)pairs);
   L.cnt = take(sizeof(int32_t) * (size_t)L.Gtot);
   L.off = take(sizeof(int32_t) * (size_t)L.Gtot);
   L.items = take(16 * 2 * (size_t)L.max_items);  // small-group items, then large-group items
@@ -655,6 +657,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.plse = reinterpret_cast<float*>(w + L.plse);
     a.po = reinterpret_cast<__nv_bfloat16*>(w + L.po);
     a.list = reinterpret_cast<int32_t*>(w + L.list);
+    a.list_q = reinterpret_cast<int32_t*>(w + L.list_q);
     a.cnt = reinterpret_cast<int32_t*>(w + L.cnt);
     a.off = reinterpret_cast<int32_t*>(w + L.off);
     a.items = reinterpret_cast<int4*>(w + L.items);

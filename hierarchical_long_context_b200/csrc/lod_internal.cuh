@@ -168,6 +168,7 @@ struct PrefillArgs {
   float* plse;              // [rows][G] pair log-sum-exp (log2 units)
   __nv_bfloat16* po;        // [rows][G][d] pair output (normalised)
   int32_t* list;            // pair ids (row * G + rank) grouped by (unit, group)
+  int32_t* list_q;          // beside each: the pair's row of q / out ((b * Hq + hq) * Tq + position)
   int32_t* cnt;             // [Gtot] pairs per (unit, group)
   int32_t* off;             // [Gtot] first pair of each (unit, group)
   int4* items;              // work items {unit * Cmax * k + group, first pair, pairs, 0}: small groups

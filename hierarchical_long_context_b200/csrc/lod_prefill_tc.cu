@@ -738,16 +738,20 @@ __global__ void __launch_bounds__(kPlanThreads) pf_plan_kernel(const __grid_cons
 // place its counting atomic returned (the order inside a run is arbitrary:
 // every pair is computed on its own).
 __global__ void __launch_bounds__(256) pf_scatter_kernel(const __grid_constant__ PrefillArgs a) {
-  const int64_t n = (int64_t)a.B * a.Hq * a.NW * a.G;
-  for (int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * 256) {
-    const int64_t wr = idx / a.G;
-    const int64_t pr = wr % a.NW;
-    if (a.w_lo + pr >= a.w_hi) continue;
+  // (32-bit index arithmetic: the wave's pairs number fewer than 2^31)
+  const int n = a.B * a.Hq * (int)a.NW * a.G;
+  const int NW = (int)a.NW;
+  for (int idx = blockIdx.x * 256 + threadIdx.x; idx < n; idx += gridDim.x * 256) {
     const int gid = a.sel[idx];
     if (gid < 0) continue;
-    const int64_t bh = wr / a.NW;
-    const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
-    a.list[a.off[u * a.Cmax * a.k + gid] + a.pos[idx]] = (int32_t)idx;
+    const int wr = idx / a.G;
+    const int bh = wr / NW;
+    const int pr = wr - bh * NW;
+    if (a.w_lo + pr >= a.w_hi) continue;
+    const int64_t u = (int64_t)(bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
+    const int64_t at = a.off[u * a.Cmax * a.k + gid] + a.pos[idx];
+    a.list[at] = (int32_t)idx;
+    a.list_q[at] = (int32_t)(bh * a.Tq + a.w_lo + pr);  // the pair's row of q / out
   }
 }
 
@@ -944,23 +948,19 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
       const int r = 32 * q4 + lane;
       const uint32_t tl = (uint32_t)(32 * q4) << 16;
       // the query row of pair t * 128 + r, staged by this thread
-      auto gather = [&](int t, int64_t& pid) {
+      auto gather = [&](int t, int& pid, int& qrow) {
         const int idx = t * kRows + r;
         const bool v = idx < f.count;
         pid = v ? a.list[f.start + idx] : -1;
-        const __nv_bfloat16* src = a.q;
-        if (v) {
-          const int64_t wr = pid / G;
-          const int64_t bh = wr / a.NW, pi = a.w_lo + wr % a.NW;
-          src = a.q + (bh * a.Tq + pi) * D;
-        }
+        qrow = v ? a.list_q[f.start + idx] : 0;
+        const __nv_bfloat16* src = a.q + (int64_t)qrow * D;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           cp_async16_zfill(Qs + (c >> 3) * kHalf + sw_off(r, c), reinterpret_cast<const uint4*>(src) + c, v);
         cp_async_mbar_arrive_noinc(q_full);
       };
-      int64_t pid_cur = -1, pid_next = -1;
-      gather(0, pid_cur);
+      int pid_cur = -1, pid_next = -1, qr_cur = 0, qr_next = 0;
+      gather(0, pid_cur, qr_cur);
       // page counts of the group (log2, for the coarse logits)
       if (r < 16) {
         float v = -INFINITY;
@@ -993,7 +993,7 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
         alive = __all_sync(0xffffffffu, mbar_wait(s_full, Tt & 1u, a.status));
         if (!alive) break;
         tc::fence_after_sync();
-        if (t + 1 < ntiles && !f.shared_qp) gather(t + 1, pid_next);
+        if (t + 1 < ntiles && !f.shared_qp) gather(t + 1, pid_next, qr_next);
         // page scores and this row's top-TP pages (score desc, slot asc)
         float sp[16];
         tc::tmem_ld16(tmem + tl + Cfg::kColSp, sp);
@@ -1102,7 +1102,7 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
             if (lane == 0) mbar_arrive(o_free);
           }
           if (vp) {
-            uint4* dst = reinterpret_cast<uint4*>(a.po + pid_cur * D + 64 * hh);
+            uint4* dst = reinterpret_cast<uint4*>(a.po + (int64_t)pid_cur * D + 64 * hh);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               dst[q] = make_uint4(pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv),
@@ -1111,14 +1111,12 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
                                   pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv));
           }
         }
-        if (t + 1 < ntiles && f.shared_qp) gather(t + 1, pid_next);
+        if (t + 1 < ntiles && f.shared_qp) gather(t + 1, pid_next, qr_next);
         if (pid_cur >= 0) {
           a.plse[pid_cur] = vp && l > 0.f ? m + log2f(l) : -INFINITY;
           if (a.sel_pages) {
-            const int64_t wr = pid_cur / G;
-            const int rank = (int)(pid_cur % G);
-            const int64_t bh = wr / a.NW, pi = a.w_lo + wr % a.NW;
-            int32_t* spo = a.sel_pages + ((bh * a.Tq + pi) * G + rank) * TP;
+            const int rank = pid_cur - (pid_cur / G) * G;
+            int32_t* spo = a.sel_pages + ((int64_t)qr_cur * G + rank) * TP;
             // the opened pages, best first (score desc, slot asc)
             uint32_t rest = vp ? selm : 0u;
             for (int x = 0; x < TP; ++x) {
@@ -1136,6 +1134,7 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
           }
         }
         pid_cur = pid_next;
+        qr_cur = qr_next;
       }
       // (a gathered tile that was never consumed: let its copies land)
       cp_async_wait_all();
@@ -1159,14 +1158,17 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
 template <int GM>
 __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ PrefillArgs a) {
   const int lane = threadIdx.x & 31;
-  const int64_t nrows = (int64_t)a.B * a.Hq * a.NW;
-  const int64_t wr = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  // (32-bit index arithmetic: the wave's rows number fewer than 2^31)
+  const int NW = (int)a.NW;
+  const int nrows = a.B * a.Hq * NW;
+  const int wr = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (wr >= nrows) return;
-  const int64_t bh = wr / a.NW, pi = a.w_lo + wr % a.NW;
+  const int bh = wr / NW;
+  const int64_t pi = a.w_lo + (wr - bh * NW);
   if (pi >= a.w_hi) return;
-  const int64_t orow = bh * a.Tq + pi;
-  const int64_t u = (bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
-  const float* stp = a.state + wr * kStateStride;
+  const int64_t orow = (int64_t)bh * a.Tq + pi;
+  const int64_t u = (int64_t)(bh / a.Hq) * a.Hkv + (bh % a.Hq) / a.g;
+  const float* stp = a.state + (int64_t)wr * kStateStride;
   const int G = a.G;
   // rank `lane`: group, coarse weight, partial's log-sum-exp
   const int gid_l = lane < G ? a.sel[wr * G + lane] : -1;
@@ -1184,7 +1186,7 @@ __global__ void __launch_bounds__(256) pf_merge_kernel(const __grid_constant__ P
     po[k] = make_uint2(0u, 0u);
     if (k < G && gid >= 0) {
       gv[k] = *reinterpret_cast<const uint2*>(a.gV + ((u * a.Cmax * a.k + gid) * D + 4 * lane));
-      po[k] = *reinterpret_cast<const uint2*>(a.po + (wr * G + k) * D + 4 * lane);
+      po[k] = *reinterpret_cast<const uint2*>(a.po + (int64_t)(wr * G + k) * D + 4 * lane);
     }
   }
   // the common max over the state and the partials
