@@ -114,35 +114,38 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- helpers
 
-def csrc_hash() -> str:
-    """SHA-256 over the library's CUDA sources (file names and contents)."""
+def csrc_hash(files=None) -> str:
+    """SHA-256 over the library's CUDA sources (file names and contents): all
+    of them, or the listed ones."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "hierarchical_long_context_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+    names = sorted(files) if files else sorted(f for f in os.listdir(d) if f.endswith((".cu", ".cuh")))
+    for f in names:
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()
 
 
 def profiled_traffic(kind: str, workload: str):
     """DRAM bytes (read + write) per launch from the committed ncu summary
     profiles/<kind>_<workload>.md, or None when that summary is missing or was
-    captured from CUDA sources other than the current ones."""
+    captured from CUDA sources other than the current ones (the summary's
+    `csrc_files:` line names the sources its kernels are built from)."""
     path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kind, workload))
     if not os.path.exists(path):
         return None
     vals = {}
     with open(path) as fh:
         for line in fh:
-            for key in ("traffic_bytes_per_launch:", "csrc_sha256:"):
+            for key in ("traffic_bytes_per_launch:", "csrc_sha256:", "csrc_files:"):
                 if line.strip().startswith(key):
-                    vals[key] = line.strip()[len(key):].strip().split()[0]
-    if vals.get("csrc_sha256:") != csrc_hash() or "traffic_bytes_per_launch:" not in vals:
+                    vals[key] = line.strip()[len(key):].strip()
+    files = vals.get("csrc_files:", "").split() or None
+    if vals.get("csrc_sha256:", "").split()[:1] != [csrc_hash(files)] or "traffic_bytes_per_launch:" not in vals:
         return None
-    return int(vals["traffic_bytes_per_launch:"])
+    return int(vals["traffic_bytes_per_launch:"].split()[0])
 
 
 def l2_flusher(dev):

@@ -835,14 +835,25 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
   uint32_t T = 0;      // tiles processed by this CTA (barrier phases)
   uint32_t ngrp = 0;   // items processed (gfull phases)
   bool alive = true;
+  // (thread 0 reads each item and its group word one item ahead)
+  int4 nx_item = make_int4(0, 0, 0, 0);
+  int nx_meta = 0;
+  if (tid == 0 && (int)blockIdx.x < n_items) {
+    nx_item = items[blockIdx.x];
+    nx_meta = a.gMeta[nx_item.x];
+  }
 
   for (int it = blockIdx.x; it < n_items && alive; it += gridDim.x) {
     // ---- the item: its group, bounds-checked, and the operand layout
     if (tid == 0) {
-      const int4 item = items[it];
+      const int4 item = nx_item;
+      const int meta = nx_meta;
+      if (it + (int)gridDim.x < n_items) {
+        nx_item = items[it + gridDim.x];
+        nx_meta = a.gMeta[nx_item.x];
+      }
       const int64_t gflat = item.x;
       const int64_t u = gflat / Gcap, gid = gflat % Gcap, c = gid / a.k;
-      const int meta = a.gMeta[gflat];
       const int n = meta & 0xffff, p0 = (meta >> 16) & 0xff, p1 = (meta >> 24) & 0xff;
       const int64_t pslot = (u * a.Cmax + c) * a.P;
       bool ok = n >= 1 && n <= (BIG ? kChunk : kSmallN) && p0 < p1 && p1 <= a.P && p1 - p0 == (n + kPage - 1) / kPage;
@@ -948,11 +959,15 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
       const int r = 32 * q4 + lane;
       const uint32_t tl = (uint32_t)(32 * q4) << 16;
       // the query row of pair t * 128 + r, staged by this thread
-      auto gather = [&](int t, int& pid, int& qrow) {
+      // the pair list entries of tile t (read one tile ahead of its gather)
+      auto entries = [&](int t, int& pid, int& qrow) {
         const int idx = t * kRows + r;
         const bool v = idx < f.count;
         pid = v ? a.list[f.start + idx] : -1;
         qrow = v ? a.list_q[f.start + idx] : 0;
+      };
+      auto gather = [&](int t, int pid, int qrow) {
+        const bool v = pid >= 0;
         const __nv_bfloat16* src = a.q + (int64_t)qrow * D;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
@@ -960,6 +975,7 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
         cp_async_mbar_arrive_noinc(q_full);
       };
       int pid_cur = -1, pid_next = -1, qr_cur = 0, qr_next = 0;
+      entries(0, pid_cur, qr_cur);
       gather(0, pid_cur, qr_cur);
       // page counts of the group (log2, for the coarse logits)
       if (r < 16) {
@@ -993,6 +1009,7 @@ __global__ void __launch_bounds__(kThreadsB, BIG ? 1 : 2)
         alive = __all_sync(0xffffffffu, mbar_wait(s_full, Tt & 1u, a.status));
         if (!alive) break;
         tc::fence_after_sync();
+        if (t + 1 < ntiles) entries(t + 1, pid_next, qr_next);
         if (t + 1 < ntiles && !f.shared_qp) gather(t + 1, pid_next, qr_next);
         // page scores and this row's top-TP pages (score desc, slot asc)
         float sp[16];

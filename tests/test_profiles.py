@@ -25,10 +25,11 @@ def test_decode_traffic_is_reported_only_for_the_current_sources():
         text = open(path).read()
         rec = re.search(r"csrc_sha256:\s*(\w+)", text)
         val = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
-        assert rec and val, path
+        files = re.search(r"csrc_files:\s*(.+)", text)
+        assert rec and val and files, path
         assert 10_000_000 < int(val.group(1)) < 1_000_000_000
         t = bench.profiled_traffic(kind, "decode_gqa_128k_bf16")
-        if rec.group(1) == bench.csrc_hash():
+        if rec.group(1) == bench.csrc_hash(files.group(1).split()):
             assert t == int(val.group(1))
         else:
             assert t is None
