@@ -16,9 +16,9 @@
 //                      and the causal block window (keys on N), one online
 //                      softmax per row (group logits carry + ln count), and
 //                      O += P V on the tensor cores; each row's top-G groups
-//                      are kept in its thread's registers.  The epilogue
-//                      removes the top-G groups' coarse terms (finer entries
-//                      replace them in B), stores the row state, and counts
+//                      are kept in registers by two selection warpgroups.
+//                      The epilogue stores the row state, the top-G groups
+//                      with the weights of their coarse terms, and counts
 //                      the (row, group) pairs of every group.
 //  plan, scatter       counting sort of the pairs by (KV head, group) and
 //                      the work items (one group's pairs, up to kItemRows).
@@ -31,8 +31,10 @@
 //                      as coarse entries (page mean value, logit + ln count)
 //                      in one MMA chain.  The pair's normalised partial
 //                      (log-sum-exp, bf16 output) is stored.
-//  merge               per row: the row state and its pairs' partials in one
-//                      softmax; out and lse.
+//  merge               per row: the opened groups' coarse terms leave the
+//                      row state (finer entries replace them in B), then the
+//                      state and its pairs' partials form one softmax; out
+//                      and lse.
 //
 // Softmax arithmetic is in log2 units (logit * log2 e) with ex2 on the SFU.
 // Removing the opened groups' coarse terms after the fact is numerically
