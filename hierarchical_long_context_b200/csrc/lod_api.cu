@@ -354,10 +354,14 @@ int32_t make_pair_maps(const lod_params* p, const lod_index* ix, lod::PairMaps* 
   return rc;
 }
 
+// Workspace of a scan/refine pair: the split states, then either every
+// group's score per query row (CUDA-core scan) or each split's best groups
+// per query row (tensor-core scan).
 size_t attend_ws_bytes(const lod_params* p, const AttendShape& s) {
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
-  size_t gsc = sizeof(float2) * (size_t)s.units * s.NQ * (size_t)(p->Tmax / p->chunk) * p->clusters;
-  return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((gsc + 255) & ~size_t(255));
+  size_t sel = s.tc ? sizeof(lod::SplitCand) * (size_t)s.units * s.nsplit * s.NQ * p->top_groups
+                    : sizeof(float2) * (size_t)s.units * s.NQ * (size_t)(p->Tmax / p->chunk) * p->clusters;
+  return lod::kWsHeader + ((part + 255) & ~size_t(255)) + ((sel + 255) & ~size_t(255));
 }
 
 void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, const void* K,
@@ -406,7 +410,10 @@ void fill_attend(lod::AttendArgs& a, const lod_params* p, const AttendShape& s, 
   size_t part = sizeof(float) * (size_t)s.units * s.nsplit * s.NQ * (p->d + 2);
   part = (part + 255) & ~size_t(255);
   a.part = reinterpret_cast<float*>(w + lod::kWsHeader);
-  a.gsc = reinterpret_cast<float2*>(w + lod::kWsHeader + part);
+  if (s.tc)
+    a.cand = reinterpret_cast<lod::SplitCand*>(w + lod::kWsHeader + part);
+  else
+    a.gsc = reinterpret_cast<float2*>(w + lod::kWsHeader + part);
 }
 
 int32_t do_build(const lod_params* p, const void* K, const void* V, const int64_t* kv, int64_t c0,
@@ -763,7 +770,7 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
     a.units = (int64_t)p->B * p->Hkv * cdiv(hi - lo, s.NP);
     const int want = split_for(p, s.tc, a.units, wb * p->clusters + p->window);
     a.nsplit = want < s.nsplit ? want : s.nsplit;
-    // part/gsc keep the worst-case layout of fill_attend; a chunk uses a prefix
+    // part/cand/gsc keep the worst-case layout of fill_attend; a chunk uses a prefix
     cudaError_t e = lod::launch_attend(a, p->dtype, p->d, s.NQ, s.tc ? &maps : nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   }

@@ -28,6 +28,8 @@
 // method's "conservative estimate" property: n exp(q.mean k) <= sum exp(q.k)),
 // so the final normaliser is never smaller than what was subtracted and the
 // cancellation error stays at the fp32 rounding level of the output.
+#include <type_traits>
+
 #include "lod_internal.cuh"
 
 namespace lod {
@@ -201,6 +203,7 @@ __device__ __forceinline__ UnitInfo unit_info(const AttendArgs& a, int64_t u) {
 struct Cand {
   float s;     // scale * q.mean_k
   int id;      // group id within the unit (chunk * k + slot), -1 = none
+  int meta;    // the group's gMeta word
 };
 
 // ------------------------------------------------------------------ scan
@@ -659,28 +662,6 @@ __device__ __forceinline__ void rows_dot_coalesced(int n, RowPtr rowptr, const f
   }
 }
 
-// Orderable 64-bit key of group `id` with score s: a larger key is a better
-// group (higher score, then smaller id; the same order as comparing the
-// floats); 0 = no group (score -inf).
-__device__ __forceinline__ uint64_t group_key(float s, int64_t id) {
-  if (s == -INFINITY) return 0;
-  uint32_t b = s == 0.f ? 0u : __float_as_uint(s);  // -0 orders as +0
-  b ^= (b & 0x80000000u) ? 0xffffffffu : 0x80000000u;
-  return ((uint64_t)b << 32) | (uint32_t)(0xffffffffu - (uint32_t)id);
-}
-// Orderable 32-bit key of a score (larger = better; -0 as +0); 0 = -inf.
-__device__ __forceinline__ uint32_t okey32(float s) {
-  if (s == -INFINITY) return 0u;
-  const uint32_t b = s == 0.f ? 0u : __float_as_uint(s);
-  return b ^ ((b & 0x80000000u) ? 0xffffffffu : 0x80000000u);
-}
-__device__ __forceinline__ float key_score(uint64_t k) {
-  uint32_t b = (uint32_t)(k >> 32);
-  b = (b & 0x80000000u) ? (b ^ 0x80000000u) : ~b;
-  return __uint_as_float(b);
-}
-__device__ __forceinline__ int key_id(uint64_t k) { return (int)(0xffffffffu - (uint32_t)k); }
-
 // Largest key over the CTA (every thread receives it); red: [kWarps] scratch.
 __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -699,7 +680,9 @@ __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* red) {
 }
 
 // Q4: three-tier INT4 (opened pages read from 4-bit codes; a.kv_bits == 4).
-template <typename T, int D, int NQ, bool Q4>
+// SC: the groups come from the splits' best lists (a.cand, tensor-core scan)
+// rather than from every group's score (a.gsc).
+template <typename T, int D, int NQ, bool Q4, bool SC>
 __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
   constexpr int DPL = D / 32;
   constexpr int EPL = 16 / sizeof(T);
@@ -794,12 +777,36 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
       pre_v[sp] = ps[sp * pstride + tid];
     }
   }
-  // ---- the top-G groups of this row from the unit's score array (higher
-  // score first, then smaller id).  A bound that G distinct groups reach (the
+  // ---- the top-G groups of this row (higher score first, then smaller id)
+  if constexpr (SC) {
+    // from the splits' own best G: every candidate's exact rank among them
+    const SplitCand* cr = a.cand + (u * nsplit * NQ + r) * (int64_t)a.G;
+    const int nall = nsplit * a.G;
+    int* cmeta = reinterpret_cast<int*>(surv + nall);
+    if (tid == 0) *nwin_s = 0;
+    for (int x = tid; x < nall; x += kThreads) {
+      const SplitCand c = cr[(int64_t)(x / a.G) * NQ * a.G + x % a.G];
+      surv[x] = c.id >= 0 ? group_key(c.s, c.id) : 0ull;
+      cmeta[x] = c.meta;
+    }
+    __syncthreads();
+    for (int x = tid; x < nall; x += kThreads) {
+      const uint64_t kx = surv[x];
+      if (kx == 0ull) continue;
+      int rx = 0;
+      for (int y = 0; y < nall; ++y) rx += surv[y] > kx ? 1 : 0;
+      if (rx < a.G) {
+        win[rx].s = key_score(kx);
+        win[rx].id = key_id(kx);
+        win[rx].meta = cmeta[x];
+        atomicMax(nwin_s, rx + 1);
+      }
+    }
+  } else {
+  // From the unit's score array: a bound that G distinct groups reach (the
   // G-th largest of a warp's per-thread best scores; the largest such bound
   // over the warps), the groups scoring at or above it (a few dozen), then
   // their exact ranks by (score, id).
-  {
     const int64_t wbq = t / kChunk - a.window / kChunk + 1;
     const int Gq = wbq > 0 ? (int)(wbq * a.k) : 0;  // visible groups of this row
     const float2* srow = a.gsc + (u * NQ + r) * (a.Cmax * a.k);
@@ -1223,7 +1230,11 @@ __global__ void __launch_bounds__(kThreads, 2) refine_kernel(AttendArgs a) {
     const int gid = win[w].id;
     const int64_t c = gid / a.k;
     // size and page range: the gMeta word the scan stored beside the score
-    const int meta = __float_as_int(a.gsc[(u * NQ + r) * (a.Cmax * a.k) + gid].y);
+    int meta;
+    if constexpr (SC)
+      meta = win[w].meta;
+    else
+      meta = __float_as_int(a.gsc[(u * NQ + r) * (a.Cmax * a.k) + gid].y);
     const int gcnt = meta & 0xffff;
     const int p0 = (meta >> 16) & 0xff, p1 = (meta >> 24) & 0xff;
     // one round trip: the group's mean value, its pages' member counts and
@@ -1435,9 +1446,21 @@ cudaError_t launch_t(const AttendArgs& a, const TcMaps* maps, cudaStream_t strea
   }
   if (rows > 0) {
     const bool q4 = a.kv_bits == 4;
-    auto rk = q4 ? refine_kernel<T, D, NQ, true> : refine_kernel<T, D, NQ, false>;
     const size_t smem = RefineSmem<T, D>::bytes;
-    e = q4 ? set_smem_once<refine_kernel<T, D, NQ, true>>(smem) : set_smem_once<refine_kernel<T, D, NQ, false>>(smem);
+    void (*rk)(AttendArgs) = nullptr;
+    if (a.cand) {  // tensor-core scan: bf16, d = 128
+      if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+        rk = q4 ? refine_kernel<T, D, NQ, true, true> : refine_kernel<T, D, NQ, false, true>;
+        e = q4 ? set_smem_once<refine_kernel<T, D, NQ, true, true>>(smem)
+               : set_smem_once<refine_kernel<T, D, NQ, false, true>>(smem);
+      } else {
+        return cudaErrorInvalidValue;
+      }
+    } else {
+      rk = q4 ? refine_kernel<T, D, NQ, true, false> : refine_kernel<T, D, NQ, false, false>;
+      e = q4 ? set_smem_once<refine_kernel<T, D, NQ, true, false>>(smem)
+             : set_smem_once<refine_kernel<T, D, NQ, false, false>>(smem);
+    }
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows);

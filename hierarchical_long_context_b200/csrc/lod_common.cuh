@@ -285,4 +285,26 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   return z ^ (z >> 31);
 }
 
+// Orderable 64-bit key of group `id` with score s: a larger key is a better
+// group (higher score, then smaller id; the same order as comparing the
+// floats); 0 = no group (score -inf).
+__device__ __forceinline__ uint64_t group_key(float s, int64_t id) {
+  if (s == -INFINITY) return 0;
+  uint32_t b = s == 0.f ? 0u : __float_as_uint(s);  // -0 orders as +0
+  b ^= (b & 0x80000000u) ? 0xffffffffu : 0x80000000u;
+  return ((uint64_t)b << 32) | (uint32_t)(0xffffffffu - (uint32_t)id);
+}
+// Orderable 32-bit key of a score (larger = better; -0 as +0); 0 = -inf.
+__device__ __forceinline__ uint32_t okey32(float s) {
+  if (s == -INFINITY) return 0u;
+  const uint32_t b = s == 0.f ? 0u : __float_as_uint(s);
+  return b ^ ((b & 0x80000000u) ? 0xffffffffu : 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint64_t k) {
+  uint32_t b = (uint32_t)(k >> 32);
+  b = (b & 0x80000000u) ? (b ^ 0x80000000u) : ~b;
+  return __uint_as_float(b);
+}
+__device__ __forceinline__ int key_id(uint64_t k) { return (int)(0xffffffffu - (uint32_t)k); }
+
 }  // namespace lod

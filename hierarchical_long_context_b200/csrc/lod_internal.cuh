@@ -90,6 +90,14 @@ constexpr int kTargetCtas = 2 * 148;
 // Rows of one scan pipeline stage (a split streams whole stages).
 constexpr int kScanSlab = 64;
 
+// One of a scan split's best groups for one query row (tensor-core scan).
+struct SplitCand {
+  float s;    // scale * q . mean k
+  int id;     // group id within the unit (chunk * k + slot); -1: none
+  int meta;   // the group's gMeta word
+  int pad;
+};
+
 // A batch of query rows handled by one scan/refine launch pair.
 //  decode:  unit = (b, kvh); the unit's NQ = g rows are its query heads, all
 //           at t = seq_lens[b] - 1.
@@ -130,9 +138,11 @@ struct AttendArgs {
   int nsplit;               // splits of each unit's row list (groups, sinks, window)
   int64_t units;            // scan units in this launch
   float* part;              // [units][nsplit][NQ][d+2]  (m, l, acc)
-  float2* gsc;              // [units][NQ][Cmax * k] (score, meta) per visible group: score =
-                            // scale * q . mean k (-inf: not in that query row's softmax),
-                            // meta = the group's gMeta word (as float bits)
+  float2* gsc;              // CUDA-core scan: [units][NQ][Cmax * k] (score, meta) per visible
+                            // group: score = scale * q . mean k (-inf: not in that query row's
+                            // softmax), meta = the group's gMeta word (as float bits)
+  SplitCand* cand;          // tensor-core scan: [units][nsplit][NQ][G] each split's best G
+                            // groups per query row (by score, then smaller id); gsc unused
   void* out;                // [B][Hq][Tq][d]
   float* lse;               // [B][Hq][Tq] or null
   int32_t* sel_groups;      // [B][Hq][Tq][G] or null

@@ -24,12 +24,20 @@
 //              exceeds it by more than kTau (then the four warps agree on the
 //              tile max and rescale O in TMEM); p goes to shared memory as the
 //              bf16 B operand of MMA 2; per-thread partial sums; each
-//              group's score goes to the score array, from which the refine
-//              kernel picks the groups to open.
+//              group tile's scores, transposed, go to a double-buffered
+//              shared-memory slot for the selection warps.
+//   warps 6-9  each query row's best `top_groups` groups of the split: 16
+//              threads per query row each keep, in registers, the best G of
+//              every 16th group (score, then smaller id); a group enters a
+//              list only if it beats the list's G-th best and the row's
+//              bound (the largest G-th best of the 16 lists: G groups reach
+//              it).  At the end the 16 lists are merged, G rounds of a
+//              16-lane maximum, into the split's G best, from which the
+//              refine kernel picks the groups to open.
 //
-// The partial state (m, l, acc[d]) and the group scores are written in the
-// same layout as the CUDA-core scan, so the refine kernel is shared.  acc and
-// l are relative to the reference max m (every weight is at most e^kTau).
+// The partial state (m, l, acc[d]) is written in the same layout as the
+// CUDA-core scan, so the refine kernel is shared.  acc and l are relative to
+// the reference max m (every weight is at most e^kTau).
 #include <cudaTypedefs.h>
 
 #include "lod_internal.cuh"
@@ -43,13 +51,14 @@ constexpr int D = 128;
 constexpr int N = 16;            // MMA N: the unit's query rows (<= 8), zero padded
 constexpr int TROWS = 128;       // rows per tile: MMA 1's M, MMA 2's K
 constexpr int kStages = 3;
-constexpr int kThreads = 192;    // warp 0 copies, warp 1 issues MMAs, warps 2-5 softmax
+constexpr int kThreads = 320;    // warp 0 copies, warp 1 issues MMAs, warps 2-5 softmax, 6-9 selection
 constexpr int kSoftThreads = 128;
 constexpr int kBarSoft = 1;      // named barrier of the softmax warps
 constexpr uint32_t kTileBytes = TROWS * D * 2;  // one operand tile: 32 KB
 constexpr float kTau = 8.f;      // weights reach at most e^kTau before m moves
 constexpr uint32_t kTmemCols = 64;  // S buffers in columns [0, 32), O in [32, 48)
 constexpr uint32_t kColO = 32;
+constexpr int kTS = TROWS + 16;  // row stride of the transposed group scores (floats)
 
 struct TcSmem {
   static constexpr size_t off_K = 0;                                       // [stages][2][128][128 B]
@@ -59,14 +68,41 @@ struct TcSmem {
   static constexpr size_t off_cnt = off_P + 4 * N * 128;                   // int [stages][128]
   static constexpr size_t off_red = off_cnt + sizeof(int) * kStages * TROWS;  // float [4][8]
   static constexpr size_t off_flag = off_red + sizeof(float) * 4 * 8;         // int abort flag
-  static constexpr int kBars = 2 * kStages + 4 * 2 + 1;
-  static constexpr size_t off_bar = (off_flag + 16 + 7) & ~size_t(7);
+  static constexpr size_t off_sT = off_flag + 16;                      // float [2][8][kTS] group scores
+  static constexpr size_t off_sM = off_sT + sizeof(float) * 2 * 8 * kTS;  // int [2][128] their gMeta words
+  static constexpr int kBars = 2 * kStages + 4 * 2 + 1 + 4;
+  static constexpr size_t off_bar = (off_sM + 4 * 2 * TROWS + 7) & ~size_t(7);
   static constexpr size_t off_tmem = off_bar + 8 * kBars;
   static constexpr size_t bytes = off_tmem + 16 + 1024;  // + alignment slack
   static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
-template <int NQ>
+// Insert (v, id, meta) into the descending list (s, ix, mt) of GM entries:
+// every entry from the first one v beats moves down by one place (ties keep
+// the earlier entry, which has the smaller id).  A list of G < GM entries
+// occupies the last G slots below GM - G sentinels of +inf, so that its G-th
+// best is always s[GM - 1]; selects only, so the list stays in registers.
+template <int GM>
+__device__ __forceinline__ void list_insert(float (&s)[GM], int (&ix)[GM], int (&mt)[GM], float v, int id, int meta) {
+  bool act = false;
+  float cs = v;
+  int ci = id, cm = meta;
+#pragma unroll
+  for (int k = 0; k < GM; ++k) {
+    act = act || (v > s[k]);
+    const float ns = act ? cs : s[k];
+    const int ni = act ? ci : ix[k];
+    const int nm = act ? cm : mt[k];
+    cs = act ? s[k] : cs;
+    ci = act ? ix[k] : ci;
+    cm = act ? mt[k] : cm;
+    s[k] = ns;
+    ix[k] = ni;
+    mt[k] = nm;
+  }
+}
+
+template <int NQ, int GM>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ AttendArgs a) {
   static_assert(NQ <= 8, "query rows per unit");
@@ -83,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* Qs = sm + TcSmem::off_Q;
   unsigned char* Ps = sm + TcSmem::off_P;
   int* cnt_s = reinterpret_cast<int*>(sm + TcSmem::off_cnt);
+  float* sT = reinterpret_cast<float*>(sm + TcSmem::off_sT);
+  int* sM = reinterpret_cast<int*>(sm + TcSmem::off_sM);
   float* red = reinterpret_cast<float*>(sm + TcSmem::off_red);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + TcSmem::off_flag);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + TcSmem::off_bar);  // K/V tile + counts landed
@@ -92,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_free + 2;                                        // weights of tile i written
   uint64_t* o_done = p_full + 2;                                        // MMA 2 of tile i complete
   uint64_t* fin = o_done + 2;                                           // every MMA complete
+  uint64_t* sel_full = fin + 1;                                         // a group tile's scores transposed
+  uint64_t* sel_free = sel_full + 2;                                    // the selection has read them
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + TcSmem::off_tmem);
 
   // ---- unit (decode: (b, kvh); prefill: (b, kvh, position block))
@@ -122,6 +162,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[i], 1);
     }
     mbar_init(fin, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sel_full[i], 4);
+      mbar_init(&sel_free[i], 4);
+    }
     *abort_s = 0;
     fence_mbar_init();
     tc::prefetch_tensormap(&maps.gK);
@@ -130,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::prefetch_tensormap(&maps.V);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, kTmemCols);
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const int t = tid - 64;
     for (int c2 = t; c2 < 4 * N * 128 / 16; c2 += kSoftThreads)
       reinterpret_cast<uint4*>(Ps)[c2] = make_uint4(0, 0, 0, 0);
@@ -166,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint4 qv[kQPer];
 #pragma unroll
   for (int i = 0; i < kQPer; ++i) qv[i] = make_uint4(0, 0, 0, 0);
-  if (warp >= 2 && a.q_host) {
+  if (warp >= 2 && warp < 6 && a.q_host) {
 #pragma unroll
     for (int i = 0; i < kQPer; ++i) qv[i] = load_q(i);
   }
@@ -251,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     for (int i = 0; i < kStages && i < ntile; ++i) issue_tile(i);
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const int t = tid - 64;
 #pragma unroll
     for (int i = 0; i < kQPer; ++i) {
@@ -340,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ================================================================ softmax
     const int q = warp & 3, wq = warp - 2;
     const int r = 32 * q + lane;  // tile row of this thread, and O's dim at the end
@@ -351,8 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       m[j] = -INFINITY;
       l[j] = 0.f;
     }
-    const int64_t gcap = a.Cmax * a.k;
-    float2* gsc = a.gsc + u * NQ * gcap;  // this unit's (group score, meta), [NQ][gcap]
     bool alive = true;
     for (int i = 0; i < ntile; ++i) {
       const int st = i % kStages, buf = i & 1;
@@ -448,11 +490,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[buf]);
-      // group scores (-inf: not in this query row's softmax)
-      if (is_group && r0 + r < G_vis) {
+      // the group tile's scores, transposed (-inf: not in the row's
+      // softmax), and gMeta words for the selection warps (group tiles come
+      // first in a split: group tile i is tile i)
+      if (is_group) {
+        const int sb = i & 1;
+        if (i >= 2 && !wait(&sel_free[sb], (uint32_t)((i - 2) >> 1) & 1u)) alive = false;
+        if (alive) {
+          const bool vg = r0 + r < G_vis;
 #pragma unroll
-        for (int j = 0; j < NQ; ++j)
-          gsc[j * gcap + r0 + r] = make_float2(lg[j] == -INFINITY ? -INFINITY : sc[j], __int_as_float(meta));
+          for (int j = 0; j < NQ; ++j) sT[(sb * 8 + j) * kTS + r] = (vg && lg[j] != -INFINITY) ? sc[j] : -INFINITY;
+          sM[sb * TROWS + r] = meta;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sel_full[sb]);
       }
     }
     // ---------------------------------------------------------------- epilogue
@@ -485,6 +536,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         part[j * (D + 2) + 1] = alive ? red[j] + red[8 + j] + red[16 + j] + red[24 + j] : 0.f;
       }
     }
+  } else {
+    // ================================================================ selection
+    // this thread keeps the best G of query row jr's groups c, c + 16, c + 32,
+    // ... of every group tile (t = 16 jr + c); rows >= NQ keep empty lists
+    const int t = tid - 192, jr = t >> 4, cls = t & 15;
+    const int G = a.G;
+    float ls[GM];
+    int li[GM], lm[GM];
+#pragma unroll
+    for (int k = 0; k < GM; ++k) {
+      ls[k] = k < GM - G ? INFINITY : -INFINITY;
+      li[k] = -1;
+      lm[k] = 0;
+    }
+    float bnd = -INFINITY;  // the largest G-th best of the row's 16 lists
+    bool alive = true;
+    const int ngt = (int)((t1 < gt ? t1 : gt) - t0);  // group tiles of this split
+    for (int i = 0; i < ngt; ++i) {
+      const int sb = i & 1;
+      alive = __all_sync(0xffffffffu, wait(&sel_full[sb], (uint32_t)(i >> 1) & 1u));
+      if (!alive) break;
+      // a group enters a list if it beats both the list's G-th best and the
+      // row's bound (the tile's groups all have larger ids than those behind
+      // the bound, so a tie with it loses)
+      if (jr < NQ) {
+        const int64_t r0 = (t0 + i) * TROWS;
+#pragma unroll
+        for (int e8 = 0; e8 < TROWS / 16; ++e8) {
+          const int e = cls + 16 * e8;
+          const float v = sT[(sb * 8 + jr) * kTS + e];
+          if (v > fmaxf(ls[GM - 1], bnd)) list_insert<GM>(ls, li, lm, v, (int)(r0 + e), sM[sb * TROWS + e]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sel_free[sb]);
+      float kb = ls[GM - 1];
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) kb = fmaxf(kb, __shfl_xor_sync(0xffffffffu, kb, o));
+      bnd = fmaxf(bnd, kb);
+    }
+    // the split's best G of row jr: G rounds in which each of the row's 16
+    // lists offers its best entry not yet taken and the largest key wins
+    // (lanes of both rows of a warp run every round: the shuffles take the
+    // whole warp)
+    SplitCand* co = a.cand + ((u * a.nsplit + s) * NQ + (jr < NQ ? jr : 0)) * G;
+    int h = GM - G, kept = 0;
+    for (int k = 0; k < G; ++k) {
+      float hs = -INFINITY;
+      int hid = -1, hm = 0;
+#pragma unroll
+      for (int x = 0; x < GM; ++x)
+        if (x == h) {
+          hs = ls[x];
+          hid = li[x];
+          hm = lm[x];
+        }
+      const uint64_t mine = (alive && jr < NQ && h < GM && hs != -INFINITY) ? group_key(hs, hid) : 0ull;
+      uint64_t best = mine;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const uint64_t x = __shfl_xor_sync(0xffffffffu, best, o);
+        best = x > best ? x : best;
+      }
+      if (best != 0ull) {
+        kept = k + 1;
+        if (mine == best) {  // one list holds it: group ids are distinct
+          SplitCand c;
+          c.s = hs;
+          c.id = hid;
+          c.meta = hm;
+          c.pad = 0;
+          co[k] = c;
+          ++h;
+        }
+      }
+    }
+    if (jr < NQ && cls < G && cls >= kept) {
+      SplitCand c;
+      c.s = -INFINITY;
+      c.id = -1;
+      c.meta = 0;
+      c.pad = 0;
+      co[cls] = c;
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -493,9 +628,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int NQ>
 cudaError_t launch_nq(const AttendArgs& a, const TcMaps& maps, cudaStream_t stream) {
-  auto kern = scan_tc_kernel<NQ>;
+  // registers for the group lists: G <= 8 or G <= 16 entries
+  auto kern = a.G <= 8 ? scan_tc_kernel<NQ, 8> : scan_tc_kernel<NQ, 16>;
   const size_t smem = TcSmem::bytes;
-  cudaError_t e = set_smem_once<scan_tc_kernel<NQ>>(smem);
+  cudaError_t e = a.G <= 8 ? set_smem_once<scan_tc_kernel<NQ, 8>>(smem) : set_smem_once<scan_tc_kernel<NQ, 16>>(smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)a.units, (unsigned)a.nsplit), dim3(kThreads), smem, stream, maps, a);
 }
