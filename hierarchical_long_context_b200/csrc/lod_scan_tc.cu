@@ -562,10 +562,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the bound, so a tie with it loses)
       if (jr < NQ) {
         const int64_t r0 = (t0 + i) * TROWS;
+        float v8[TROWS / 16];
+        unsigned cm = 0;  // this lane's candidates (bit e8: group cls + 16 e8)
+        const float th = fmaxf(ls[GM - 1], bnd);
 #pragma unroll
         for (int e8 = 0; e8 < TROWS / 16; ++e8) {
+          v8[e8] = sT[(sb * 8 + jr) * kTS + cls + 16 * e8];
+          cm |= (v8[e8] > th ? 1u : 0u) << e8;
+        }
+        while (cm) {  // in id order; each must still beat the list's G-th best
+          const int e8 = __ffs(cm) - 1;
+          cm &= cm - 1;
+          float v = v8[0];
+#pragma unroll
+          for (int x = 1; x < TROWS / 16; ++x) v = x == e8 ? v8[x] : v;
           const int e = cls + 16 * e8;
-          const float v = sT[(sb * 8 + jr) * kTS + e];
           if (v > fmaxf(ls[GM - 1], bnd)) list_insert<GM>(ls, li, lm, v, (int)(r0 + e), sM[sb * TROWS + e]);
         }
       }
