@@ -450,64 +450,90 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           for (int e = 0; e < 32; ++e) y[e] = e <= rc ? fmaf(y[e], scl, -sub) : -INFINITY;
         }
       };
-      // ---- pass 1: the logit max
-      float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent max chains
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float y[32];
-        logits(c, y, 0.f);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) xa[e & 3] = fmaxf(xa[e & 3], y[e]);
-      }
-      const float xm = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
-      // the reference max moves when a logit exceeds it by more than kTau2
-      const bool need = xm > m + kTau2;
+      // Weights 2^(logit - m) into P, in one pass against the current
+      // reference max m: a chunk with a logit above m + kTau2 (and a row's
+      // first tile) sends the warp through the max pass first, after which
+      // the weights are computed again.  Both give the same weights
+      // whenever the reference max does not move.
+      bool redo = __any_sync(0xffffffffu, m == -INFINITY);
       bool waited = false;
-      if (__any_sync(0xffffffffu, need)) {
-        const float mn = need ? xm : m;
-        const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - mn);
-        l *= corr;
-        m = mn;
-        if (i > 0) {
-          alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u));
-          waited = true;
-          if (alive) {
-            tc::fence_after_sync();
+      float la[4];  // independent sum chains
+      for (int att = 0; att < 2; ++att) {
+        if (redo) {
+          // ---- the logit max of the tile
+          float xa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent max chains
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float y[32];
+            logits(c, y, 0.f);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float ov[32];
-              tc::tmem_ld32(tmem + tl + kColO + 32 * c, ov);
+            for (int e = 0; e < 32; ++e) xa[e & 3] = fmaxf(xa[e & 3], y[e]);
+          }
+          const float xm = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+          // the reference max moves when a logit exceeds it by more than kTau2
+          const bool need = xm > m + kTau2;
+          if (__any_sync(0xffffffffu, need)) {
+            const float mn = need ? xm : m;
+            const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - mn);
+            l *= corr;
+            m = mn;
+            if (i > 0) {
+              alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u));
+              waited = true;
+              if (alive) {
+                tc::fence_after_sync();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] *= corr;
-              tc::tmem_st32(tmem + tl + kColO + 32 * c, ov);
+                for (int c = 0; c < 4; ++c) {
+                  float ov[32];
+                  tc::tmem_ld32(tmem + tl + kColO + 32 * c, ov);
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) ov[e] *= corr;
+                  tc::tmem_st32(tmem + tl + kColO + 32 * c, ov);
+                }
+              }
             }
           }
         }
-      }
-      // P is free once MMA 2 of the previous tile is done
-      if (i > 0 && !waited) alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u)) && alive;
-      if (!alive) break;
-      const float mu = m == -INFINITY ? 0.f : m;
-      // ---- pass 2: the weights 2^(logit - m) into P
-      float la[4] = {0.f, 0.f, 0.f, 0.f};  // independent sum chains
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float y[32];
-        logits(c, y, mu);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = ex2_approx(y[8 * q + e]);
-            la[e & 3] += p[e];
-          }
-          const int ch = 4 * c + q;
-          *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
-              make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                         pack_bf16x2(p[6], p[7]));
+        // P is free once MMA 2 of the previous tile is done
+        if (i > 0 && !waited) {
+          alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u)) && alive;
+          waited = true;
         }
+        if (!alive) break;
+        const float mu = m == -INFINITY ? 0.f : m;
+        la[0] = la[1] = la[2] = la[3] = 0.f;
+        bool bail = false;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float y[32];
+          logits(c, y, mu);
+          if (!redo) {  // would this chunk move the reference max?
+            float ym[4] = {y[0], y[1], y[2], y[3]};
+#pragma unroll
+            for (int e = 4; e < 32; ++e) ym[e & 3] = fmaxf(ym[e & 3], y[e]);
+            if (__any_sync(0xffffffffu, fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3])) > kTau2)) {
+              bail = true;
+              break;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              p[e] = ex2_approx(y[8 * q + e]);
+              la[e & 3] += p[e];
+            }
+            const int ch = 4 * c + q;
+            *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
+                make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                           pack_bf16x2(p[6], p[7]));
+          }
+        }
+        if (!bail) break;
+        redo = true;
       }
+      if (!alive) break;
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[st]);
