@@ -1,7 +1,9 @@
 // lod_attend.cu -- LoD decode and prefill attention ("Level of Detail
 // Attention", How It Works, paragraphs 2-3).
 //
-// Two kernels per batch of query rows:
+// Two kernels per batch of query rows (bf16 caches with d = 128 take the
+// tensor-core scan of lod_scan_tc.cu, which hands the refine kernel each
+// split's best groups instead of every group's score):
 //
 //  scan    grid (unit, split).  A unit is one KV head of one sequence with its
 //          NQ query rows (decode: the g query heads; prefill: g heads x NP
@@ -15,7 +17,8 @@
 //          leaving a partial softmax state (max, sum, acc[d]) over ALL its rows.
 //  refine  one CTA per query row, launched as a programmatic dependent of the
 //          scan.  It merges the split states, picks the top `top_groups`
-//          groups from the unit's score array, removes those groups'
+//          groups from the unit's score array (or from the splits' best
+//          groups), removes those groups'
 //          coarse terms (they are replaced by finer entries), scores each
 //          opened group's page summaries, opens the top `top_pages` pages and
 //          adds their tokens exactly (values staged by TMA), adds the other
@@ -24,8 +27,9 @@
 //
 // Removing the opened groups after the fact (instead of holding them out of
 // the scan) is numerically safe: the entries that replace an opened group --
-// its pages, or their tokens -- carry at least the group's own mass (the
-// method's "conservative estimate" property: n exp(q.mean k) <= sum exp(q.k)),
+// its pages, or their tokens -- carry at least the group's own mass (by
+// Jensen's inequality, n exp(q.mean k) <= sum exp(q.k): the coarse term never
+// overstates a group),
 // so the final normaliser is never smaller than what was subtracted and the
 // cancellation error stays at the fp32 rounding level of the output.
 #include <type_traits>

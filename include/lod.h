@@ -311,10 +311,11 @@ int32_t lod_prefill(const lod_params* p, const void* q, int64_t q_begin, int64_t
  *     that loads the library holds that array until the process exits.
  *     Shapes whose scratch (lod_workspace_bytes(LOD_OP_DECODE)) exceeds it
  *     are rejected with LOD_EINVAL and a message naming both sizes; nothing
- *     is enqueued then.  (The 128K-context decode of 4 sequences x 8 KV heads
- *     x 8 query heads per KV head needs about 4.7 MB; a 1M-context decode of
- *     one sequence with the same heads needs about 9.0 MB, more than the
- *     array holds, and must use lod_decode.)
+ *     is enqueued then.  (With bf16 caches and d = 128 the 128K-context
+ *     decode of 4 sequences x 8 KV heads x 8 query heads per KV head needs
+ *     about 0.66 MB and a 1M-context decode of one sequence with the same
+ *     heads about 0.75 MB; fp32 caches or d = 64 keep every group's score
+ *     and need more, e.g. about 9.6 MB for that 1M decode in fp32.)
  *   - status: nullable device pointer to a 4-byte aligned uint32_t that
  *     receives (bitwise OR) this call's LOD_ST_* bits; the caller zeroes it
  *     (a misaligned pointer is rejected with LOD_EINVAL).  When NULL the

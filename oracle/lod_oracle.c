@@ -19,7 +19,7 @@
  *     unopened group enters as its average key and value repeated by its key
  *     count, and the unopened pages of opened groups enter the same way.
  *   - paragraph 4: with zero-variance groups this equals full attention, and
- *     otherwise it is a conservative estimate of the attention mass.
+ *     otherwise the coarse terms never overstate a group's attention mass.
  *
  * Where the page is silent the oracle takes these readings (each one is also
  * listed with its reason in the design notes of the repository):
