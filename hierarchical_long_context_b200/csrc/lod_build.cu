@@ -537,14 +537,24 @@ __global__ void append_kv_kernel(uint4* K, uint4* V, int64_t sb, int64_t sh, int
   // its input-free set-up now; it reads the cache only after this grid is done
   pdl_launch_dependents();
   const int b = blockIdx.x;
+  const int n = Hkv * row16;
+  // this thread's first piece of the new rows goes out before the sequence
+  // length is known (the rows may sit in host memory: two round trips over
+  // the host link would otherwise follow one another)
+  const int i0 = threadIdx.x;
+  uint4 k0 = make_uint4(0, 0, 0, 0), v0 = k0;
+  if (i0 < n) {
+    k0 = kn[(int64_t)b * n + i0];
+    v0 = vn[(int64_t)b * n + i0];
+  }
   const int64_t t = seq_lens[b] - 1;
   if (t < 0 || t >= Tmax) return;
-  for (int i = threadIdx.x; i < Hkv * row16; i += blockDim.x) {
+  for (int i = i0; i < n; i += blockDim.x) {
     const int h = i / row16, c = i % row16;
     const int64_t dst = b * sb + h * sh + t * st + c;
-    const int64_t src = ((int64_t)b * Hkv + h) * row16 + c;
-    K[dst] = kn[src];
-    V[dst] = vn[src];
+    const int64_t src = (int64_t)b * n + i;
+    K[dst] = i == i0 ? k0 : kn[src];
+    V[dst] = i == i0 ? v0 : vn[src];
   }
 }
 

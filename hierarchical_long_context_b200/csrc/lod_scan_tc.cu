@@ -186,11 +186,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_l2(static_cast<const __nv_bfloat16*>(a.q) + (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D + (t & 1) * 64);
     }
   }
-  // launched as a programmatic dependent: inputs are read only after the
-  // preceding kernel has completed; the refine kernel may launch right away
-  // (it waits for this grid's completion before reading what it writes)
-  pdl_wait();
-  pdl_launch_dependents();
 
   // query piece i of this softmax thread (16 bytes; zero for a missing row)
   constexpr int kQPer = N * (D / 8) / kSoftThreads;  // 16-byte pieces per softmax thread
@@ -204,9 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     return __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
                                                  (((int64_t)b * a.Hq + hq) * a.Tq + pi) * D) + c);
   };
-  // q in host memory: its loads go out first (which rows exist does not
-  // depend on the sequence length, so they overlap its read; rows of an
-  // invalid sequence are zeroed below); q in device memory is read after
+  // q in host memory was written by the host before the call was enqueued
+  // (the entry points' contract), so its loads over the host link go out
+  // before the dependency wait, overlapping the preceding kernel (which rows
+  // exist does not depend on the sequence length; rows of an invalid
+  // sequence are zeroed below); q in device memory is read after the wait
   uint4 qv[kQPer];
 #pragma unroll
   for (int i = 0; i < kQPer; ++i) qv[i] = make_uint4(0, 0, 0, 0);
@@ -214,6 +211,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < kQPer; ++i) qv[i] = load_q(i);
   }
+
+  // launched as a programmatic dependent: device inputs are read only after
+  // the preceding kernel has completed; the refine kernel may launch right away
+  // (it waits for this grid's completion before reading what it writes)
+  pdl_wait();
+  pdl_launch_dependents();
 
   int64_t t_row[NQ];
   bool ok[NQ];

@@ -19,10 +19,14 @@
  *    v_new, status) may also be page-locked host memory mapped at its host
  *    address (cudaHostAlloc / cudaMallocHost under unified addressing): the
  *    kernels then read or write those bytes over the host link themselves,
- *    with no separate copy.  The entry points check these buffers and refuse
- *    pageable host memory and another device's memory (LOD_EINVAL) before
- *    anything is enqueued.  The KV cache, the index and the workspace must
- *    be device memory.
+ *    with no separate copy.  Inputs in such host memory (q, k_new, v_new)
+ *    must be written by the host before the call is enqueued, not by GPU
+ *    work still pending on the stream: the kernels may read them as soon as
+ *    they start, before earlier kernels on the stream have finished (device
+ *    inputs are read only after that).  The entry points check these buffers
+ *    and refuse pageable host memory and another device's memory
+ *    (LOD_EINVAL) before anything is enqueued.  The KV cache, the index and
+ *    the workspace must be device memory.
  *  - The caller owns every buffer.  The library never allocates or frees
  *    device memory and never synchronises the stream, with one exception:
  *    lod_get_status() copies 4 bytes to the host and waits for them.
