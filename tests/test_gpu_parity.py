@@ -133,6 +133,8 @@ def test_decode_on_gpu_index_matches_oracle(name, T, seq_lens):
     dict(top_pages=0),                                                         # two-tier LoD, g=8
     dict(d=64, dtype="f32", Hq=4, Hkv=2, top_groups=16, top_pages=0),          # two-tier, CUDA-core scan
     dict(Hq=16, Hkv=2, sinks=100),                                             # more sinks than free lanes
+    dict(Hq=2, Hkv=2),                                                         # bf16 d=128 MHA: one query row per scan unit
+    dict(Hq=8, Hkv=2, top_groups=12),                                          # g=4, G between 8 and 16
 ])
 def test_decode_parameter_sweep(kw):
     """Head ratios, head sizes, dtypes, cluster counts and selection widths at
@@ -383,6 +385,54 @@ def test_zero_variance_decode_equals_dense():
         out = api.lod_decode(p, q, Kd, Vd, torch.tensor([w.T], device="cuda"), ix)
         dout, _ = oracle.dense_row(cfg, _np(q[0, 0]), w.T - 1, K, V)
         assert np.max(np.abs(_np(out[0, 0]) - dout)) < 1e-5
+
+
+@pytest.mark.parametrize("B, Hkv", [(1, 1), (4, 8)])
+def test_tied_group_scores_open_the_smallest_ids_across_splits(B, Hkv):
+    """Groups with equal scores rank by smaller id (D8) however the scan
+    splits the unit's groups: a best key S sits in every 37th chunk and a
+    second key G in every chunk, every chunk's four keys repeated 64 times,
+    so the index's group means are those keys exactly and all S groups (and
+    all G groups) tie.  The query points at S: the 8 opened groups must be
+    the S groups of chunks 0, 37, .., 222 by id, then the G group of chunk 0
+    (with B = 4, Hkv = 8 each split scans several group tiles)."""
+    dev = _cuda()
+    T, k, d = 65536, 4, 128
+    w = synth.WORKLOADS["decode_gqa_128k_bf16"].with_(B=B, Hkv=Hkv, Hq=8 * Hkv, T=T)
+    p = lt.params_of(w, k, Tmax=T)
+    e = torch.eye(d)
+    S, G = 2.0 * e[0], 1.0 * e[0]
+    filler = [e[1] * 0.5, e[2] * 0.5, e[3] * 0.5, e[4] * 0.5]
+    keys = torch.zeros(T // 256, 4, d)
+    for c in range(T // 256):
+        ks = [S, G, filler[0], filler[1]] if c % 37 == 0 else [G, filler[0], filler[1], filler[2]]
+        keys[c] = torch.stack(ks)
+    Kc = keys.repeat_interleave(64, dim=1).reshape(T, d)  # each key on 64 consecutive positions
+    Kd = Kc.to(torch.bfloat16).to(dev).expand(B, Hkv, T, d).contiguous()
+    Vd = torch.randn(B, Hkv, T, d, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16).to(dev)
+    ix = api.Index(p)
+    api.lod_build_index(p, Kd, Vd, 0, T // 256, ix)
+    q = torch.zeros(B, 8 * Hkv, d)
+    q[..., 0] = 1.0
+    q = q.to(torch.bfloat16).to(dev)
+    sg = torch.empty(B, 8 * Hkv, p.top_groups, dtype=torch.int32, device=dev)
+    ws = api.workspace(p, api._lib.LOD_OP_DECODE)
+    api.lod_decode(p, q, Kd, Vd, torch.full((B,), T, dtype=torch.int64, device=dev), ix, sel_groups=sg, ws=ws)
+    torch.cuda.synchronize()
+    assert api.lod_get_status(ws) == 0
+    gK = ix.gK.float().cpu()
+    sgc = sg.cpu()
+    vis = (T // 256 - p.window // 256) * k  # groups of the complete chunks before the window
+    for b in range(B):
+        for h in range(Hkv):
+            def slot_of(c, key):
+                hit = [j for j in range(k) if torch.equal(gK[b, h, c * k + j], key)]
+                assert len(hit) == 1, (c, hit)
+                return c * k + hit[0]
+            want = [slot_of(c, S) for c in range(0, T // 256, 37) if (c + 1) * k <= vis]
+            want = (want + [slot_of(0, G)])[: p.top_groups]
+            for hq in range(h * 8, h * 8 + 8):
+                assert sgc[b, hq].tolist() == want, (b, hq, sgc[b, hq].tolist(), want)
 
 
 # ------------------------------------------------------------------ prefill
