@@ -4,8 +4,8 @@
 // "Level of Detail Attention", section "How It Works": every visible group
 // summary (mean key, mean value, ln count) and every window token of one
 // (sequence, KV head) enters one online softmax for each of the unit's query
-// rows; every group's score is kept so that the best `top_groups` groups can
-// be opened.  A unit's rows are cut into tiles of 128; a CTA streams a
+// rows, and each split keeps its best `top_groups` groups per query row for
+// the groups to open.  A unit's rows are cut into tiles of 128; a CTA streams a
 // contiguous run of tiles through a warp-specialised pipeline:
 //
 //   warp 0     producer: TMA copies of the K and V tiles (two 64-column boxes
