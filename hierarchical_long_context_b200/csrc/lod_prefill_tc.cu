@@ -670,6 +670,14 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         const int gid = alive ? ti[k] : -1;
         pos[k] = (k >= GM - a.G && gid >= 0) ? atomicAdd(a.cnt + grow0 + gid, 1) : -1;
       }
+      // the groups' sizes, all loads in flight together (the stores below
+      // would otherwise keep each load behind the previous one's stores)
+      int gsz[GM];
+#pragma unroll
+      for (int k = 0; k < GM; ++k) {
+        const int gid = alive ? ti[k] : -1;
+        gsz[k] = (k >= GM - a.G && gid >= 0) ? __ldg(a.gMeta + grow0 + gid) & 0xffff : 0;
+      }
       *reinterpret_cast<float2*>(stp) = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
       const float mu = m == -INFINITY ? 0.f : m;
 #pragma unroll
@@ -679,7 +687,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           const int gid = alive ? ti[k] : -1;
           float wk = 0.f;
           if (gid >= 0) {
-            const int c = a.gMeta[grow0 + gid] & 0xffff;
+            const int c = gsz[k];
             wk = ex2_approx(fmaf(ts[k], scl, log2f((float)(c > 0 ? c : 1))) - mu);
           }
           a.sel[wr * a.G + j] = gid;
