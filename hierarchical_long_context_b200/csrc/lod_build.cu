@@ -286,12 +286,28 @@ __global__ void __launch_bounds__(kBuildThreads,
       float2 dot[KMAX];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) dot[j] = make_float2(0.f, 0.f);
+      if constexpr (KMAX == 4) {
+        // every slot of the centroid row, two per 16-byte load (the slots
+        // past k hold no centroid; their sums are never read)
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        const float2 x = pair_of<T>(kw, p);
+        for (int p = 0; p < NP; ++p) {
+          const float2 x = pair_of<T>(kw, p);
+          const float4* c4 = reinterpret_cast<const float4*>(cen2 + p * KMAX);
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (j < k) dot[j] = ffma2(x, cen2[p * KMAX + j], dot[j]);
+          for (int j2 = 0; j2 < KMAX / 2; ++j2) {
+            const float4 cc = c4[j2];
+            dot[2 * j2] = ffma2(x, make_float2(cc.x, cc.y), dot[2 * j2]);
+            dot[2 * j2 + 1] = ffma2(x, make_float2(cc.z, cc.w), dot[2 * j2 + 1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const float2 x = pair_of<T>(kw, p);
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j)
+            if (j < k) dot[j] = ffma2(x, cen2[p * KMAX + j], dot[j]);
+        }
       }
       auto cn = [&](int j) {
         float v = cnorm[j * NSLOT];
