@@ -487,11 +487,30 @@ __global__ void __launch_bounds__(kBuildThreads,
     constexpr int C16 = ROWB / 16;  // 16-byte pieces per row
     uint4* mKc = reinterpret_cast<uint4*>(static_cast<T*>(a.mK) + ((unit * a.Cmax + c) * kChunk) * D);
     uint4* mVc = reinterpret_cast<uint4*>(static_cast<T*>(a.mV) + ((unit * a.Cmax + c) * kChunk) * D);
-    for (int item = tid; item < n * C16; item += kBuildThreads) {
-      const int m = item / C16, q = item % C16;
-      const int row = first + perm_s[m];
-      mKc[item] = reinterpret_cast<const uint4*>(xs + row * D)[q];
-      mVc[item] = __ldg(reinterpret_cast<const uint4*>(Vc + (int64_t)row * a.st) + q);
+    // four pieces per thread at a time, every load before any store (a
+    // store would otherwise hold the next load back until the previous
+    // load's round trip had ended)
+    constexpr int U = 4;
+    for (int base = tid; base < n * C16; base += U * kBuildThreads) {
+      uint4 kq[U], vq[U];
+#pragma unroll
+      for (int x = 0; x < U; ++x) {
+        const int item = base + x * kBuildThreads;
+        if (item < n * C16) {
+          const int m = item / C16, q = item % C16;
+          const int row = first + perm_s[m];
+          kq[x] = reinterpret_cast<const uint4*>(xs + row * D)[q];
+          vq[x] = __ldg(reinterpret_cast<const uint4*>(Vc + (int64_t)row * a.st) + q);
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < U; ++x) {
+        const int item = base + x * kBuildThreads;
+        if (item < n * C16) {
+          mKc[item] = kq[x];
+          mVc[item] = vq[x];
+        }
+      }
     }
   }
   // unused page slots hold zeros
