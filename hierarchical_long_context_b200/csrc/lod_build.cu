@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kBuildThreads,
       float2 dot[KMAX];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) dot[j] = make_float2(0.f, 0.f);
-      if constexpr (KMAX == 4) {
+      if constexpr (KMAX <= 8) {
         // every slot of the centroid row, two per 16-byte load (the slots
         // past k hold no centroid; their sums are never read)
 #pragma unroll
