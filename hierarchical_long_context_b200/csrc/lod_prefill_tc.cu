@@ -77,18 +77,20 @@ constexpr int kBarSelA = 3;      // named barrier of warpgroups 2 and 3 (merge o
 constexpr int kBarEndA = 4;      // named barrier of warpgroups 0-2 before TMEM is released
 
 // Tensor memory of the scan: S double-buffered in columns [0, 256), O in
-// [256, 384), the query tile (bf16 pairs, MMA 1's A operand) in [384, 448).
-constexpr uint32_t kColO = 256, kColQ = 384;
+// [256, 384), the weights P (bf16 pairs, MMA 2's A operand) double-buffered
+// in [384, 512), so the softmax of tile i + 1 does not wait for MMA 2 of
+// tile i.
+constexpr uint32_t kColO = 256, kColP = 384;
 
 struct SmemA {
   static constexpr size_t off_K = 0;                          // [2 stages][2 halves][128][128 B]
   static constexpr size_t off_V = off_K + 2 * kTileBytes;     // [2 stages]
-  static constexpr size_t off_P = off_V + 2 * kTileBytes;     // [2 halves][128][128 B]
-  static constexpr size_t off_cand = off_P + kTileBytes;      // float2 [2][128][kCandCap + 1] (+1: a junk slot)
+  static constexpr size_t off_Q = off_V + 2 * kTileBytes;     // the query tile [2 halves][128][128 B]
+  static constexpr size_t off_cand = off_Q + kTileBytes;      // float2 [2][128][kCandCap + 1] (+1: odd row stride)
   static constexpr size_t off_meta = off_cand + 2 * 128 * (kCandCap + 1) * 8;  // int [2][128]
   static constexpr size_t off_lnc = off_meta + 2 * 128 * 4;   // float [2][128]
   static constexpr size_t off_ml = off_lnc + 2 * 128 * 4;   // float2 [128] softmax state handed over
-  static constexpr int kBars = 18;
+  static constexpr int kBars = 20;
   static constexpr size_t off_bar = off_ml + 128 * 8;
   static constexpr size_t off_misc = off_bar + 8 * kBars;     // tmem slot, abort flag
   static constexpr size_t bytes = off_misc + 16 + 1024;
@@ -137,6 +139,15 @@ __device__ __forceinline__ void topk_insert_ranked(float (&s)[GM], int (&ix)[GM]
   }
 }
 
+// Store (x, y) to shared memory at p when c holds (a predicated store: a
+// miss costs an issue slot but no shared-memory bandwidth).
+__device__ __forceinline__ void sts_f2_if(float2* p, float x, float y, bool c) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n @q st.shared.v2.f32 [%0], {%1, %2};\n}" ::"r"(smem_u32(p)),
+      "f"(x), "f"(y), "r"((int)c)
+      : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -176,7 +187,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                                                        ~uintptr_t(1023));
   unsigned char* Kring = sm + SmemA::off_K;
   unsigned char* Vring = sm + SmemA::off_V;
-  unsigned char* Ps = sm + SmemA::off_P;
+  unsigned char* Qs = sm + SmemA::off_Q;
   float2* cand_s = reinterpret_cast<float2*>(sm + SmemA::off_cand);
   int* meta_s = reinterpret_cast<int*>(sm + SmemA::off_meta);
   float* lnc_s = reinterpret_cast<float*>(sm + SmemA::off_lnc);
@@ -187,11 +198,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   uint64_t* vempty = vfull + 2;
   uint64_t* s_full = vempty + 2;
   uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* fin = o_done + 1;
+  uint64_t* p_full = s_free + 2;  // [2]: weights of tile i written (buffer i & 1)
+  uint64_t* o_done = p_full + 2;  // [2]: MMA 2 of tile i complete
+  uint64_t* fin = o_done + 2;
   uint64_t* lnc_ready = fin + 1;  // [2]: ln counts of a group tile written
-  uint64_t* q_ready = lnc_ready + 2;  // the query tile is in TMEM
+  uint64_t* q_ready = lnc_ready + 2;  // the query tile is in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SmemA::off_misc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + SmemA::off_misc + 4);
 
@@ -228,8 +239,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 12);  // four softmax warps + eight top-G warps
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_done[i], 1);
+    }
     mbar_init(fin, 1);
     mbar_init(q_ready, 4);
     *abort_s = 0;
@@ -312,20 +325,20 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       const uint32_t idO = tc::idesc_bf16(128, 128, false, true);
-      const uint32_t pb = smem_u32(Ps);
-      auto mma2 = [&](int j) -> bool {  // O += P_j V_j
-        if (!wait(p_full, (uint32_t)j & 1u)) return false;
+      const uint32_t qb = smem_u32(Qs);
+      auto mma2 = [&](int j) -> bool {  // O += P_j V_j (P_j from tensor memory)
+        if (!wait(&p_full[j & 1], (uint32_t)(j >> 1) & 1u)) return false;
         if (!wait(&vfull[j & 1], (uint32_t)(j >> 1) & 1u)) return false;
         tc::fence_after_sync();
         const uint32_t vb = smem_u32(Vring + (j & 1) * kTileBytes);
+        const uint32_t pt = tmem + kColP + 64 * (uint32_t)(j & 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = tc::desc_kmajor_sw128(pb + (kk >> 2) * kHalf + (kk & 3) * 32);
           const uint64_t bd = tc::desc_mnmajor_sw128(vb + kk * 2048, kHalf);
-          tc::mma_bf16(tmem + kColO, ad, bd, idO, j > 0 || kk > 0);
+          tc::mma_bf16_ts(tmem + kColO, pt + 8 * kk, bd, idO, j > 0 || kk > 0);
         }
         tc::mma_commit(&vempty[j & 1]);
-        tc::mma_commit(o_done);
+        tc::mma_commit(&o_done[j & 1]);
         return true;
       };
       bool go = wait(q_ready, 0), any = false;  // the query tile, staged by the softmax warps
@@ -336,8 +349,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         const uint32_t kb = smem_u32(Kring + (i & 1) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = tc::desc_kmajor_sw128(qb + (kk >> 2) * kHalf + (kk & 3) * 32);
           const uint64_t bd = tc::desc_kmajor_sw128(kb + (kk >> 2) * kHalf + (kk & 3) * 32);
-          tc::mma_bf16_ts(tmem + (uint32_t)(i & 1) * 128, tmem + kColQ + 8 * kk, bd, idS, kk > 0);
+          tc::mma_bf16(tmem + (uint32_t)(i & 1) * 128, ad, bd, idS, kk > 0);
         }
         tc::mma_commit(&kempty[i & 1]);
         tc::mma_commit(&s_full[i & 1]);
@@ -360,24 +374,19 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     const int r = 32 * q4 + lane;  // query row of this thread (and the key row it stages)
     const uint32_t tl = (uint32_t)(32 * q4) << 16;
     {
-      // the query tile into TMEM lane r (MMA 1's A operand): row r = position r / g, head r % g
+      // the query tile, row r of MMA 1's A operand (128-byte swizzled, like
+      // a key tile): row r = position r / g, head r % g
       const int64_t pi = pos0 + r / a.g;
       const int hq = kvh * a.g + r % a.g;
       const bool okr = pi < pos_end;
       const __nv_bfloat16* src = a.q + (((int64_t)b * a.Hq + hq) * a.Tq + (okr ? pi : 0)) * D;
+      uint4 qw[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float qv[32];
+      for (int c = 0; c < 16; ++c)
+        qw[c] = okr ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 w = okr ? __ldg(reinterpret_cast<const uint4*>(src) + 8 * h + c) : make_uint4(0, 0, 0, 0);
-          qv[4 * c] = __uint_as_float(w.x);
-          qv[4 * c + 1] = __uint_as_float(w.y);
-          qv[4 * c + 2] = __uint_as_float(w.z);
-          qv[4 * c + 3] = __uint_as_float(w.w);
-        }
-        tc::tmem_st32(tmem + tl + kColQ + 32 * h, qv);
-      }
+      for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(Qs + (c >> 3) * kHalf + sw_off(r, c)) = qw[c];
+      tc::fence_proxy_async();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
@@ -478,7 +487,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             l *= corr;
             m = mn;
             if (i > 0) {
-              alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u));
+              alive = __all_sync(0xffffffffu, wait(&o_done[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u));
               waited = true;
               if (alive) {
                 tc::fence_after_sync();
@@ -494,9 +503,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             }
           }
         }
-        // P is free once MMA 2 of the previous tile is done
-        if (i > 0 && !waited) {
-          alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(i - 1) & 1u)) && alive;
+        // P's buffer i & 1 is free once MMA 2 of tile i - 2 is done (a wait
+        // for tile i - 1 above covers it)
+        if (i > 1 && !waited) {
+          alive = __all_sync(0xffffffffu, wait(&o_done[i & 1], (uint32_t)((i - 2) >> 1) & 1u)) && alive;
           waited = true;
         }
         if (!alive) break;
@@ -516,6 +526,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
               break;
             }
           }
+          uint32_t pw[16];  // the chunk's weights as bf16 pairs: columns 16 c .. 16 c + 15 of P
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float p[8];
@@ -524,11 +535,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
               p[e] = ex2_approx(y[8 * q + e]);
               la[e & 3] += p[e];
             }
-            const int ch = 4 * c + q;
-            *reinterpret_cast<uint4*>(Ps + (ch >> 3) * kHalf + sw_off(r, ch)) =
-                make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                           pack_bf16x2(p[6], p[7]));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pw[4 * q + e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
           }
+          tc::tmem_st16(tmem + tl + kColP + 64 * (uint32_t)st + 16 * c, pw);
         }
         if (!bail) break;
         redo = true;
@@ -538,10 +548,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[st]);
       l += (la[0] + la[1]) + (la[2] + la[3]);
-      tc::fence_proxy_async();
+      tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[st]);
     }
     // the row's softmax state goes to the selection warps, which write it
     ml_s[r] = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
@@ -605,10 +615,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
             for (int hh = 0; hh < 2; ++hh) {
               if (__any_sync(0xffffffffu, ncand > kCandCap - 16)) topk_merge<GM>(ts, ti, thr, ncand, cbuf);
 #pragma unroll
-              for (int e = 16 * hh; e < 16 * hh + 16; ++e) {  // (branch-free: a miss writes the junk slot)
+              for (int e = 16 * hh; e < 16 * hh + 16; ++e) {  // (predicated: only hits reach shared memory)
                 const float y = v[e];
                 const bool hit = y > thr;
-                cbuf[hit ? ncand : kCandCap] = make_float2(y, __int_as_float(id0 + e));
+                sts_f2_if(cbuf + ncand, y, __int_as_float(id0 + e), hit);
                 ncand += hit ? 1 : 0;
               }
             }
@@ -642,7 +652,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     const float m = ml.x;
     float l = ml.y;
     if (ml.x == -INFINITY && ml.y == 0.f && gt + st_ < ntile) alive = false;  // the softmax gave up
-    if (alive && ntile > 0) alive = __all_sync(0xffffffffu, wait(o_done, (uint32_t)(ntile - 1) & 1u));
+    if (alive && ntile > 0)
+      alive = __all_sync(0xffffffffu, wait(&o_done[(ntile - 1) & 1], (uint32_t)((ntile - 1) >> 1) & 1u));
     tc::fence_after_sync();
     const int64_t wr = ((int64_t)b * a.Hq + hq) * a.NW + (pi - a.w_lo);  // wave row
     const int64_t orow = ((int64_t)b * a.Hq + hq) * a.Tq + pi;
