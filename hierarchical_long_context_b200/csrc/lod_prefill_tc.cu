@@ -139,6 +139,20 @@ __device__ __forceinline__ void topk_insert_ranked(float (&s)[GM], int (&ix)[GM]
   }
 }
 
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane, without
+// waiting (tmem_st_wait() before an MMA or another thread reads them).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Wait until this thread's earlier TMEM stores have completed.
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Store (x, y) to shared memory at p when c holds (a predicated store: a
 // miss costs an issue slot but no shared-memory bandwidth).
 __device__ __forceinline__ void sts_f2_if(float2* p, float x, float y, bool c) {
@@ -538,7 +552,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) pw[4 * q + e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
           }
-          tc::tmem_st16(tmem + tl + kColP + 64 * (uint32_t)st + 16 * c, pw);
+          tmem_st16(tmem + tl + kColP + 64 * (uint32_t)st + 16 * c, pw);
         }
         if (!bail) break;
         redo = true;
@@ -548,7 +562,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[st]);
       l += (la[0] + la[1]) + (la[2] + la[3]);
-      tc::tmem_st_wait();
+      tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[st]);

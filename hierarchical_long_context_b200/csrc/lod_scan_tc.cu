@@ -51,7 +51,6 @@ constexpr int D = 128;
 constexpr int N = 16;            // MMA N: the unit's query rows (<= 8), zero padded
 constexpr int TROWS = 128;       // rows per tile: MMA 1's M, MMA 2's K
 constexpr int kStages = 3;
-constexpr int kFirstTiles = 2;   // ring slots filled during the set-up
 constexpr int kThreads = 320;    // warp 0 copies, warp 1 issues MMAs, warps 2-5 softmax, 6-9 selection
 constexpr int kSoftThreads = 128;
 constexpr int kBarSoft = 1;      // named barrier of the softmax warps
@@ -297,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- the first ring stages (warp 0) and the query operand (softmax warps)
   if (warp == 0) {
     __syncwarp();
-    for (int i = 0; i < kFirstTiles && i < ntile; ++i) issue_tile(i);
+    for (int i = 0; i < kStages && i < ntile; ++i) issue_tile(i);
   }
   if (warp >= 2 && warp < 6) {
     const int t = tid - 64;
@@ -331,12 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    int issued = ntile < kFirstTiles ? ntile : kFirstTiles;  // issued during the set-up
-    for (int i = kFirstTiles; i < ntile; ++i) {
-      // a slot left free at set-up is filled once the first tile has landed
-      // (so every CTA's first tile is ahead of the later ones in DRAM)
-      const bool ok = i < kStages ? wait(&full[0], 0u) : wait(&empty[i % kStages], (uint32_t)(i / kStages - 1) & 1u);
-      if (!ok) break;
+    int issued = ntile < kStages ? ntile : kStages;  // issued during the set-up
+    for (int i = kStages; i < ntile; ++i) {
+      if (!wait(&empty[i % kStages], (uint32_t)(i / kStages - 1) & 1u)) break;
       issue_tile(i);
       ++issued;
     }
